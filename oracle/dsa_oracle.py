@@ -1,0 +1,296 @@
+"""Plain CPU oracle for the DSA lightning indexer — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product path (the CUDA library and
+its Python binding) never calls it, and it shares no code with that path.
+
+Everything here is slow and direct: float64 numpy, a full stable sort per
+query row, no tiling and no fusion.  It follows the pages as follows.
+
+* Score.  The pages say the DeepSeek Sparse Attention (DSA) "lightning
+  indexer" scores every key of the causal prefix for every query and keeps the
+  top k = 2048 (MLI page, section "Core Idea"; PIVOT abstract; IndexCache page,
+  section "The Quadratic Tax"), but none of them prints the score itself.  This
+  library takes the standard DSA indexer form
+
+      I[t, s] = sum_h w[t, h] * ReLU( q[t, h, :] . k[s, :] )
+
+  with no extra scale factor.  For fp8 keys with a per-token scale, the key
+  is k[s, :] = decode_e4m3(bytes[s, :]) * scale[s].
+* Causality.  Query row t sits at key position p = q_pos0 + t and sees keys
+  0..p (AttentionIndex page, "Key findings": each query only sees its own
+  prefix).
+* Top-k.  Keys are ranked by (score descending, key index ascending) with one
+  full stable sort; the first min(k, p + 1) are kept.  Rows that see fewer than
+  k keys return all of them, padded with index -1 and score -inf.
+* Group-shared form (PIVOT abstract): fixed-size groups of consecutive
+  queries; the proxy is the mean of the members' q and w; one full-prefix scan
+  by the proxy over the prefix of the group's last member gives a candidate
+  bank of the best B keys; Refine re-scores the bank with each member's own
+  q, w and takes its own top-k; Reuse gives each member the proxy's ranking
+  over the bank, restricted to keys the member may see, cut to k.
+* Decode (PIVOT abstract, MLI "Core Idea"): sequence b holds N_b cached keys
+  and m_b new queries; new query j sits at position N_b - m_b + j.
+
+Pins: every function here is checked in ``tests/test_oracle.py`` against
+hand-worked values (``tests/golden/``), the fp8 format's published value
+table, brute-force enumeration of subsets, closed forms and invariants.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "decode_e4m3", "key_values", "score_rows", "select_topk", "dense",
+    "proxy", "group", "decode", "REFINE", "REUSE",
+]
+
+REFINE = 0
+REUSE = 1
+
+
+# ----------------------------------------------------------------------------
+# small steps (kept separate so that each can be checked on its own)
+# ----------------------------------------------------------------------------
+def _relu(x):
+    """max(0, x) elementwise."""
+    return np.maximum(x, 0.0)
+
+
+def _n_visible(p):
+    """A query at position p sees keys 0..p: p + 1 keys."""
+    return p + 1
+
+
+def _rank_order(scores, idx):
+    """Order by score descending, then key index ascending (full stable sort)."""
+    return np.lexsort((idx, -scores))
+
+
+def decode_e4m3(b):
+    """Decode OCP FP8 E4M3 bytes to float64.
+
+    Layout: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits.  Exponent
+    field 0 encodes subnormals m * 2^-9; otherwise (1 + m/8) * 2^(e - 7).
+    S.1111.111 is NaN; there are no infinities, so the largest finite value is
+    S.1111.110 = 448.
+    """
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = b & 0x7
+    sub = m.astype(np.float64) * 2.0 ** -9
+    nrm = (1.0 + m / 8.0) * np.power(2.0, e - 7.0)
+    v = sign * np.where(e == 0, sub, nrm)
+    v = np.where((b & 0x7F) == 0x7F, np.nan, v)
+    return v
+
+
+def key_values(K, k_scale=None):
+    """Keys as float64 [N, d]: fp8 bytes are decoded and times their token's scale."""
+    K = np.asarray(K)
+    if K.dtype == np.uint8:
+        assert k_scale is not None, "fp8 keys need a per-token scale"
+        s = np.asarray(k_scale, dtype=np.float64)
+        return decode_e4m3(K) * s[:, None]
+    assert k_scale is None
+    return K.astype(np.float64)
+
+
+def score_rows(q_rows, w_rows, Kd):
+    """I[r, s] = sum_h w[r, h] * ReLU(q[r, h, :] . Kd[s, :]) for every row r, key s.
+
+    q_rows [R, H, d], w_rows [R, H], Kd [S, d] (float64).  No causal cut here.
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    w_rows = np.asarray(w_rows, dtype=np.float64)
+    R, H, d = q_rows.shape
+    dots = (q_rows.reshape(R * H, d) @ Kd.T).reshape(R, H, Kd.shape[0])
+    return np.einsum("rh,rhs->rs", w_rows, _relu(dots))
+
+
+def select_topk(scores, k, idx=None):
+    """First min(k, n) entries of the (score desc, index asc) order.
+
+    ``scores`` [n]; ``idx`` [n] key indices (default 0..n-1).  Returns
+    (indices int64, scores float64) in rank order.
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    idx = np.arange(scores.shape[0], dtype=np.int64) if idx is None else np.asarray(idx, np.int64)
+    order = _rank_order(scores, idx)[:min(k, scores.shape[0])]
+    return idx[order], scores[order]
+
+
+def _pad(sel_idx, sel_val, k):
+    oi = np.full(k, -1, dtype=np.int64)
+    ov = np.full(k, -np.inf, dtype=np.float64)
+    oi[:sel_idx.shape[0]] = sel_idx
+    ov[:sel_val.shape[0]] = sel_val
+    return oi, ov
+
+
+def _row_chunks(rows, H, span, budget=1 << 27):
+    step = max(1, budget // max(1, H * span * 8))
+    for i in range(0, len(rows), step):
+        yield rows[i:i + step]
+
+
+def dense(q, w, K, k, q_pos0=0, k_scale=None, rows=None, return_scores=False):
+    """Dense indexer: per query row its top-k over keys 0..q_pos0+t.
+
+    Returns dict with ``idx`` [R, k] int64 (-1 padded), ``val`` [R, k] float64
+    (-inf padded), ``count`` [R], ``rows``; with ``return_scores`` also
+    ``scores``: list of the full prefix score vectors (for parity checks).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Kd = key_values(K, k_scale)
+    T, H, _ = q.shape
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    out_i = np.full((R, k), -1, dtype=np.int64)
+    out_v = np.full((R, k), -np.inf, dtype=np.float64)
+    cnt = np.zeros(R, dtype=np.int64)
+    full = [None] * R
+    pos = {int(r): j for j, r in enumerate(rows)}
+    order = np.argsort(rows)
+    srows = rows[order]
+    span = int(q_pos0 + srows.max() + 1) if R else 0
+    for ch in _row_chunks(srows, H, span):
+        nvis_max = _n_visible(int(q_pos0 + ch.max()))
+        S = score_rows(q[ch], w[ch], Kd[:nvis_max])
+        for j, r in enumerate(ch):
+            nv = _n_visible(int(q_pos0 + r))
+            row = S[j, :nv]
+            si, sv = select_topk(row, k)
+            o = pos[int(r)]
+            out_i[o], out_v[o] = _pad(si, sv, k)
+            cnt[o] = si.shape[0]
+            if return_scores:
+                full[o] = row.copy()
+    res = {"idx": out_i, "val": out_v, "count": cnt, "rows": rows}
+    if return_scores:
+        res["scores"] = full
+    return res
+
+
+def proxy(q, w, G):
+    """PIVOT proxy per group of G consecutive rows: the members' mean q and mean w.
+
+    A last group with fewer than G rows averages over its actual members.
+    Returns (qbar [ng, H, d], wbar [ng, H]) in float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    T = q.shape[0]
+    ng = (T + G - 1) // G
+    qb = np.stack([q[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
+    wb = np.stack([w[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
+    return qb, wb
+
+
+def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=None,
+          groups=None, members=None, bank_override=None):
+    """PIVOT group-shared indexer (Refine or Reuse).
+
+    For group g (rows gG..min(T,(g+1)G)-1) with last member position L_g:
+      1. proxy scores over keys 0..L_g with (qbar[g], wbar[g]);
+      2. bank = first min(bank, L_g + 1) keys of the proxy's (score desc,
+         index asc) order;
+      3. Refine: member t scores bank keys <= p_t with its own q, w and keeps
+         its top-k; Reuse: member t keeps the first k bank entries (in the
+         proxy's order) with key <= p_t, valued by the proxy score.
+
+    ``qbar``/``wbar`` default to ``proxy(q, w, G)``; a caller may pass the
+    proxy exactly as another implementation rounded it.  ``groups`` restricts
+    the work to some groups; ``members`` (list of row indices) to some rows.
+    ``bank_override`` {g: bank index array in proxy order} replaces step 1-2.
+    Returns dict with ``bank_idx``/``bank_val`` {g: arrays in proxy order},
+    ``bank_scores`` {g: full proxy score vector}, and ``idx``/``val``/``count``
+    {row: padded arrays}, plus ``member_scores`` {row: full member score vector
+    over keys 0..p_t} for Refine.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Kd = key_values(K, k_scale)
+    T = q.shape[0]
+    ng = (T + G - 1) // G
+    if qbar is None or wbar is None:
+        qb, wb = proxy(q, w, G)
+        qbar = qb if qbar is None else qbar
+        wbar = wb if wbar is None else wbar
+    qbar = np.asarray(qbar, dtype=np.float64)
+    wbar = np.asarray(wbar, dtype=np.float64)
+    if groups is None:
+        groups = range(ng)
+    mem_set = None if members is None else set(int(m) for m in members)
+    res = {"bank_idx": {}, "bank_val": {}, "bank_scores": {}, "idx": {}, "val": {},
+           "count": {}, "member_scores": {}}
+    for g in groups:
+        r0, r1 = g * G, min(T, (g + 1) * G)
+        L = q_pos0 + r1 - 1
+        nv = _n_visible(L)
+        ps = score_rows(qbar[g:g + 1], wbar[g:g + 1], Kd[:nv])[0]
+        res["bank_scores"][g] = ps
+        if bank_override is not None and g in bank_override:
+            b_idx = np.asarray(bank_override[g], dtype=np.int64)
+            b_val = ps[b_idx]
+        else:
+            b_idx, b_val = select_topk(ps, bank)
+        res["bank_idx"][g], res["bank_val"][g] = b_idx, b_val
+        rows = [r for r in range(r0, r1) if mem_set is None or r in mem_set]
+        for r in rows:
+            p = q_pos0 + r
+            keep = b_idx <= p
+            if mode == REFINE:
+                ms = score_rows(q[r:r + 1], w[r:r + 1], Kd[:_n_visible(p)])[0]
+                res["member_scores"][r] = ms
+                si, sv = select_topk(ms[b_idx[keep]], k, idx=b_idx[keep])
+            elif mode == REUSE:
+                si, sv = b_idx[keep][:k], b_val[keep][:k]
+            else:
+                raise ValueError(mode)
+            res["idx"][r], res["val"][r] = _pad(si, sv, k)
+            res["count"][r] = si.shape[0]
+    return res
+
+
+def decode(q, w, K, k_offsets, q_offsets, k, k_scale=None, return_scores=False):
+    """Decode indexer over a batch of key caches.
+
+    Sequence b owns keys K[k_offsets[b]:k_offsets[b+1]] (N_b of them, indexed
+    0..N_b-1 within the sequence) and query rows q_offsets[b]..q_offsets[b+1]-1
+    (m_b of them); new query j sits at position N_b - m_b + j and sees keys
+    0..N_b - m_b + j.  Returns idx/val [sum m_b, k] with indices local to the
+    sequence.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    ko = np.asarray(k_offsets, dtype=np.int64)
+    qo = np.asarray(q_offsets, dtype=np.int64)
+    B = ko.shape[0] - 1
+    M = int(qo[-1])
+    out_i = np.full((M, k), -1, dtype=np.int64)
+    out_v = np.full((M, k), -np.inf, dtype=np.float64)
+    cnt = np.zeros(M, dtype=np.int64)
+    scores = [None] * M
+    Kall = np.asarray(K)
+    sc = None if k_scale is None else np.asarray(k_scale)
+    for b in range(B):
+        k0, k1 = int(ko[b]), int(ko[b + 1])
+        Nb = k1 - k0
+        mb = int(qo[b + 1] - qo[b])
+        Kd = key_values(Kall[k0:k1], None if sc is None else sc[k0:k1])
+        for j in range(mb):
+            r = int(qo[b]) + j
+            p = Nb - mb + j
+            S = score_rows(q[r:r + 1], w[r:r + 1], Kd[:_n_visible(p)])[0]
+            si, sv = select_topk(S, k)
+            out_i[r], out_v[r] = _pad(si, sv, k)
+            cnt[r] = si.shape[0]
+            if return_scores:
+                scores[r] = S
+    res = {"idx": out_i, "val": out_v, "count": cnt}
+    if return_scores:
+        res["scores"] = scores
+    return res

@@ -1,0 +1,399 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each ``pin_*`` function checks the oracle against something other than
+itself: values worked by hand (``tests/golden``), the fp8 format's published
+value table, brute-force enumeration of subsets, library routines on special
+cases, closed-form identities and invariants.  ``test_mutants_are_caught``
+plants plausible mistakes in the oracle (on the CPU) and requires that some pin
+fails for each.
+"""
+import contextlib
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _nan_to_neginf(a):
+    return np.array([[-np.inf if v is None else v for v in r] for r in a], dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# pins (each raises AssertionError on a mismatch)
+# ---------------------------------------------------------------------------
+def pin_e4m3_table(O):
+    g = _load("e4m3_values.json")
+    for hx, v in g["values"].items():
+        got = O.decode_e4m3(np.array([int(hx, 16)], dtype=np.uint8))[0]
+        assert got == v and math.copysign(1, got) == math.copysign(1, v), (hx, got, v)
+    for hx in g["nan"]:
+        assert np.isnan(O.decode_e4m3(np.array([int(hx, 16)], dtype=np.uint8))[0])
+
+
+def pin_e4m3_library(O):
+    allb = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(allb).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.decode_e4m3(allb)
+    fin = ~np.isnan(lib)
+    assert np.array_equal(np.isnan(got), ~fin)
+    assert np.array_equal(got[fin], lib[fin])
+
+
+def pin_dense_hand(O):
+    g = _load("dense_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k"], float)
+    S = O.score_rows(q, w, K)
+    for t, row in enumerate(g["scores"]):
+        for s, v in enumerate(row):
+            if v is not None:
+                assert S[t, s] == v, (t, s, S[t, s], v)
+    for kk, exp in g["topk"].items():
+        r = O.dense(q, w, K, int(kk), q_pos0=g["q_pos0"])
+        assert np.array_equal(r["idx"], np.array(exp["idx"])), (kk, r["idx"], exp["idx"])
+        assert np.array_equal(r["val"], _nan_to_neginf(exp["val"])), (kk, r["val"])
+
+
+def pin_ties_hand(O):
+    g = _load("ties_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k"], float)
+    for kk, exp in g["topk"].items():
+        r = O.dense(q, w, K, int(kk), q_pos0=g["q_pos0"])
+        assert np.array_equal(r["idx"], np.array(exp["idx"])), (kk, r["idx"])
+
+
+def pin_relu_zero_hand(O):
+    g = _load("relu_zero_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k"], float)
+    S = O.score_rows(q, w, K)
+    assert np.array_equal(S, np.array(g["scores"], float)), S
+    assert not np.signbit(S[0]).any()   # exact +0, not a residue or -0
+
+
+def pin_group_hand(O):
+    g = _load("group_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k"], float)
+    qb, wb = O.proxy(q, w, g["G"])
+    assert np.array_equal(qb, np.array(g["proxy_q"], float)) and np.array_equal(wb, np.array(g["proxy_w"], float))
+    for c in g["cases"]:
+        for mode, key in ((O.REFINE, "refine"), (O.REUSE, "reuse")):
+            r = O.group(q, w, K, c["k"], g["G"], c["bank"], mode, q_pos0=g["q_pos0"])
+            assert list(r["bank_idx"][0]) == c["bank_idx"], (c, r["bank_idx"])
+            assert list(r["bank_val"][0]) == c["bank_val"]
+            for m in range(2):
+                assert list(r["idx"][m]) == c[key + "_idx"][m], (key, c, m, r["idx"][m])
+                assert list(r["val"][m]) == c[key + "_val"][m], (key, c, m, r["val"][m])
+
+
+def pin_decode_hand(O):
+    g = _load("decode_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["keys"], float)
+    r = O.decode(q, w, K, g["k_offsets"], g["q_offsets"], g["k"])
+    assert np.array_equal(r["idx"], np.array(g["idx"])), r["idx"]
+    assert np.array_equal(r["val"], _nan_to_neginf(g["val"])), r["val"]
+
+
+def _rand_case(seed, T=6, N=9, H=3, d=5, q_pos0=3):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H, d))
+    w = rng.uniform(0, 1, (T, H))
+    K = rng.standard_normal((N, d))
+    return q, w, K, q_pos0
+
+
+def pin_single_head_matmul(O):
+    # one head, w = 1, non-negative q and k: every dot is >= 0 so the score is the
+    # plain matrix product (library matmul)
+    rng = np.random.default_rng(1)
+    q = rng.uniform(0, 1, (7, 1, 6))
+    K = rng.uniform(0, 1, (11, 6))
+    S = O.score_rows(q, np.ones((7, 1)), K)
+    assert np.allclose(S, np.matmul(q[:, 0, :], K.T), rtol=1e-14, atol=0)
+
+
+def pin_relu_odd_identity(O):
+    # ReLU(x) - ReLU(-x) = x, so for one head S(q) - S(-q) = w * (q . k)
+    q, w, K, _ = _rand_case(2, H=1)
+    d = O.score_rows(q, w, K) - O.score_rows(-q, w, K)
+    assert np.allclose(d, w[:, :1] * np.matmul(q[:, 0, :], K.T), rtol=1e-12, atol=1e-14)
+
+
+def pin_head_structure(O):
+    # heads add up (split H into two parts), weights scale linearly, and a
+    # permutation of heads (with their weights) changes nothing
+    q, w, K, _ = _rand_case(3, H=4)
+    S = O.score_rows(q, w, K)
+    S_a = O.score_rows(q[:, :2], w[:, :2], K)
+    S_b = O.score_rows(q[:, 2:], w[:, 2:], K)
+    assert np.allclose(S, S_a + S_b, rtol=1e-13, atol=1e-15)
+    assert np.allclose(O.score_rows(q, 2.5 * w, K), 2.5 * S, rtol=1e-13)
+    perm = [2, 0, 3, 1]
+    assert np.allclose(O.score_rows(q[:, perm], w[:, perm], K), S, rtol=1e-13)
+    # positive scale of q passes through ReLU
+    assert np.allclose(O.score_rows(3.0 * q, w, K), 3.0 * S, rtol=1e-13)
+    # row / key correspondence: swapping two keys swaps two score columns
+    K2 = K.copy()
+    K2[[1, 4]] = K2[[4, 1]]
+    S2 = O.score_rows(q, w, K2)
+    assert np.allclose(S2[:, [4, 1]], S[:, [1, 4]], rtol=1e-13)
+
+
+def pin_fp8_keys_scale(O):
+    # per-token scale > 0 passes through ReLU: scores with scaled fp8 keys equal
+    # scale[s] times the scores with the decoded bytes
+    rng = np.random.default_rng(4)
+    b = rng.integers(0, 256, (10, 4), dtype=np.uint8)
+    b[(b & 0x7F) == 0x7F] = 0x38          # no NaN codes
+    s = rng.uniform(0.5, 2.0, 10)
+    q = rng.standard_normal((3, 2, 4))
+    w = rng.uniform(0, 1, (3, 2))
+    S = O.score_rows(q, w, O.key_values(b, s))
+    S0 = O.score_rows(q, w, O.decode_e4m3(b))
+    assert np.allclose(S, S0 * s[None, :], rtol=1e-13, atol=1e-300)
+
+
+def _brute_topk(scores, k):
+    """Max-sum k-subset; among equal sums the lexicographically smallest sorted index tuple."""
+    n = len(scores)
+    best = None
+    for comb in itertools.combinations(range(n), min(k, n)):
+        key = (-sum(scores[i] for i in comb), comb)
+        if best is None or key < best:
+            best = key
+    return sorted(best[1])
+
+
+def pin_topk_bruteforce(O):
+    rng = np.random.default_rng(5)
+    for trial in range(60):
+        n = int(rng.integers(1, 12))
+        k = int(rng.integers(1, 4))
+        sc = rng.integers(-3, 4, n).astype(np.float64)   # many exact ties
+        si, _ = O.select_topk(sc, k)
+        assert sorted(si.tolist()) == _brute_topk(list(sc), k), (sc, k, si)
+    # exhaustive: every row of a small causal problem, k <= 3, N <= 64
+    q, w, K, q0 = _rand_case(6, T=8, N=64, H=2, d=3, q_pos0=56)
+    K[10] = K[3]                                       # duplicate key -> exact tie
+    for k in (1, 2, 3):
+        r = O.dense(q, w, K, k, q_pos0=q0, return_scores=True)
+        for t in range(8):
+            row = r["scores"][t]
+            assert len(row) == q0 + t + 1
+            exp = _brute_topk(list(row), k)
+            assert sorted(r["idx"][t][:r["count"][t]].tolist()) == exp
+
+
+def pin_causality(O):
+    q, w, K, _ = _rand_case(7, T=12, N=12, q_pos0=0)
+    k = 5
+    r = O.dense(q, w, K, k, q_pos0=0)
+    for t in range(12):
+        sel = r["idx"][t][r["idx"][t] >= 0]
+        assert (sel <= t).all()
+        if t + 1 < k:
+            assert sorted(sel.tolist()) == list(range(t + 1))
+            assert (r["idx"][t][t + 1:] == -1).all() and np.isneginf(r["val"][t][t + 1:]).all()
+        else:
+            assert len(sel) == k
+    # a key beyond a query's position never changes that query's result
+    K2 = K.copy()
+    K2[11] = 100.0 * np.abs(K2[11])
+    r2 = O.dense(q, w, K2, k, q_pos0=0)
+    assert np.array_equal(r["idx"][:11], r2["idx"][:11])
+
+
+def pin_group_invariants(O):
+    q, w, K, _ = _rand_case(8, T=12, N=20, H=3, d=4, q_pos0=8)
+    q0, k, G = 8, 4, 4
+    dn = O.dense(q, w, K, k, q_pos0=q0)
+    # Refine with a bank covering the whole prefix is dense selection
+    rf = O.group(q, w, K, k, G, 64, O.REFINE, q_pos0=q0)
+    for t in range(12):
+        assert np.array_equal(rf["idx"][t], dn["idx"][t])
+    # G = 1: the proxy is the query itself, so Reuse == Refine == dense
+    for mode in (O.REFINE, O.REUSE):
+        r1 = O.group(q, w, K, k, 1, 6, mode, q_pos0=q0)
+        for t in range(12):
+            assert np.array_equal(r1["idx"][t], dn["idx"][t]), (mode, t)
+    # Reuse: the last member of a group gets exactly the proxy's top-k
+    ru = O.group(q, w, K, k, G, 7, O.REUSE, q_pos0=q0)
+    for g in range(3):
+        last = g * G + G - 1
+        ps = ru["bank_scores"][g]
+        pi, _ = O.select_topk(ps, k)
+        assert sorted(ru["idx"][last].tolist()) == sorted(pi.tolist())
+        # every member only receives keys it may see
+        for t in range(g * G, g * G + G):
+            sel = ru["idx"][t][ru["idx"][t] >= 0]
+            assert (sel <= q0 + t).all()
+    # the proxy of identical rows is the row; the proxy of two rows is their midpoint
+    qq = np.repeat(q[:1], 4, axis=0)
+    ww = np.repeat(w[:1], 4, axis=0)
+    qb, wb = O.proxy(qq, ww, 4)
+    assert np.allclose(qb[0], q[0], rtol=1e-15) and np.allclose(wb[0], w[0], rtol=1e-15)
+    qb, wb = O.proxy(q[:2], w[:2], 2)
+    assert np.allclose(qb[0], 0.5 * (q[0] + q[1]), rtol=1e-15)
+    assert np.allclose(wb[0], 0.5 * (w[0] + w[1]), rtol=1e-15)
+    # partial last group averages over its actual members
+    qb, _ = O.proxy(q[:5], w[:5], 4)
+    assert qb.shape[0] == 2 and np.allclose(qb[1], q[4], rtol=1e-15)
+
+
+def pin_decode_matches_dense(O):
+    # a decode batch equals dense prefill on each sequence restricted to its
+    # last m_b query positions
+    rng = np.random.default_rng(9)
+    lengths, ms = [7, 1, 12], [2, 1, 3]
+    H, d, k = 2, 3, 4
+    Ks = [rng.standard_normal((n, d)) for n in lengths]
+    qs = [rng.standard_normal((m, H, d)) for m in ms]
+    ws = [rng.uniform(0, 1, (m, H)) for m in ms]
+    ko = np.concatenate([[0], np.cumsum(lengths)])
+    qo = np.concatenate([[0], np.cumsum(ms)])
+    r = O.decode(np.concatenate(qs), np.concatenate(ws), np.concatenate(Ks), ko, qo, k)
+    for b in range(3):
+        dn = O.dense(qs[b], ws[b], Ks[b], k, q_pos0=lengths[b] - ms[b])
+        assert np.array_equal(r["idx"][qo[b]:qo[b + 1]], dn["idx"]), b
+
+
+PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
+        pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
+        pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
+        pin_topk_bruteforce, pin_causality, pin_group_invariants,
+        pin_decode_matches_dense]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin(pin):
+    pin(O)
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must be caught by at least one pin
+# ---------------------------------------------------------------------------
+def _m_no_relu(mp):
+    mp.setattr(O, "_relu", lambda x: x)
+
+
+def _m_abs_relu(mp):
+    mp.setattr(O, "_relu", lambda x: np.abs(x))
+
+
+def _m_causal_exclusive(mp):
+    mp.setattr(O, "_n_visible", lambda p: p)
+
+
+def _m_causal_plus_one(mp):
+    mp.setattr(O, "_n_visible", lambda p: p + 2)
+
+
+def _m_tiebreak_high(mp):
+    mp.setattr(O, "_rank_order", lambda s, i: np.lexsort((-i, -s)))
+
+
+def _m_ascending(mp):
+    mp.setattr(O, "_rank_order", lambda s, i: np.lexsort((i, s)))
+
+
+def _m_e4m3_bias8(mp):
+    real = O.decode_e4m3
+
+    def bad(b):
+        return real(b) * 0.5
+    mp.setattr(O, "decode_e4m3", bad)
+
+
+def _m_e4m3_no_subnormal(mp):
+    real = O.decode_e4m3
+
+    def bad(b):
+        v = real(b)
+        e = (np.asarray(b).astype(np.int64) >> 3) & 0xF
+        return np.where(e == 0, 0.0, v)
+    mp.setattr(O, "decode_e4m3", bad)
+
+
+def _m_weight_outside(mp):
+    def bad(qr, wr, Kd):
+        R, H, d = qr.shape
+        dots = (qr.reshape(R * H, d) @ Kd.T).reshape(R, H, -1)
+        return O._relu(np.einsum("rh,rhs->rs", wr, dots))
+    mp.setattr(O, "score_rows", bad)
+
+
+def _m_transposed_weight(mp):
+    def bad(qr, wr, Kd):
+        R, H, d = qr.shape
+        dots = (qr.reshape(R * H, d) @ Kd.T).reshape(R, H, -1)
+        wt = wr[:, ::-1]
+        return np.einsum("rh,rhs->rs", wt, O._relu(dots))
+    mp.setattr(O, "score_rows", bad)
+
+
+def _m_head_mean(mp):
+    real = O.score_rows
+    mp.setattr(O, "score_rows", lambda qr, wr, Kd: real(qr, wr, Kd) / qr.shape[1])
+
+
+def _m_proxy_sum(mp):
+    def bad(q, w, G):
+        T = q.shape[0]
+        ng = (T + G - 1) // G
+        return (np.stack([q[g * G:(g + 1) * G].sum(0) for g in range(ng)]),
+                np.stack([w[g * G:(g + 1) * G].sum(0) for g in range(ng)]))
+    mp.setattr(O, "proxy", bad)
+
+
+def _m_proxy_first_member(mp):
+    def bad(q, w, G):
+        T = q.shape[0]
+        ng = (T + G - 1) // G
+        return (np.stack([q[g * G] for g in range(ng)]), np.stack([w[g * G] for g in range(ng)]))
+    mp.setattr(O, "proxy", bad)
+
+
+def _m_decode_first_positions(mp):
+    # decode queries placed at the first m positions instead of the last m
+    real_dense = O.dense
+
+    def bad(q, w, K, k_offsets, q_offsets, k, k_scale=None, return_scores=False):
+        ko = np.asarray(k_offsets)
+        qo = np.asarray(q_offsets)
+        outs_i, outs_v = [], []
+        for b in range(len(ko) - 1):
+            r = real_dense(q[qo[b]:qo[b + 1]], w[qo[b]:qo[b + 1]], K[ko[b]:ko[b + 1]], k, q_pos0=0)
+            outs_i.append(r["idx"])
+            outs_v.append(r["val"])
+        return {"idx": np.concatenate(outs_i), "val": np.concatenate(outs_v)}
+    mp.setattr(O, "decode", bad)
+
+
+MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
+           _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
+           _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
+           _m_proxy_first_member, _m_decode_first_positions]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
+def test_mutants_are_caught(mutant):
+    caught = []
+    for pin in PINS:
+        with pytest.MonkeyPatch.context() as mp:
+            mutant(mp)
+            try:
+                pin(O)
+            except (AssertionError, ValueError, IndexError):
+                caught.append(pin.__name__)
+    assert caught, f"no pin catches {mutant.__name__}"
