@@ -1,0 +1,174 @@
+/*
+ * dsa_index.h — C ABI of the B200 (sm_100a) lightning-indexer library.
+ *
+ * The DeepSeek Sparse Attention (DSA) lightning indexer selects, for every
+ * query, the k keys of its causal prefix that sparse attention will read.
+ * In the pages this library follows, the indexer has to score each key that
+ * precedes a query and it retains the k = 2048 best positions (PIVOT:
+ * Efficient Query-Group Indexing for Token-Level Sparse Attention — Abstract;
+ * MLI Restructures DeepSeek Sparse Attention — Core Idea); the pages do not
+ * print the score itself.
+ * This library uses the standard DSA indexer score
+ *
+ *     I[t, s] = sum_h  w[t, h] * ReLU( q[t, h, :] . k[s, :] )
+ *
+ * with fp32 accumulation, no extra scale, and (fp8 keys) k[s, :] =
+ * e4m3(bytes[s, :]) * K_scale[s].  Query row t sits at key position
+ * p_t = q_pos0 + t and sees keys 0..p_t (causal prefix; AttentionIndex
+ * Architecture — Key findings: causality is a hard constraint).
+ *
+ * Selection: the k largest I[t, s] over s <= p_t, ties broken toward the
+ * lower key index.  Each output row is a SET: its min(k, p_t + 1) entries
+ * (index, score) come in no particular order; the remaining slots hold
+ * index -1 and score -inf.
+ *
+ * Conventions for every call below
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     row-major and contiguous, 16-byte aligned.  Offsets arrays of the decode
+ *     call are device pointers too.
+ *   - The caller owns every buffer, including `workspace`; the library never
+ *     allocates, never frees and never synchronises `stream` (a cudaStream_t;
+ *     NULL is the legacy default stream).  Calls are asynchronous.
+ *   - Size the workspace with the matching *_workspace_size call; its first
+ *     bytes hold a device status word that kernels set on a device-side
+ *     failure (a bounded wait that gave up); read it with dsa_check_status.
+ *   - Return value: DSA_OK or a negative DSA_ERR_* code; on an error nothing
+ *     has been launched.
+ *   - Supported shapes: bf16 Q/K with H = 64, d = 128 run on the tcgen05
+ *     tensor-core kernel; fp32 Q/K (any H <= 128, d <= 256, H*d <= 8192) and
+ *     other bf16 / fp8-key shapes run on an exact fp32 CUDA-core kernel.
+ *   - Inputs must be finite.
+ */
+#ifndef DSA_INDEX_H
+#define DSA_INDEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define DSA_DTYPE_BF16 0
+#define DSA_DTYPE_FP32 1
+#define DSA_DTYPE_FP8_E4M3 2 /* keys only; needs K_scale */
+
+/* status codes */
+#define DSA_OK 0
+#define DSA_ERR_INVALID_ARG (-1) /* null pointer, bad size, misaligned pointer */
+#define DSA_ERR_UNSUPPORTED (-2) /* valid but not implemented shape / dtype */
+#define DSA_ERR_WORKSPACE (-3)   /* workspace too small */
+#define DSA_ERR_CUDA (-4)        /* a CUDA runtime call or launch failed */
+#define DSA_ERR_TIMEOUT (-5)     /* a device-side bounded wait gave up */
+#define DSA_ERR_DEVICE (-6)      /* current device is not sm_100 */
+#define DSA_ERR_INTERNAL (-7)    /* a device-side consistency check failed */
+
+/* group modes (PIVOT abstract: the Refine and Reuse variants) */
+#define DSA_GROUP_REFINE 0
+#define DSA_GROUP_REUSE 1
+
+/* Human-readable text for a status code (static storage). */
+const char* dsa_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int dsa_version(void);
+
+/* Synchronises `stream`, then reads and clears the device status word kept
+ * in `workspace`.  Returns DSA_OK, the recorded DSA_ERR_TIMEOUT or
+ * DSA_ERR_INTERNAL, or DSA_ERR_CUDA if the stream reported an error. */
+int dsa_check_status(void* workspace, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dense prefill indexer.
+ *   Q   [T, H, d]  bf16 or fp32 (q_dtype)
+ *   w   [T, H]     fp32 head weights
+ *   K   [N, d]     bf16, fp32 or fp8 e4m3 bytes (k_dtype)
+ *   K_scale [N]    fp32 per-key scale (> 0), fp8 keys only, else NULL
+ *   q_pos0         key position of query row 0; needs 0 <= q_pos0 and
+ *                  q_pos0 + T <= N
+ *   k              keys kept per query, 1 <= k <= 65536
+ *   idx [T, k] int32, val [T, k] fp32 — outputs (see selection above)
+ * Cost: O(sum_t (p_t + 1) * H * d) multiply-adds; the [T, N] score matrix
+ * is never written to memory.
+ * ---------------------------------------------------------------------- */
+int dsa_index_dense_workspace_size(int T, int N, int H, int d, int k,
+                                   int q_dtype, int k_dtype, size_t* bytes);
+int dsa_index_dense(const void* Q, const float* w, const void* K,
+                    const float* K_scale, int T, int N, int H, int d,
+                    int64_t q_pos0, int k, int q_dtype, int k_dtype,
+                    int32_t* idx, float* val, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Group-shared prefill indexer (PIVOT abstract): the queries of a group are
+ * merged into one proxy query, one scan of the whole prefix by that proxy
+ * yields a candidate bank, and each query's top-k is then taken from the
+ * bank.
+ *   group  G >= 1: rows gG .. min(T,(g+1)G)-1 form group g; ng = ceil(T/G)
+ *   bank   B >= k: candidate-bank size of the proxy scan
+ *   mode   DSA_GROUP_REFINE: member t re-scores the bank keys <= p_t with
+ *          its own q, w and keeps its top-k.
+ *          DSA_GROUP_REUSE: member t keeps the first k bank keys <= p_t in
+ *          the proxy's ranking, valued by the proxy score.
+ *   Proxy: qbar[g] = mean of the members' q (fp32 mean, rounded to q_dtype),
+ *          wbar[g] = mean of the members' w (fp32).  The proxy scans keys
+ *          0..L_g, L_g = position of the group's last member.
+ *   bank_idx [ng, B] int32, bank_val [ng, B] fp32: optional outputs (NULL to
+ *          skip) — the bank in the proxy's ranking order (Reuse needs that
+ *          order; for Refine it is a set).  Unused slots: -1 / -inf.
+ *   proxy_q [ng, H, d] (q_dtype), proxy_w [ng, H] fp32: optional outputs.
+ * ---------------------------------------------------------------------- */
+int dsa_index_group_workspace_size(int T, int N, int H, int d, int k,
+                                   int group, int bank, int q_dtype,
+                                   int k_dtype, size_t* bytes);
+int dsa_index_group(const void* Q, const float* w, const void* K,
+                    const float* K_scale, int T, int N, int H, int d,
+                    int64_t q_pos0, int k, int group, int bank, int mode,
+                    int q_dtype, int k_dtype, int32_t* idx, float* val,
+                    int32_t* bank_idx, float* bank_val, void* proxy_q,
+                    float* proxy_w, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* ------------------------------------------------------------------------
+ * Decode indexer over a batch of key caches (ADIndex — Why the Indexer
+ * Becomes the Bottleneck: each decode query rescans the historical keys;
+ * PIVOT abstract: the queries of one multi-token-prediction step).
+ *   K [sum N_b, d]: sequence b owns rows k_offsets[b] .. k_offsets[b+1]-1
+ *   Q [sum m_b, H, d], w [sum m_b, H]: sequence b owns query rows
+ *          q_offsets[b] .. q_offsets[b+1]-1 (1 <= m_b <= min(4, N_b))
+ *   New query j of sequence b sits at position N_b - m_b + j and sees its
+ *   sequence's keys 0 .. N_b - m_b + j.  Output indices are local to the
+ *   sequence (0 .. N_b - 1).
+ *   k_offsets [B+1] int64, q_offsets [B+1] int32: DEVICE arrays.
+ *   total_keys: k_offsets[B] (host value: rows of K; tensor copies never
+ *          read beyond it).
+ *   max_keys: an upper bound on every N_b (host value; sizes the split of
+ *          each cache over the GPU's multiprocessors and the workspace).
+ * ---------------------------------------------------------------------- */
+int dsa_index_decode_workspace_size(int B, int total_q, int max_keys, int H,
+                                    int d, int k, int q_dtype, int k_dtype,
+                                    size_t* bytes);
+int dsa_index_decode(const void* Q, const float* w, const void* K,
+                     const float* K_scale, const int64_t* k_offsets,
+                     const int32_t* q_offsets, int B, int total_q,
+                     int64_t total_keys, int max_keys, int H, int d, int k,
+                     int q_dtype,
+                     int k_dtype, int32_t* idx, float* val, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Test aid: the full score matrix S [T, N] fp32 of the dense call (the same
+ * kernel and epilogue arithmetic; entries with s > p_t hold -inf).
+ * Needs T * N <= 2^26.  Uses the dense workspace.
+ * ---------------------------------------------------------------------- */
+int dsa_debug_scores(const void* Q, const float* w, const void* K,
+                     const float* K_scale, int T, int N, int H, int d,
+                     int64_t q_pos0, int q_dtype, int k_dtype, float* S,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEX_H */

@@ -7,10 +7,10 @@ its Python binding) never calls it, and it shares no code with that path.
 Everything here is slow and direct: float64 numpy, a full stable sort per
 query row, no tiling and no fusion.  It follows the pages as follows.
 
-* Score.  The pages say the DeepSeek Sparse Attention (DSA) "lightning
-  indexer" scores every key of the causal prefix for every query and keeps the
-  top k = 2048 (MLI page, section "Core Idea"; PIVOT abstract; IndexCache page,
-  section "The Quadratic Tax"), but none of them prints the score itself.  This
+* Score.  In the pages, the DeepSeek Sparse Attention (DSA) lightning
+  indexer scores every key of the causal prefix for every query and keeps the
+  top k = 2048 (MLI page, section Core Idea; PIVOT abstract; IndexCache page,
+  section The Quadratic Tax), but none of them prints the score itself.  This
   library takes the standard DSA indexer form
 
       I[t, s] = sum_h w[t, h] * ReLU( q[t, h, :] . k[s, :] )
@@ -18,8 +18,8 @@ query row, no tiling and no fusion.  It follows the pages as follows.
   with no extra scale factor.  For fp8 keys with a per-token scale, the key
   is k[s, :] = decode_e4m3(bytes[s, :]) * scale[s].
 * Causality.  Query row t sits at key position p = q_pos0 + t and sees keys
-  0..p (AttentionIndex page, "Key findings": each query only sees its own
-  prefix).
+  0..p (AttentionIndex page, Key findings: causality is enforced, a query
+  never uses keys beyond its own prefix).
 * Top-k.  Keys are ranked by (score descending, key index ascending) with one
   full stable sort; the first min(k, p + 1) are kept.  Rows that see fewer than
   k keys return all of them, padded with index -1 and score -inf.

@@ -1,0 +1,30 @@
+"""B200 (sm_100a) DSA lightning indexer: dense, group-shared (PIVOT) and decode.
+
+A thin Python binding over the C ABI in ``include/dsa_index.h``
+(``libdsa_index.so``, built in-tree by ``sparse_attention_token_index_b200.build``).
+The functions here only marshal arguments: torch provides device memory and
+the current CUDA stream; every step of the indexer runs in the library's
+CUDA kernels.  There is no CPU path: without the library or a CUDA device
+these functions raise.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    DSA_DTYPE_BF16,
+    DSA_DTYPE_FP32,
+    DSA_DTYPE_FP8_E4M3,
+    DSA_GROUP_REFINE,
+    DSA_GROUP_REUSE,
+    DsaError,
+    lib,
+    lib_path,
+    dsa_index_dense,
+    dsa_index_group,
+    dsa_index_decode,
+    dsa_debug_scores,
+    dsa_check_status,
+    dense_workspace_bytes,
+    group_workspace_bytes,
+    decode_workspace_bytes,
+    EXPORTED_SYMBOLS,
+)

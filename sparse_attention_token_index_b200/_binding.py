@@ -1,0 +1,259 @@
+"""ctypes binding of ``libdsa_index.so`` (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+DSA_DTYPE_BF16 = 0
+DSA_DTYPE_FP32 = 1
+DSA_DTYPE_FP8_E4M3 = 2
+DSA_GROUP_REFINE = 0
+DSA_GROUP_REUSE = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libdsa_index.so")
+
+EXPORTED_SYMBOLS = (
+    "dsa_status_string", "dsa_version", "dsa_check_status",
+    "dsa_index_dense_workspace_size", "dsa_index_dense",
+    "dsa_index_group_workspace_size", "dsa_index_group",
+    "dsa_index_decode_workspace_size", "dsa_index_decode",
+    "dsa_debug_scores",
+)
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = _status_text(status) if _LIB is not None else str(status)
+        super().__init__(f"{what}: {msg} ({status})" if what else f"{msg} ({status})")
+
+
+_LIB = None
+
+_c_int, _c_i64, _c_sz, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+_SIGS = {
+    "dsa_status_string": (ctypes.c_char_p, [_c_int]),
+    "dsa_version": (_c_int, []),
+    "dsa_check_status": (_c_int, [_vp, _vp]),
+    "dsa_index_dense_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_dense": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                 _c_int, _vp, _vp, _vp, _c_sz, _vp]),
+    "dsa_index_group_workspace_size": (_c_int, [_c_int] * 9 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_group": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_sz, _vp]),
+    "dsa_index_decode_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_sz, _vp]),
+    "dsa_debug_scores": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                  _vp, _vp, _c_sz, _vp]),
+}
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(f"{lib_path} is missing: build it with "
+                               "`python -m sparse_attention_token_index_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _status_text(s: int) -> str:
+    return lib().dsa_status_string(int(s)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise DsaError(status, what)
+
+
+def _dtype_code(t: torch.Tensor, allow_fp8=False) -> int:
+    if t.dtype == torch.bfloat16:
+        return DSA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DSA_DTYPE_FP32
+    if allow_fp8 and t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return DSA_DTYPE_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (the indexer has no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace has {workspace.numel()} bytes, needs {nbytes}")
+        return workspace
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def dense_workspace_bytes(T, N, H, d, k, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_dense_workspace_size(T, N, H, d, k, q_dtype, k_dtype, ctypes.byref(n)),
+           "dsa_index_dense_workspace_size")
+    return n.value
+
+
+def group_workspace_bytes(T, N, H, d, k, group, bank, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_group_workspace_size(T, N, H, d, k, group, bank, q_dtype, k_dtype, ctypes.byref(n)),
+           "dsa_index_group_workspace_size")
+    return n.value
+
+
+def decode_workspace_bytes(B, total_q, max_keys, H, d, k, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_decode_workspace_size(B, total_q, max_keys, H, d, k, q_dtype, k_dtype,
+                                                 ctypes.byref(n)), "dsa_index_decode_workspace_size")
+    return n.value
+
+
+def dsa_check_status(workspace: torch.Tensor, stream=None) -> None:
+    """Waits for the stream and raises if a kernel recorded a device-side failure."""
+    _check(lib().dsa_check_status(_ptr(workspace), _stream(stream)), "device status")
+
+
+def _outputs(rows, k, device, out):
+    if out is not None:
+        idx, val = out
+        _need_cuda(idx, val)
+        assert idx.dtype == torch.int32 and val.dtype == torch.float32
+        assert idx.shape == (rows, k) and val.shape == (rows, k)
+        return idx, val
+    return (torch.empty((rows, k), dtype=torch.int32, device=device),
+            torch.empty((rows, k), dtype=torch.float32, device=device))
+
+
+def dsa_index_dense(Q: torch.Tensor, w: torch.Tensor, K: torch.Tensor, k: int, q_pos0: Optional[int] = None,
+                    K_scale: Optional[torch.Tensor] = None, out=None, workspace=None, stream=None,
+                    check: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Dense prefill indexer: per query row t the top-k keys among 0..q_pos0+t.
+
+    Q [T,H,d] bf16/fp32, w [T,H] fp32, K [N,d] bf16/fp32 or fp8 e4m3 bytes
+    (then ``K_scale`` [N] fp32).  Returns (idx [T,k] int32, val [T,k] fp32);
+    each row is a set, padded with -1 / -inf.
+    """
+    _need_cuda(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    nb = dense_workspace_bytes(T, N, H, d, k, qd, kd)
+    ws = _workspace(nb, Q.device, workspace)
+    idx, val = _outputs(T, k, Q.device, out)
+    _check(lib().dsa_index_dense(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, k, qd, kd,
+                                 _ptr(idx), _ptr(val), _ptr(ws), ws.numel(), _stream(stream)), "dsa_index_dense")
+    if check:
+        dsa_check_status(ws, stream)
+    return idx, val
+
+
+def dsa_index_group(Q, w, K, k: int, group: int, bank: int, mode: int = DSA_GROUP_REFINE,
+                    q_pos0: Optional[int] = None, K_scale=None, out=None, return_bank: bool = False,
+                    return_proxy: bool = False, workspace=None, stream=None, check: bool = False):
+    """Group-shared (PIVOT) prefill indexer, Refine or Reuse.
+
+    Returns (idx, val) and, on request, (bank_idx [ng,B], bank_val [ng,B]) in
+    the proxy's ranking order and (proxy_q [ng,H,d], proxy_w [ng,H]).
+    """
+    _need_cuda(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    ng = (T + group - 1) // group
+    nb = group_workspace_bytes(T, N, H, d, k, group, bank, qd, kd)
+    ws = _workspace(nb, Q.device, workspace)
+    idx, val = _outputs(T, k, Q.device, out)
+    bi = bv = pq = pw = None
+    if return_bank:
+        bi = torch.empty((ng, bank), dtype=torch.int32, device=Q.device)
+        bv = torch.empty((ng, bank), dtype=torch.float32, device=Q.device)
+    if return_proxy:
+        pq = torch.empty((ng, H, d), dtype=Q.dtype, device=Q.device)
+        pw = torch.empty((ng, H), dtype=torch.float32, device=Q.device)
+    _check(lib().dsa_index_group(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, k, group, bank,
+                                 int(mode), qd, kd, _ptr(idx), _ptr(val), _ptr(bi), _ptr(bv), _ptr(pq), _ptr(pw),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "dsa_index_group")
+    if check:
+        dsa_check_status(ws, stream)
+    res = [idx, val]
+    if return_bank:
+        res += [bi, bv]
+    if return_proxy:
+        res += [pq, pw]
+    return tuple(res)
+
+
+def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.Tensor,
+                     max_keys: Optional[int] = None, K_scale=None, out=None, workspace=None, stream=None,
+                     check: bool = False):
+    """Decode indexer over B key caches; offsets are [B+1] (host or device).
+
+    Returns (idx [sum m_b, k], val) with key indices local to each sequence.
+    """
+    _need_cuda(Q, w, K, K_scale)
+    total_q, H, d = Q.shape
+    B = k_offsets.numel() - 1
+    ko_host = k_offsets.to("cpu", torch.int64)
+    if max_keys is None:
+        max_keys = int((ko_host[1:] - ko_host[:-1]).max())
+    total_keys = int(ko_host[-1])
+    ko = k_offsets.to(Q.device, torch.int64).contiguous()
+    qo = q_offsets.to(Q.device, torch.int32).contiguous()
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    nb = decode_workspace_bytes(B, total_q, max_keys, H, d, k, qd, kd)
+    ws = _workspace(nb, Q.device, workspace)
+    idx, val = _outputs(total_q, k, Q.device, out)
+    _check(lib().dsa_index_decode(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), _ptr(ko), _ptr(qo), B, total_q,
+                                  total_keys, max_keys, H, d, k, qd, kd, _ptr(idx), _ptr(val), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "dsa_index_decode")
+    if check:
+        dsa_check_status(ws, stream)
+    return idx, val
+
+
+def dsa_debug_scores(Q, w, K, q_pos0: Optional[int] = None, K_scale=None, workspace=None, stream=None,
+                     check: bool = False) -> torch.Tensor:
+    """Test aid: the full [T, N] score matrix of the dense kernels (-inf beyond each prefix)."""
+    _need_cuda(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    nb = dense_workspace_bytes(T, N, H, d, 1, qd, kd) + 8 * T + 1024
+    ws = _workspace(nb, Q.device, workspace)
+    S = torch.empty((T, N), dtype=torch.float32, device=Q.device)
+    _check(lib().dsa_debug_scores(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, qd, kd, _ptr(S),
+                                  _ptr(ws), ws.numel(), _stream(stream)), "dsa_debug_scores")
+    if check:
+        dsa_check_status(ws, stream)
+    return S

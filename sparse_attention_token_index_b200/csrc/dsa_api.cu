@@ -1,0 +1,561 @@
+// dsa_api.cu — the extern "C" entry points declared in include/dsa_index.h.
+//
+// Host side only: argument validation, workspace layout, TMA tensor-map
+// encoding and kernel dispatch.  Nothing here allocates device memory or
+// synchronises a stream (except dsa_check_status, whose job that is).
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+using namespace dsa;
+
+namespace {
+
+constexpr int kMaxK = 65536;
+
+struct DeviceInfo {
+  bool ok = false;
+  int sms = 0;
+};
+
+int device_info(DeviceInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  static DeviceInfo cache[64];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return DSA_ERR_DEVICE;
+  if (!cache[dev].ok) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (major != 10 || minor != 0) return DSA_ERR_DEVICE;
+    cache[dev].sms = sms;
+    cache[dev].ok = true;
+  }
+  out = cache[dev];
+  return DSA_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over [rows, inner] with a box of 64 elements (128 B)
+// x box_rows rows, 128-byte swizzle (the layout the MMA descriptors expect).
+int make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return DSA_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt_size(int dt) { return dt == DSA_DTYPE_FP32 ? 4 : (dt == DSA_DTYPE_BF16 ? 2 : 1); }
+
+// Simple bump layout over the caller's workspace (256-byte aligned pieces).
+struct Layout {
+  size_t off = sizeof(WsHeader);
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  }
+};
+
+bool use_tc(int H, int d, int q_dtype, int k_dtype) {
+  return q_dtype == DSA_DTYPE_BF16 && k_dtype == DSA_DTYPE_BF16 && H == 64 && d == 128;
+}
+
+int check_common(int H, int d, int k, int q_dtype, int k_dtype) {
+  if (H < 1 || H > 128 || d < 1 || d > 256 || H * d > 8192) return DSA_ERR_UNSUPPORTED;
+  if (k < 1 || k > kMaxK) return DSA_ERR_INVALID_ARG;
+  if (q_dtype != DSA_DTYPE_BF16 && q_dtype != DSA_DTYPE_FP32) return DSA_ERR_UNSUPPORTED;
+  if (k_dtype != DSA_DTYPE_BF16 && k_dtype != DSA_DTYPE_FP32 && k_dtype != DSA_DTYPE_FP8_E4M3)
+    return DSA_ERR_UNSUPPORTED;
+  if (q_dtype == DSA_DTYPE_FP32 && k_dtype == DSA_DTYPE_BF16) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+int simt_grid(const DeviceInfo& di, int64_t tasks) {
+  int64_t g = (tasks + 1) / 2;
+  const int64_t cap = (int64_t)di.sms * 4;
+  return (int)(g < cap ? (g < 1 ? 1 : g) : cap);
+}
+
+// Dense / proxy-scan workspace pieces.
+struct DensePlan {
+  bool tc;
+  int grid;
+  int64_t cand_cap;
+  size_t cand_off;
+  size_t total;
+};
+
+DensePlan plan_dense(const DeviceInfo& di, int T, int N, int H, int d, int q_dtype, int k_dtype, Layout& L) {
+  DensePlan p;
+  p.tc = use_tc(H, d, q_dtype, k_dtype);
+  p.cand_cap = ((int64_t)N + 127) / 128 * 128;
+  if (p.tc) {
+    const int units = (T + 3) / 4;
+    p.grid = units < di.sms ? units : di.sms;
+    p.cand_off = L.take((size_t)p.grid * 4 * p.cand_cap * sizeof(uint2));
+  } else {
+    p.grid = simt_grid(di, T);
+    p.cand_off = L.take((size_t)p.grid * 2 * p.cand_cap * sizeof(uint2));
+  }
+  p.total = L.off;
+  return p;
+}
+
+int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, const float* w, const void* K,
+                   const float* K_scale, int n_rows, int N, int H, int d, int64_t pos_base, int64_t pos_mul,
+                   int64_t pos_add, int64_t pos_clamp, int k, int q_dtype, int k_dtype, int32_t* idx, float* val,
+                   uint8_t* ws, float* dbg, int64_t dbg_ld, cudaStream_t st) {
+  int* status = reinterpret_cast<int*>(ws);
+  uint2* cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+  if (p.tc) {
+    CUtensorMap tmQ, tmK;
+    int r = make_map_bf16(&tmQ, Q, (uint64_t)n_rows * H, (uint64_t)d, 64);
+    if (r != DSA_OK) return r;
+    r = make_map_bf16(&tmK, K, (uint64_t)N, (uint64_t)d, 128);
+    if (r != DSA_OK) return r;
+    TcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.kind = 0;
+    a.n_rows = n_rows;
+    a.n_units = (n_rows + 3) / 4;
+    a.k = k;
+    a.pos_base = pos_base;
+    a.pos_mul = pos_mul;
+    a.pos_add = pos_add;
+    a.pos_clamp = pos_clamp;
+    a.w = w;
+    a.out_idx = idx;
+    a.out_val = val;
+    a.out_ld = k;
+    a.cand = cand;
+    a.cand_cap = p.cand_cap;
+    a.status = status;
+    a.dbg_scores = dbg;
+    a.dbg_ld = dbg_ld;
+    const int grid = a.n_units < p.grid ? a.n_units : p.grid;
+    return launch_tc_index(tmQ, tmK, a, grid, st);
+  }
+  if (pos_mul != 1 || pos_add != 0) return DSA_ERR_UNSUPPORTED;  // proxy rows use the tensor-core kernel
+  SimtArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 0;
+  a.n_tasks = n_rows;
+  a.H = H;
+  a.d = d;
+  a.k = k;
+  a.q_dtype = q_dtype;
+  a.k_dtype = k_dtype;
+  a.Q = Q;
+  a.w = w;
+  a.K = K;
+  a.K_scale = K_scale;
+  a.q_pos0 = pos_base;
+  a.out_idx = idx;
+  a.out_val = val;
+  a.out_ld = k;
+  a.cand = cand;
+  a.cand_cap = p.cand_cap;
+  a.status = status;
+  a.dbg_scores = dbg;
+  a.dbg_ld = dbg_ld;
+  const int grid = simt_grid(di, n_rows) < p.grid ? simt_grid(di, n_rows) : p.grid;
+  return launch_simt_index(a, grid, st);
+}
+
+int validate_dense(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
+                   int64_t q_pos0, int k, int q_dtype, int k_dtype) {
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!Q || !w || !K) return DSA_ERR_INVALID_ARG;
+  if (T < 1 || N < 1 || q_pos0 < 0 || q_pos0 + (int64_t)T > (int64_t)N) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)T * H * d >= ((int64_t)1 << 40)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_status_string(int status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device-side wait timed out";
+    case DSA_ERR_DEVICE: return "device is not sm_100";
+    case DSA_ERR_INTERNAL: return "device-side consistency check failed";
+    default: return "unknown status";
+  }
+}
+
+int dsa_version(void) { return 100; }
+
+int dsa_check_status(void* workspace, void* stream) {
+  if (!workspace) return DSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (h[0] != 0) {
+    const int z[2] = {0, 0};
+    if (cudaMemcpy(workspace, z, sizeof(z), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+    return h[0];
+  }
+  return DSA_OK;
+}
+
+int dsa_index_dense_workspace_size(int T, int N, int H, int d, int k, int q_dtype, int k_dtype, size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (T < 1 || N < 1) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  Layout L;
+  *bytes = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L).total;
+  return DSA_OK;
+}
+
+int dsa_index_dense(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
+                    int64_t q_pos0, int k, int q_dtype, int k_dtype, int32_t* idx, float* val, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  Layout L;
+  DensePlan p = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L);
+  if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
+  return run_dense_rows(di, p, Q, w, K, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype, k_dtype,
+                        idx, val, static_cast<uint8_t*>(workspace), nullptr, 0,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int dsa_debug_scores(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
+                     int64_t q_pos0, int q_dtype, int k_dtype, float* S, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  const int k = 1;
+  int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!S || !workspace) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)T * N > ((int64_t)1 << 26)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  Layout L;
+  DensePlan p = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L);
+  // the top-1 outputs of this run go to scratch behind the plan
+  const size_t oi = L.take((size_t)T * sizeof(int32_t));
+  const size_t ov = L.take((size_t)T * sizeof(float));
+  if (workspace_bytes < L.off) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((r = launch_fill_scores(S, (int64_t)T * N, st)) != DSA_OK) return r;
+  return run_dense_rows(di, p, Q, w, K, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype, k_dtype,
+                        reinterpret_cast<int32_t*>(ws + oi), reinterpret_cast<float*>(ws + ov), ws, S, N, st);
+}
+
+}  // extern "C"
+
+// --------------------------------------------------------------------------
+// group and decode
+// --------------------------------------------------------------------------
+namespace {
+
+struct GroupPlan {
+  int ng;
+  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off;
+  DensePlan scan;       // proxy scan
+  int64_t ref_cap;      // refine candidate capacity
+  size_t ref_cand_off;
+  int ref_grid;
+  size_t total;
+};
+
+int plan_group(const DeviceInfo& di, int T, int N, int H, int d, int k, int G, int B, int q_dtype, int k_dtype,
+               GroupPlan& gp) {
+  Layout L;
+  gp.ng = (T + G - 1) / G;
+  gp.qbar_off = L.take((size_t)gp.ng * H * d * elt_size(q_dtype));
+  gp.wbar_off = L.take((size_t)gp.ng * H * sizeof(float));
+  gp.bidx_off = L.take((size_t)gp.ng * B * sizeof(int32_t));
+  gp.bval_off = L.take((size_t)gp.ng * B * sizeof(float));
+  gp.scan = plan_dense(di, gp.ng, N, H, d, q_dtype, k_dtype, L);
+  gp.kg_off = 0;
+  gp.ref_cand_off = 0;
+  gp.ref_cap = ((int64_t)B + 127) / 128 * 128;
+  gp.ref_grid = 0;
+  if (use_tc(H, d, q_dtype, k_dtype)) {
+    gp.kg_off = L.take((size_t)gp.ng * B * d * elt_size(k_dtype));
+    const int mblocks = (G + 3) / 4;
+    const int64_t units = (int64_t)gp.ng * mblocks;
+    gp.ref_grid = units < di.sms ? (int)units : di.sms;
+    gp.ref_cand_off = L.take((size_t)gp.ref_grid * 4 * gp.ref_cap * sizeof(uint2));
+  }
+  gp.total = L.off;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_index_group_workspace_size(int T, int N, int H, int d, int k, int group, int bank, int q_dtype, int k_dtype,
+                                   size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (T < 1 || N < 1 || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  GroupPlan gp;
+  plan_group(di, T, N, H, d, k, group, bank, q_dtype, k_dtype, gp);
+  *bytes = gp.total;
+  return DSA_OK;
+}
+
+int dsa_index_group(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
+                    int64_t q_pos0, int k, int group, int bank, int mode, int q_dtype, int k_dtype, int32_t* idx,
+                    float* val, int32_t* bank_idx, float* bank_val, void* proxy_q, float* proxy_w, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!idx || !val || !workspace || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if ((proxy_q && !aligned16(proxy_q)) || (proxy_w && !aligned16(proxy_w))) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  GroupPlan gp;
+  plan_group(di, T, N, H, d, k, group, bank, q_dtype, k_dtype, gp);
+  if (workspace_bytes < gp.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* qbar = proxy_q ? proxy_q : ws + gp.qbar_off;
+  float* wbar = proxy_w ? proxy_w : reinterpret_cast<float*>(ws + gp.wbar_off);
+  int32_t* bi = bank_idx ? bank_idx : reinterpret_cast<int32_t*>(ws + gp.bidx_off);
+  float* bv = bank_val ? bank_val : reinterpret_cast<float*>(ws + gp.bval_off);
+  // 1. proxies
+  if ((r = launch_proxy_mean(Q, w, T, H, d, group, q_dtype, qbar, wbar, st)) != DSA_OK) return r;
+  // 2. one full-prefix scan per proxy: bank = its top-`bank` keys
+  if ((r = run_dense_rows(di, gp.scan, qbar, wbar, K, K_scale, gp.ng, N, H, d, q_pos0, group, group - 1,
+                          (int64_t)T - 1, bank, q_dtype, k_dtype, bi, bv, ws, nullptr, 0, st)) != DSA_OK)
+    return r;
+  // 3. rank the bank; Reuse finishes here
+  if ((r = launch_bank_rank_reuse(bi, bv, gp.ng, bank, group, T, q_pos0, k, idx, val, mode == DSA_GROUP_REUSE,
+                                  st)) != DSA_OK)
+    return r;
+  if (mode == DSA_GROUP_REUSE) return DSA_OK;
+  // 4. Refine: members re-score their group's bank on tensor cores
+  void* Kg = ws + gp.kg_off;
+  if ((r = launch_bank_gather(K, k_dtype, d, bi, gp.ng, bank, Kg, st)) != DSA_OK) return r;
+  CUtensorMap tmQ, tmK;
+  if ((r = make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)gp.ng * bank, (uint64_t)d, 128)) != DSA_OK) return r;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 2;
+  a.n_rows = T;
+  a.mblocks = (group + 3) / 4;
+  a.n_units = gp.ng * a.mblocks;
+  a.k = k;
+  a.pos_base = q_pos0;
+  a.w = w;
+  a.out_idx = idx;
+  a.out_val = val;
+  a.out_ld = k;
+  a.cand = reinterpret_cast<uint2*>(ws + gp.ref_cand_off);
+  a.cand_cap = gp.ref_cap;
+  a.status = reinterpret_cast<int*>(ws);
+  a.key_map = bi;
+  a.bank = bank;
+  a.group = group;
+  a.T = T;
+  return launch_tc_index(tmQ, tmK, a, gp.ref_grid, st);
+}
+
+}  // extern "C"
+
+namespace {
+
+struct DecodePlan {
+  bool tc;
+  int splits, tiles_per_split;
+  int grid;
+  int64_t cand_cap;
+  size_t cand_off, pidx_off, pval_off, pcnt_off, mscr_off, total;
+};
+
+void plan_decode(const DeviceInfo& di, int B, int total_q, int max_keys, int H, int d, int k, int q_dtype,
+                 int k_dtype, DecodePlan& p) {
+  p.tc = use_tc(H, d, q_dtype, k_dtype);
+  const int tiles_max = (max_keys + 127) / 128;
+  // choose the split count minimising (rounds of units) x (tiles per unit + a
+  // fixed per-unit cost of about 4 tiles)
+  int best_s = 1;
+  double best_cost = 1e300;
+  for (int s = 1; s <= 256 && s <= tiles_max; ++s) {
+    const int tps = (tiles_max + s - 1) / s;
+    const int s_eff = (tiles_max + tps - 1) / tps;
+    const int64_t units = (int64_t)B * s_eff;
+    const int64_t rounds = (units + di.sms - 1) / di.sms;
+    const double cost = (double)rounds * (tps + 4) + 0.01 * s_eff;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_s = s_eff;
+    }
+  }
+  p.splits = best_s;
+  p.tiles_per_split = (tiles_max + best_s - 1) / best_s;
+  p.cand_cap = (int64_t)p.tiles_per_split * 128;
+  Layout L;
+  if (p.tc) {
+    const int64_t units = (int64_t)B * p.splits;
+    p.grid = units < di.sms ? (int)units : di.sms;
+    p.cand_off = L.take((size_t)p.grid * 4 * p.cand_cap * sizeof(uint2));
+  } else {
+    p.grid = simt_grid(di, (int64_t)total_q * p.splits);
+    p.cand_off = L.take((size_t)p.grid * 2 * p.cand_cap * sizeof(uint2));
+  }
+  const size_t parts = (size_t)total_q * p.splits;
+  p.pidx_off = L.take(parts * k * sizeof(int32_t));
+  p.pval_off = L.take(parts * k * sizeof(float));
+  p.pcnt_off = L.take(parts * sizeof(int));
+  p.mscr_off = L.take(parts * k * sizeof(uint2));
+  p.total = L.off;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_index_decode_workspace_size(int B, int total_q, int max_keys, int H, int d, int k, int q_dtype, int k_dtype,
+                                    size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (B < 1 || total_q < 1 || max_keys < 1) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  DecodePlan p;
+  plan_decode(di, B, total_q, max_keys, H, d, k, q_dtype, k_dtype, p);
+  *bytes = p.total;
+  return DSA_OK;
+}
+
+int dsa_index_decode(const void* Q, const float* w, const void* K, const float* K_scale, const int64_t* k_offsets,
+                     const int32_t* q_offsets, int B, int total_q, int64_t total_keys, int max_keys, int H, int d,
+                     int k, int q_dtype, int k_dtype, int32_t* idx, float* val, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
+  if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  DecodePlan p;
+  plan_decode(di, B, total_q, max_keys, H, d, k, q_dtype, k_dtype, p);
+  if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = reinterpret_cast<int*>(ws);
+  int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
+  float* pval = reinterpret_cast<float*>(ws + p.pval_off);
+  int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
+  if (p.tc) {
+    CUtensorMap tmQ, tmK;
+    if ((r = make_map_bf16(&tmQ, Q, (uint64_t)total_q * H, (uint64_t)d, 64)) != DSA_OK) return r;
+    // rows: the whole key array; a tile running past its sequence's end is
+    // masked per key, and rows past the array's end read as zeros
+    if ((r = make_map_bf16(&tmK, K, (uint64_t)total_keys, (uint64_t)d, 128)) != DSA_OK) return r;
+    TcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.kind = 1;
+    a.n_rows = total_q;
+    a.n_units = B * p.splits;
+    a.k = k;
+    a.w = w;
+    a.out_idx = pidx;
+    a.out_val = pval;
+    a.out_ld = k;
+    a.out_cnt = pcnt;
+    a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+    a.cand_cap = p.cand_cap;
+    a.status = status;
+    a.k_off = k_offsets;
+    a.q_off = q_offsets;
+    a.splits = p.splits;
+    a.tiles_per_split = p.tiles_per_split;
+    if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
+  } else {
+    SimtArgs a;
+    memset(&a, 0, sizeof(a));
+    a.kind = 1;
+    a.n_tasks = total_q * p.splits;
+    a.H = H;
+    a.d = d;
+    a.k = k;
+    a.q_dtype = q_dtype;
+    a.k_dtype = k_dtype;
+    a.Q = Q;
+    a.w = w;
+    a.K = K;
+    a.K_scale = K_scale;
+    a.out_idx = pidx;
+    a.out_val = pval;
+    a.out_ld = k;
+    a.out_cnt = pcnt;
+    a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+    a.cand_cap = p.cand_cap;
+    a.status = status;
+    a.k_off = k_offsets;
+    a.q_off = q_offsets;
+    a.B = B;
+    a.splits = p.splits;
+    a.keys_per_split = p.tiles_per_split * 128;
+    if ((r = launch_simt_index(a, p.grid, st)) != DSA_OK) return r;
+  }
+  return launch_decode_merge(pidx, pval, pcnt, total_q, p.splits, k, idx, val,
+                             reinterpret_cast<uint2*>(ws + p.mscr_off), status, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,94 @@
+// dsa_internal.h — launch interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// Arguments of the tensor-core kernel (see dsa_tc.cu).
+//   kind 0: prefill rows.  Row r of Q sits at position
+//           pos_base + min(r * pos_mul + pos_add, pos_clamp) and sees keys
+//           0..pos (dense: pos_mul 1, pos_add 0; group proxies: pos_mul G,
+//           pos_add G-1 so the proxy scans its group's last member's prefix).
+//   kind 1: decode segments; unit v = (sequence v / splits, split v % splits).
+//   kind 2: group refine; unit v = (group v / mblocks, member block v % mblocks);
+//           keys are the group's gathered bank rows, key_map gives their
+//           positions.
+struct TcArgs {
+  int kind;
+  int n_rows;
+  int n_units;
+  int k;
+  int64_t pos_base, pos_mul, pos_add, pos_clamp;
+  const float* w;
+  int32_t* out_idx;
+  float* out_val;
+  int64_t out_ld;
+  int* out_cnt;
+  uint2* cand;
+  int64_t cand_cap;
+  int* status;
+  float* dbg_scores;
+  int64_t dbg_ld;
+  // decode
+  const int64_t* k_off;
+  const int32_t* q_off;
+  int splits;
+  int tiles_per_split;
+  // refine
+  const int32_t* key_map;   // [ng, bank] bank key positions (-1 = empty)
+  int bank;
+  int group;
+  int mblocks;
+  int T;
+};
+
+int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
+                    cudaStream_t stream);
+size_t tc_smem_bytes();
+
+// Exact fp32 CUDA-core path (any H <= 128, d <= 256, H*d <= 8192).
+struct SimtArgs {
+  int kind;          // 0 prefill rows, 1 decode (row task = (query row, split))
+  int n_tasks;
+  int H, d, k;
+  int q_dtype, k_dtype;
+  const void* Q;
+  const float* w;
+  const void* K;
+  const float* K_scale;
+  int64_t q_pos0;
+  int32_t* out_idx;
+  float* out_val;
+  int64_t out_ld;
+  int* out_cnt;
+  uint2* cand;
+  int64_t cand_cap;
+  int* status;
+  float* dbg_scores;
+  int64_t dbg_ld;
+  const int64_t* k_off;
+  const int32_t* q_off;
+  int B;
+  int splits;
+  int keys_per_split;
+};
+int launch_simt_index(const SimtArgs& a, int grid, cudaStream_t stream);
+size_t simt_smem_bytes(int H, int d);
+
+// Auxiliary kernels.
+int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
+                      float* wbar, cudaStream_t stream);
+int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
+                       void* Kg, cudaStream_t stream);
+int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,
+                           int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse,
+                           cudaStream_t stream);
+int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
+                        int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
+                        cudaStream_t stream);
+int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
+
+}  // namespace dsa

@@ -4,10 +4,10 @@ The pages evaluate on long-context suites with real models; neither is
 available here, so these generators stand in for their *shape*: long causal
 prefixes, k = 2048, long-tailed score rows (planted high-score keys) and
 neighbouring queries whose top-k overlap (a shared low-rank latent that
-drifts slowly with position).  See the PIVOT abstract ("nearby queries select
-highly overlapping top-k tokens, and the indexer scores are long-tailed along
-the key axis") and the AttentionIndex worked example (clustered keys scattered
-over positions).
+drifts slowly with position).  The PIVOT abstract observes both properties
+(neighbouring queries pick largely the same keys; along the keys, indexer
+scores have a long tail), and the AttentionIndex worked example scatters
+similar keys over positions, which the fp8 recipe's key clusters follow.
 
 Every draw comes from ``torch.Generator(device).manual_seed(seed)``; the same
 call on the same device type always returns the same tensors.  Nothing here

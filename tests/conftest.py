@@ -10,3 +10,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Make sure the in-tree library is built from the current sources."""
+    from sparse_attention_token_index_b200 import build as B
+    B.build()
+    yield

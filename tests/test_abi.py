@@ -1,0 +1,76 @@
+"""C-ABI library (no GPU): it builds, loads, exports every declared symbol, and
+rejects bad arguments on the host before touching a device."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import sparse_attention_token_index_b200 as dsa
+from sparse_attention_token_index_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return dsa.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(dsa_\w+)\s*\(", txt, flags=re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(dsa.EXPORTED_SYMBOLS) <= names
+
+
+def test_version_and_status_strings(L):
+    assert L.dsa_version() == 100
+    assert L.dsa_status_string(0) == b"ok"
+    for code in (-1, -2, -3, -4, -5, -6, -7):
+        assert L.dsa_status_string(code) != b"unknown status"
+
+
+def test_host_validation_before_device(L):
+    n = ctypes.c_size_t(0)
+    f = L.dsa_index_dense
+    ok_ptr = ctypes.c_void_p(4096)
+    # null Q
+    assert f(None, ok_ptr, ok_ptr, None, 4, 4, 64, 128, 0, 2, 0, 0, ok_ptr, ok_ptr, ok_ptr, 1 << 20, None) == -1
+    # k out of range
+    assert f(ok_ptr, ok_ptr, ok_ptr, None, 4, 4, 64, 128, 0, 0, 0, 0, ok_ptr, ok_ptr, ok_ptr, 1 << 20, None) == -1
+    # causal range past the keys
+    assert f(ok_ptr, ok_ptr, ok_ptr, None, 4, 4, 64, 128, 1, 2, 0, 0, ok_ptr, ok_ptr, ok_ptr, 1 << 20, None) == -1
+    # unsupported shape (H * d too large)
+    assert f(ok_ptr, ok_ptr, ok_ptr, None, 4, 4, 128, 256, 0, 2, 0, 0, ok_ptr, ok_ptr, ok_ptr, 1 << 20, None) == -2
+    # misaligned Q
+    assert f(ctypes.c_void_p(4100), ok_ptr, ok_ptr, None, 4, 4, 64, 128, 0, 2, 0, 0, ok_ptr, ok_ptr, ok_ptr,
+             1 << 20, None) == -1
+    # fp8 keys need a scale
+    assert f(ok_ptr, ok_ptr, ok_ptr, None, 4, 4, 64, 128, 0, 2, 0, 2, ok_ptr, ok_ptr, ok_ptr, 1 << 20, None) == -1
+    # group: bank smaller than k
+    g = L.dsa_index_group
+    assert g(ok_ptr, ok_ptr, ok_ptr, None, 8, 8, 64, 128, 0, 4, 2, 2, 0, 0, 0, ok_ptr, ok_ptr, None, None, None,
+             None, ok_ptr, 1 << 20, None) == -1
+    # workspace-size query rejects a null output pointer
+    assert L.dsa_index_dense_workspace_size(4, 4, 64, 128, 2, 0, 0, None) == -1
+    assert n.value == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(2, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dsa.dsa_index_dense(q, torch.zeros(2, 64), torch.zeros(4, 128, dtype=torch.bfloat16), 2)
