@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const int32_t* __rest
     if (tid < 32) row_update(M.st, k, lane);
     named_bar(1, 128);
   }
-  row_select(M.st, cand, k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k, M.stage, 2048, tid, 128, 1,
+  row_select(M.st, single_list(cand, M.st.cnt), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k, M.stage, 2048, tid, 128, 1,
              status);
 }
 

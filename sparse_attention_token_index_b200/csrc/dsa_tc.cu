@@ -7,30 +7,36 @@
 //
 //   * one persistent CTA per SM; a work unit is up to 4 queries (N = 4 x 64
 //     = 256 columns) against the keys they see, streamed in tiles of 128;
-//   * warp 8 issues TMA loads (no multicast): the unit's Q block once, then
+//   * warp 16 issues TMA loads (no multicast): the unit's Q block once, then
 //     key tiles into a 3-stage ring (128B-swizzled, K-major);
-//   * warp 9 allocates 512 TMEM columns and issues tcgen05.mma
+//   * warp 17 allocates 512 TMEM columns and issues tcgen05.mma
 //     (M=128, N=nq*64, K=16 steps) into one of two 256-column accumulators;
-//   * warps 0-7 (two warpgroups) drain TMEM with tcgen05.ld: each thread owns
-//     one key row, so ReLU, the head weighting and the head sum stay in
-//     registers; the causal cut and the streaming top-k filter follow at once.
+//   * warps 0-15 form four epilogue warpgroups, one per query of the unit.
+//     Each thread owns one key row of the tile: tcgen05.ld brings its 64 head
+//     dot products into registers, ReLU and the head weights are applied with
+//     packed fp32x2 FMAs, and the causal cut and the streaming top-k filter
+//     follow at once.
 //
-// Work units come in two kinds: prefill rows (dense queries or group proxies,
-// each row with its own causal position) and decode segments (the m new
-// queries of one sequence against one slice of that sequence's key cache,
-// whose local top-k lists a merge kernel combines).
+// Work units come in three kinds: prefill rows (dense queries or group
+// proxies, each row with its own causal position), decode segments (the m
+// new queries of one sequence against one slice of that sequence's key
+// cache; a merge kernel combines the slices), and group-refine blocks (up to
+// 4 members of a group against the group's gathered candidate bank).
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
 
-constexpr int kTcThreads = 320;
+constexpr int kEpiWarps = 16;
+constexpr int kTcThreads = (kEpiWarps + 2) * 32;  // + TMA producer + MMA issuer
+constexpr int kProducerWarp = kEpiWarps;
+constexpr int kMmaWarp = kEpiWarps + 1;
 constexpr int kQB = 4;            // queries per unit
 constexpr int kHeads = 64;
 constexpr int kTileKeys = 128;
 constexpr int kStages = 3;
-constexpr int kStageCap = 2048;   // staged entries of the threshold bin, per warpgroup
+constexpr int kStageCap = 1024;   // staged entries of the threshold bin, per query
 constexpr int kQChunkBytes = kQB * kHeads * 64 * 2;      // 32 KB: 256 rows x 128 B
 constexpr int kQHeadBlockBytes = kHeads * 64 * 2;        // 8 KB: one query, one d-chunk
 constexpr int kKChunkBytes = kTileKeys * 64 * 2;         // 16 KB
@@ -41,7 +47,7 @@ struct TcSmem {
   uint8_t k[kStages][kKStageBytes];            // [stage][2][128 rows][128 B]
   RowState rows[kQB];
   float w[kQB][kHeads];
-  uint2 stage[2][kStageCap];
+  uint2 stage[kQB][kStageCap];
   uint64_t q_full, q_empty, drain;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t t_full[2], t_empty[2];
@@ -50,16 +56,16 @@ struct TcSmem {
 };
 
 constexpr size_t kTcSmemBytes = sizeof(TcSmem) + 1024;  // + alignment slack
+static_assert(kTcSmemBytes <= 232448, "fits the 227 KB opt-in shared memory of one CTA");
 
 struct UnitInfo {
-  int nq;            // queries in the unit (0 = no unit)
+  int nq;            // queries in the unit (0 = no work)
   int row0;          // first Q row
   int key_row0;      // first K row of the streamed key range (global row)
   int tile0;         // first key tile (local to the key range)
   int ntiles;        // tiles streamed
   int nkeys;         // keys in the range (local index < nkeys is valid)
-  int64_t pos[kQB];  // causal position of each query (local key index)
-  int seq_split;     // decode: output slot (row * splits + split); prefill: -1
+  int seq_split;     // decode: split index; refine: group index
 };
 
 __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
@@ -77,8 +83,7 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     const int unit = a.n_units - 1 - v;
     u.row0 = unit * kQB;
     u.nq = min(kQB, a.n_rows - u.row0);
-    for (int j = 0; j < kQB; ++j) u.pos[j] = prefill_pos(a, u.row0 + min(j, u.nq - 1));
-    const int64_t maxpos = u.pos[u.nq - 1];
+    const int64_t maxpos = prefill_pos(a, u.row0 + u.nq - 1);
     u.key_row0 = 0;
     u.tile0 = 0;
     u.ntiles = (int)(maxpos / kTileKeys) + 1;
@@ -91,7 +96,6 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     const int nb = (int)(k1 - k0), mb = q1 - q0;
     u.row0 = q0;
     u.nq = mb;
-    for (int j = 0; j < kQB; ++j) u.pos[j] = (int64_t)nb - mb + min(j, mb - 1);
     const int tiles_b = (nb + kTileKeys - 1) / kTileKeys;
     const int t0 = min(tiles_b, sp * a.tiles_per_split);
     const int t1 = min(tiles_b, t0 + a.tiles_per_split);
@@ -107,7 +111,6 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     const int r_end = min(a.T, (g + 1) * a.group);
     u.row0 = g * a.group + mbk * kQB;
     u.nq = max(0, min(kQB, r_end - u.row0));
-    for (int j = 0; j < kQB; ++j) u.pos[j] = a.pos_base + u.row0 + min(j, max(u.nq - 1, 0));
     const int64_t L = a.pos_base + r_end - 1;
     const int nbk = (int)min((int64_t)a.bank, L + 1);
     u.key_row0 = g * a.bank;
@@ -117,6 +120,13 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     u.seq_split = g;
   }
   return true;
+}
+
+// Causal position of query `slot` of a unit (slot < u.nq), in key-index units.
+__device__ __forceinline__ int64_t slot_pos(const TcArgs& a, const UnitInfo& u, int slot) {
+  if (a.kind == 0) return prefill_pos(a, u.row0 + slot);
+  if (a.kind == 1) return (int64_t)u.nkeys - u.nq + slot;
+  return a.pos_base + u.row0 + slot;
 }
 
 __device__ __forceinline__ bool group_and(int bar, int nthr, bool ok) {
@@ -132,6 +142,33 @@ __device__ __forceinline__ bool group_and(int bar, int nthr, bool ok) {
   return r != 0;
 }
 
+// c + a * b on two fp32 lanes at once (fma.rn.f32x2, per-lane IEEE fma).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t ra, rb, rc, rd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  return d;
+}
+
+// acc += w[h] * max(v[h], 0) over 32 heads (w4 points at those heads'
+// weights), four packed accumulators.
+__device__ __forceinline__ void head_accumulate32(const float (&v)[32], const float4* __restrict__ w4,
+                                                  float2 (&acc)[4]) {
+#pragma unroll
+  for (int h = 0; h < 32; h += 8) {
+    const float4 wa = w4[h >> 2], wb = w4[(h >> 2) + 1];
+    acc[0] = ffma2(make_float2(wa.x, wa.y), make_float2(fmaxf(v[h + 0], 0.f), fmaxf(v[h + 1], 0.f)), acc[0]);
+    acc[1] = ffma2(make_float2(wa.z, wa.w), make_float2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), acc[1]);
+    acc[2] = ffma2(make_float2(wb.x, wb.y), make_float2(fmaxf(v[h + 4], 0.f), fmaxf(v[h + 5], 0.f)), acc[2]);
+    acc[3] = ffma2(make_float2(wb.z, wb.w), make_float2(fmaxf(v[h + 6], 0.f), fmaxf(v[h + 7], 0.f)), acc[3]);
+  }
+}
+
+template <bool kDebug>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_index_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ TcArgs a) {
@@ -150,13 +187,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.t_full[b], 1);
-      mbar_init(&S.t_empty[b], 8);
+      mbar_init(&S.t_empty[b], kEpiWarps);
     }
     S.abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) tmem_alloc(&S.tmem_base, 512);
-  if (warp == 8 && lane == 0) {
+  if (warp == kMmaWarp) tmem_alloc(&S.tmem_base, 512);
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
   }
@@ -165,7 +202,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int s = 0;
@@ -202,13 +239,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (armed[t]) mbar_wait(&S.k_full[t], armed_ph[t], abort_flag, a.status, 12);
       if (qi > 0) mbar_wait(&S.q_full, (qi - 1) & 1, abort_flag, a.status, 13);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
       int qi = 0, buf = 0;
-      uint32_t tph[2] = {0u, 0u};
+      uint32_t tph = 0u;  // bit b: phase of accumulator buffer b
       bool ok = true;
       UnitInfo u;
       const uint32_t q_addr = smem_u32(S.q);
@@ -219,7 +256,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t idesc = idesc_bf16_f32(128, u.nq * kHeads);
         for (int j = 0; j < u.ntiles; ++j) {
           if (!(ok = mbar_wait(&S.k_full[s], ph, abort_flag, a.status, 21))) break;
-          if (!(ok = mbar_wait(&S.t_empty[buf], tph[buf] ^ 1u, abort_flag, a.status, 22))) break;
+          if (!(ok = mbar_wait(&S.t_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort_flag, a.status, 22))) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
           const uint32_t k_addr = smem_u32(S.k[s]);
@@ -234,7 +271,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tc_commit(&S.k_empty[s]);
           tc_commit(&S.t_full[buf]);
-          tph[buf] ^= 1u;
+          tph ^= 1u << buf;
           buf ^= 1;
           if (++s == kStages) {
             s = 0;
@@ -249,100 +286,107 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait(&S.drain, 0, abort_flag, a.status, 23);
     }
   } else {
-    // ---------------- epilogue: warps 0-7, two warpgroups ----------------
-    const int wg = warp >> 2, lq = warp & 3, tid = threadIdx.x & 127;
-    const int bar = 1 + wg;
-    uint32_t eph[2] = {0u, 0u};
+    // ---------------- epilogue: warpgroup `slot` follows query `slot` ----------------
+    // Per tile a warp waits for its accumulator, pulls its 32 key rows x 64
+    // heads out of TMEM, frees the buffer, scores, and appends survivors of
+    // the threshold to its own candidate segment.  No barrier inside the
+    // tile loop: warp 0 of the group raises the threshold every few tiles
+    // from the shared histogram alone.
+    const int slot = warp >> 2, lq = warp & 3, tid = threadIdx.x & 127;
+    const int bar = 1 + slot;
+    RowState& st = S.rows[slot];
+    const int64_t seg_stride = a.cand_cap / 4;
+    uint2* const cand0 = a.cand + ((int64_t)blockIdx.x * kQB + slot) * a.cand_cap;
+    uint2* const my_seg = cand0 + lq * seg_stride;
+    const float4* w4 = reinterpret_cast<const float4*>(S.w[slot]);
+    const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
+    uint32_t eph = 0u;  // bit b: phase of accumulator buffer b
     int buf = 0;
     UnitInfo u;
     bool ok = true;
     for (int round = 0; ok && unit_at(a, round, u); ++round) {
-      // my query slots: wg, wg + 2
-      const int ns = (u.nq > wg) + (u.nq > wg + 2);
-      for (int j = 0; j < ns; ++j) {
-        const int slot = wg + 2 * j;
-        row_reset(S.rows[slot], tid, 128);
-        if (tid < kHeads) S.w[slot][tid] = a.w[(int64_t)(u.row0 + slot) * kHeads + tid];
+      // per-unit scalars (kept in registers through the tile loop)
+      const bool has_q = slot < u.nq;
+      const int64_t row = (int64_t)u.row0 + slot;
+      const int64_t pos = has_q ? slot_pos(a, u, slot) : -1;
+      const int ntiles = u.ntiles, nkeys = u.nkeys;
+      const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
+      const int32_t* kmap = (a.kind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
+      if (has_q) {
+        row_reset(st, tid, 128);
+        if (tid < kHeads) S.w[slot][tid] = a.w[row * kHeads + tid];
       }
-      // causal positions of my two slots (constant indices keep them in registers)
-      int64_t mypos[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) mypos[j] = (wg == 0) ? u.pos[2 * j] : u.pos[2 * j + 1];
       named_bar(bar, 128);
-      int64_t cslot_base = (int64_t)blockIdx.x * kQB;
-      for (int jt = 0; jt < u.ntiles; ++jt) {
-        bool w_ok = mbar_wait(&S.t_full[buf], eph[buf], abort_flag, a.status, 30);
-        if (!group_and(bar, 128, w_ok)) {
+      int count = 0;       // my segment's fill
+      int raised_at = 0;   // my fill at warp 0's last threshold raise
+      for (int jt = 0; jt < ntiles; ++jt) {
+        if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float v[2][64];
-        const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (j < ns) {
-            const uint32_t col = (uint32_t)(buf * 256 + (wg + 2 * j) * kHeads);
-            tmem_ld_32x32b_x32(tmem_base + lane_base + col, &v[j][0]);
-            tmem_ld_32x32b_x32(tmem_base + lane_base + col + 32, &v[j][32]);
-          }
+        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + slot * kHeads);
+        if (has_q) {
+          float v[32];
+          tmem_ld_32x32b_x32(col, v);
+          tmem_ld_wait();
+          head_accumulate32(v, w4, acc);
+          tmem_ld_32x32b_x32(col + 32, v);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.t_empty[buf]);
+          head_accumulate32(v, w4 + 8, acc);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.t_empty[buf]);
         }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.t_empty[buf]);
-        eph[buf] ^= 1u;
+        eph ^= 1u << buf;
         buf ^= 1;
-
-        const int key = (u.tile0 + jt) * kTileKeys + lq * 32 + lane;  // local key index
-        const bool in_range = key < u.nkeys;
-        int64_t kpos = key;
-        if (a.kind == 2) kpos = in_range ? (int64_t)a.key_map[(int64_t)u.seq_split * a.bank + key] : -1;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (j < ns) {
-            const int slot = wg + 2 * j;
-            const float4* w4 = reinterpret_cast<const float4*>(S.w[slot]);
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-            for (int h = 0; h < kHeads; h += 4) {
-              const float4 ww = w4[h >> 2];
-              s0 = fmaf(ww.x, fmaxf(v[j][h + 0], 0.f), s0);
-              s1 = fmaf(ww.y, fmaxf(v[j][h + 1], 0.f), s1);
-              s2 = fmaf(ww.z, fmaxf(v[j][h + 2], 0.f), s2);
-              s3 = fmaf(ww.w, fmaxf(v[j][h + 3], 0.f), s3);
-            }
-            float score = (s0 + s1) + (s2 + s3);
-            score = score + 0.0f;  // -0 -> +0
-            const bool valid = in_range && kpos >= 0 && kpos <= mypos[j];
-            if (a.dbg_scores != nullptr && valid)
-              a.dbg_scores[(int64_t)(u.row0 + slot) * a.dbg_ld + kpos] = score;
-            uint2* cand = a.cand + (cslot_base + slot) * a.cand_cap;
-            row_append(S.rows[slot], cand, score, (uint32_t)kpos, valid, lane);
+        if (has_q) {
+          const int key = key0 + jt * kTileKeys;  // local key index
+          const bool in_range = key < nkeys;
+          int64_t kpos = key;
+          if (kmap != nullptr) kpos = in_range ? (int64_t)kmap[key] : -1;
+          float score = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+          score = score + 0.0f;  // -0 -> +0
+          const bool valid = in_range && kpos >= 0 && kpos <= pos;
+          if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
+          row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
+          if (lq == 0 && count - raised_at >= 64) {
+            row_raise(st, a.k, lane, false);
+            raised_at = count;
           }
         }
-        named_bar(bar, 128);
-        if (lq < ns) row_update(S.rows[wg + 2 * lq], a.k, lane);
-        named_bar(bar, 128);
       }
+      // the whole group agrees on success before any further barrier
+      ok = group_and(bar, 128, ok);
       if (!ok) break;
-      // final selection for my slots
-      for (int j = 0; j < ns; ++j) {
-        const int slot = wg + 2 * j;
-        const uint2* cand = a.cand + (cslot_base + slot) * a.cand_cap;
+      if (has_q) {
+        if (lane == 0) st.seg_cnt[lq] = count;
+        named_bar(bar, 128);
+        if (lq == 0) row_raise(st, a.k, lane, true);
+        named_bar(bar, 128);
+        CandList cl;
+        cl.base = cand0;
+        cl.stride = seg_stride;
+        cl.nseg = 4;
+#pragma unroll
+        for (int s2 = 0; s2 < 4; ++s2) cl.cnt[s2] = st.seg_cnt[s2];
         int32_t* oi;
         float* ov;
         if (a.kind != 1) {
-          oi = a.out_idx + (int64_t)(u.row0 + slot) * a.out_ld;
-          ov = a.out_val + (int64_t)(u.row0 + slot) * a.out_ld;
+          oi = a.out_idx + row * a.out_ld;
+          ov = a.out_val + row * a.out_ld;
         } else {
-          const int64_t o = ((int64_t)(u.row0 + slot) * a.splits + u.seq_split);
+          const int64_t o = row * a.splits + u.seq_split;
           oi = a.out_idx + o * a.out_ld;
           ov = a.out_val + o * a.out_ld;
         }
-        const int cnt = row_select(S.rows[slot], cand, a.k, oi, ov, S.stage[wg], kStageCap, tid, 128, bar,
-                                   a.status);
-        if (a.kind == 1 && tid == 0) a.out_cnt[(int64_t)(u.row0 + slot) * a.splits + u.seq_split] = cnt;
+        const int cnt = row_select(st, cl, a.k, oi, ov, S.stage[slot], kStageCap, tid, 128, bar, a.status);
+        if (a.kind == 1 && tid == 0) a.out_cnt[row * a.splits + u.seq_split] = cnt;
       }
     }
   }
@@ -350,20 +394,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem_base, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tmem_base, 512);
 }
 
-int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
-                    cudaStream_t stream) {
+template <bool kDebug>
+static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_index_kernel<kDebug>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kTcSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
     configured = true;
   }
-  tc_index_kernel<<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
+  tc_index_kernel<kDebug><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
+                    cudaStream_t stream) {
+  return a.dbg_scores != nullptr ? launch_tc<true>(tmQ, tmK, a, grid, stream)
+                                 : launch_tc<false>(tmQ, tmK, a, grid, stream);
 }
 
 size_t tc_smem_bytes() { return kTcSmemBytes; }
