@@ -29,9 +29,10 @@
 namespace dsa {
 
 constexpr int kEpiWarps = 16;
-constexpr int kTcThreads = (kEpiWarps + 2) * 32;  // + TMA producer + MMA issuer
+constexpr int kTcThreads = (kEpiWarps + 3) * 32;  // + TMA producer + MMA issuer + threshold warp
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
+constexpr int kThreshWarp = kEpiWarps + 2;
 constexpr int kQB = 4;            // queries per unit
 constexpr int kHeads = 64;
 constexpr int kTileKeys = 128;
@@ -53,6 +54,7 @@ struct TcSmem {
   uint64_t t_full[2], t_empty[2];
   uint32_t tmem_base;
   int abort_flag;
+  int epi_done;  // epilogue warpgroups that left their unit loop
 };
 
 constexpr size_t kTcSmemBytes = sizeof(TcSmem) + 1024;  // + alignment slack
@@ -142,29 +144,38 @@ __device__ __forceinline__ bool group_and(int bar, int nthr, bool ok) {
   return r != 0;
 }
 
-// c + a * b on two fp32 lanes at once (fma.rn.f32x2, per-lane IEEE fma).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t ra, rb, rc, rd;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+// Two fp32 values in one 64-bit register pair, and c + a * b on both lanes
+// at once (fma.rn.f32x2: per-lane IEEE fma).  Accumulators and weights stay
+// in 64-bit form so that only the ReLU results need pairing.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ float2 unpack2(uint64_t r) {
   float2 d;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(r));
   return d;
 }
 
-// acc += w[h] * max(v[h], 0) over 32 heads (w4 points at those heads'
-// weights), four packed accumulators.
-__device__ __forceinline__ void head_accumulate32(const float (&v)[32], const float4* __restrict__ w4,
-                                                  float2 (&acc)[4]) {
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// acc += w[h] * max(v[h], 0) over 32 heads (w2 points at those heads'
+// weights, four per 16-byte load), four packed accumulators.
+__device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
+                                                  uint64_t (&acc)[4]) {
 #pragma unroll
   for (int h = 0; h < 32; h += 8) {
-    const float4 wa = w4[h >> 2], wb = w4[(h >> 2) + 1];
-    acc[0] = ffma2(make_float2(wa.x, wa.y), make_float2(fmaxf(v[h + 0], 0.f), fmaxf(v[h + 1], 0.f)), acc[0]);
-    acc[1] = ffma2(make_float2(wa.z, wa.w), make_float2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), acc[1]);
-    acc[2] = ffma2(make_float2(wb.x, wb.y), make_float2(fmaxf(v[h + 4], 0.f), fmaxf(v[h + 5], 0.f)), acc[2]);
-    acc[3] = ffma2(make_float2(wb.z, wb.w), make_float2(fmaxf(v[h + 6], 0.f), fmaxf(v[h + 7], 0.f)), acc[3]);
+    const ulonglong2 wa = w2[h >> 2], wb = w2[(h >> 2) + 1];
+    acc[0] = ffma2(wa.x, pack2(fmaxf(v[h + 0], 0.f), fmaxf(v[h + 1], 0.f)), acc[0]);
+    acc[1] = ffma2(wa.y, pack2(fmaxf(v[h + 2], 0.f), fmaxf(v[h + 3], 0.f)), acc[1]);
+    acc[2] = ffma2(wb.x, pack2(fmaxf(v[h + 4], 0.f), fmaxf(v[h + 5], 0.f)), acc[2]);
+    acc[3] = ffma2(wb.y, pack2(fmaxf(v[h + 6], 0.f), fmaxf(v[h + 7], 0.f)), acc[3]);
   }
 }
 
@@ -190,6 +201,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&S.t_empty[b], kEpiWarps);
     }
     S.abort_flag = 0;
+    S.epi_done = 0;
+    for (int q = 0; q < kQB; ++q) S.rows[q].tb = 0u;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) tmem_alloc(&S.tmem_base, 512);
@@ -208,8 +221,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int s = 0;
       uint32_t ph = 0;
       int qi = 0;
-      bool armed[kStages] = {};
-      uint32_t armed_ph[kStages] = {};
+      uint32_t armed = 0u, armed_ph = 0u;  // bit s: stage s armed / its phase
       bool ok = true;
       UnitInfo u;
       for (int round = 0; ok && unit_at(a, round, u); ++round) {
@@ -226,8 +238,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int row = u.key_row0 + (u.tile0 + j) * kTileKeys;
           for (int c = 0; c < 2; ++c)
             tma_load_2d(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row);
-          armed[s] = true;
-          armed_ph[s] = ph;
+          armed |= 1u << s;
+          armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
           if (++s == kStages) {
             s = 0;
             ph ^= 1u;
@@ -236,7 +248,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // never leave with a copy in flight
       for (int t = 0; t < kStages; ++t)
-        if (armed[t]) mbar_wait(&S.k_full[t], armed_ph[t], abort_flag, a.status, 12);
+        if ((armed >> t) & 1u) mbar_wait(&S.k_full[t], (armed_ph >> t) & 1u, abort_flag, a.status, 12);
       if (qi > 0) mbar_wait(&S.q_full, (qi - 1) & 1, abort_flag, a.status, 13);
     }
   } else if (warp == kMmaWarp) {
@@ -285,6 +297,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_commit(&S.drain);
       mbar_wait(&S.drain, 0, abort_flag, a.status, 23);
     }
+  } else if (warp == kThreshWarp) {
+    // ---------------- threshold warp ----------------
+    // Raises each active row's threshold bin from its histogram, off the
+    // epilogue's critical path, until every epilogue warpgroup is done.
+    while (*(volatile int*)&S.epi_done < 4 && !*abort_flag) {
+#pragma unroll 1
+      for (int q = 0; q < kQB; ++q) tb_raise(S.rows[q], a.k, lane);
+      __nanosleep(200);
+    }
   } else {
     // ---------------- epilogue: warpgroup `slot` follows query `slot` ----------------
     // Per tile a warp waits for its accumulator, pulls its 32 key rows x 64
@@ -298,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t seg_stride = a.cand_cap / 4;
     uint2* const cand0 = a.cand + ((int64_t)blockIdx.x * kQB + slot) * a.cand_cap;
     uint2* const my_seg = cand0 + lq * seg_stride;
-    const float4* w4 = reinterpret_cast<const float4*>(S.w[slot]);
+    const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[slot]);
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
     uint32_t eph = 0u;  // bit b: phase of accumulator buffer b
     int buf = 0;
@@ -313,31 +334,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (a.kind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
       if (has_q) {
+        if (tid == 0) tb_retire(st);
+        named_bar(bar, 128);
         row_reset(st, tid, 128);
         if (tid < kHeads) S.w[slot][tid] = a.w[row * kHeads + tid];
       }
       named_bar(bar, 128);
-      int count = 0;       // my segment's fill
-      int raised_at = 0;   // my fill at warp 0's last threshold raise
+      if (has_q && tid == 0) tb_open(st);
+      int count = 0;  // my segment's fill
       for (int jt = 0; jt < ntiles; ++jt) {
         if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + slot * kHeads);
         if (has_q) {
           float v[32];
           tmem_ld_32x32b_x32(col, v);
           tmem_ld_wait();
-          head_accumulate32(v, w4, acc);
+          head_accumulate32(v, w2, acc);
           tmem_ld_32x32b_x32(col + 32, v);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.t_empty[buf]);
-          head_accumulate32(v, w4 + 8, acc);
+          head_accumulate32(v, w2 + 8, acc);
         } else {
           tc_fence_before();
           __syncwarp();
@@ -350,15 +373,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const bool in_range = key < nkeys;
           int64_t kpos = key;
           if (kmap != nullptr) kpos = in_range ? (int64_t)kmap[key] : -1;
-          float score = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+          const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
+          float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && kpos >= 0 && kpos <= pos;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
           row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
-          if (lq == 0 && count - raised_at >= 64) {
-            row_raise(st, a.k, lane, false);
-            raised_at = count;
-          }
         }
       }
       // the whole group agrees on success before any further barrier
@@ -366,15 +386,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok) break;
       if (has_q) {
         if (lane == 0) st.seg_cnt[lq] = count;
+        if (tid == 0) tb_close(st);
         named_bar(bar, 128);
-        if (lq == 0) row_raise(st, a.k, lane, true);
+        if (lq == 0) tb_finish(st, a.k, lane);
         named_bar(bar, 128);
         CandList cl;
         cl.base = cand0;
         cl.stride = seg_stride;
-        cl.nseg = 4;
-#pragma unroll
-        for (int s2 = 0; s2 < 4; ++s2) cl.cnt[s2] = st.seg_cnt[s2];
+        cl.c0 = st.seg_cnt[0];
+        cl.c1 = st.seg_cnt[1];
+        cl.c2 = st.seg_cnt[2];
+        cl.c3 = st.seg_cnt[3];
         int32_t* oi;
         float* ov;
         if (a.kind != 1) {
@@ -389,6 +411,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (a.kind == 1 && tid == 0) a.out_cnt[row * a.splits + u.seq_split] = cnt;
       }
     }
+    if (tid == 0) atomicAdd(&S.epi_done, 1);
   }
 
   tc_fence_before();

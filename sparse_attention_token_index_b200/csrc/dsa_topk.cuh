@@ -31,27 +31,26 @@ struct RowState {
   int stage_cnt;   // select: entries staged from the b* bin
   int dsel, above, hsel;  // select: radix step result
   int top;         // highest bin holding an appended entry
-  int pad[2];
+  uint32_t tb;     // tagged threshold (segmented path): gen << 17 | active << 16 | bstar
+  int pad[1];
 };
 
-// Candidate list: nseg segments of `stride` entries each, cnt[s] used.
+constexpr uint32_t kTbActive = 1u << 16;
+
+// Candidate list: up to four segments of `stride` entries each, c0..c3 used
+// (scalars, so that the list lives in registers).
 struct CandList {
   const uint2* base;
   int64_t stride;
-  int nseg;
-  int cnt[4];
-  __device__ __forceinline__ int total() const {
-    int n = 0;
-    for (int s = 0; s < nseg; ++s) n += cnt[s];
-    return n;
-  }
+  int c0, c1, c2, c3;
+  __device__ __forceinline__ int total() const { return c0 + c1 + c2 + c3; }
   __device__ __forceinline__ uint2 at(int i) const {
-    int s = 0;
-    while (s + 1 < nseg && i >= cnt[s]) {
-      i -= cnt[s];
-      ++s;
-    }
-    return base[s * stride + i];
+    if (i < c0) return base[i];
+    i -= c0;
+    if (i < c1) return base[stride + i];
+    i -= c1;
+    if (i < c2) return base[2 * stride + i];
+    return base[3 * stride + (i - c2)];
   }
 };
 
@@ -86,44 +85,39 @@ __device__ __forceinline__ void row_append(RowState& st, uint2* __restrict__ can
 }
 
 // Appends to a warp-private segment: `count` (a register, warp-uniform) is
-// the segment's fill; only the histogram is shared.  All 32 lanes call it.
+// the segment's fill; only the histogram and the top bin are shared.  All 32
+// lanes call it.
 __device__ __forceinline__ void row_append_seg(RowState& st, uint2* __restrict__ seg, int& count, float score,
                                                uint32_t key_out, bool valid, int lane) {
   const int bin = score_bin(score);
-  const bool pass = valid && (bin >= *(volatile int*)&st.bstar);
+  const bool pass = valid && (bin >= (int)(*(volatile uint32_t*)&st.tb & 0xFFFFu));
   const unsigned m = __ballot_sync(0xffffffffu, pass);
   if (m == 0u) return;
   if (pass) {
     seg[count + __popc(m & ((1u << lane) - 1u))] = make_uint2(__float_as_uint(score), key_out);
-    const unsigned mm = __match_any_sync(m, bin);
-    if ((__ffs(mm) - 1) == lane) atomicAdd(&st.hist[bin], (uint32_t)__popc(mm));
+    atomicAdd(&st.hist[bin], 1u);
+    // the top bin rises after the histogram: a raise reading an older top
+    // only skips bins, which undercounts and stays safe
+    if (bin > *(volatile int*)&st.top) atomicMax(&st.top, bin);
   }
-  // highest occupied bin, raised after the histogram update; a raise that
-  // reads an older value only skips bins, which undercounts and stays safe
-  const int bmax = __reduce_max_sync(0xffffffffu, pass ? bin : 0);
-  if (lane == 0 && bmax > *(volatile int*)&st.top) atomicMax(&st.top, bmax);
   count += __popc(m);
 }
 
-// Raises the threshold bin to the largest b with sum_{b' >= b} hist[b'] >= k,
-// reading the histogram once, top bin first.  Safe while other warps append:
-// every value read is at most the bin's current count, so the sum it acts on
-// is never more than the true one.  With `exact` (no appends in flight) it
-// also sets cge = that sum (or the total when fewer than k were appended).
-// Called by all 32 lanes of one warp.
-__device__ __forceinline__ void row_raise(RowState& st, int k, int lane, bool exact) {
-  const int b0 = *(volatile int*)&st.bstar;
-  const int top = *(volatile int*)&st.top;
+// Largest bin b in [b0, top] with sum_{b' >= b} hist[b'] >= k, reading the
+// histogram once, top bin first (128 bins per step, 4 per lane).  Returns
+// (b, that sum), or (-1, sum over [b0, top]) when fewer than k entries lie
+// there.  Safe while other warps append: every value read is at most the
+// bin's current count, so any sum it acts on undercounts.  All 32 lanes.
+__device__ __forceinline__ int2 hist_scan(const RowState& st, int b0, int top, int k, int lane) {
   int S = 0;
   int found = -1, cge = 0;
-  // 128 bins per step, 4 consecutive bins per lane, lane 0 highest
   for (int hi = top; hi >= b0; hi -= 128) {
     int x[4];
     int t = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = hi - 4 * lane - j;
-      x[j] = (i >= b0) ? (int)*(volatile uint32_t*)&st.hist[i] : 0;
+      x[j] = (i >= b0) ? (int)*(volatile const uint32_t*)&st.hist[i] : 0;
       t += x[j];
     }
     int p = t;
@@ -137,27 +131,69 @@ __device__ __forceinline__ void row_raise(RowState& st, int k, int lane, bool ex
     if (m) {
       const int l = __ffs(m) - 1;
       if (lane == l) {
-        int c = before;
+        // the first of my four bins (highest first) where the running sum reaches k
+        int c = before, f = -1, g = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           c += x[j];
-          if (c >= k) {
-            found = hi - 4 * lane - j;
-            cge = c;
-            break;
-          }
+          const bool hit = (f < 0) && (c >= k);
+          f = hit ? hi - 4 * lane - j : f;
+          g = hit ? c : g;
         }
+        found = f;
+        cge = g;
       }
       found = __shfl_sync(0xffffffffu, found, l);
       cge = __shfl_sync(0xffffffffu, cge, l);
-      break;
+      return make_int2(found, cge);
     }
     S += __shfl_sync(0xffffffffu, p, 31);
   }
+  return make_int2(-1, S);
+}
+
+// Segmented path, unit start (one thread, then the caller zeroes the
+// histogram and calls tb_open after a barrier): retag the threshold word with
+// a new generation, inactive, so that no raise computed on the old row lands.
+__device__ __forceinline__ void tb_retire(RowState& st) {
+  const uint32_t gen = (*(volatile uint32_t*)&st.tb >> 17) + 1u;
+  *(volatile uint32_t*)&st.tb = gen << 17;
+  __threadfence_block();
+}
+
+__device__ __forceinline__ void tb_open(RowState& st) {
+  __threadfence_block();
+  *(volatile uint32_t*)&st.tb = (*(volatile uint32_t*)&st.tb & ~0xFFFFu) | kTbActive;
+  __threadfence_block();
+}
+
+// Segmented path, row end (one thread, no appends in flight): stop raises.
+__device__ __forceinline__ void tb_close(RowState& st) {
+  atomicAnd(&st.tb, ~kTbActive);
+  __threadfence_block();
+}
+
+// One pass of the threshold warp over a row: raise b* as far as the
+// histogram allows, unless the row was retired or closed meanwhile.
+__device__ __forceinline__ void tb_raise(RowState& st, int k, int lane) {
+  const uint32_t t = *(volatile uint32_t*)&st.tb;
+  if (!(t & kTbActive)) return;
+  const int b0 = (int)(t & 0xFFFFu);
+  const int top = *(volatile int*)&st.top;
+  const int2 r = hist_scan(st, b0, top, k, lane);
+  if (lane == 0 && r.x > b0) atomicCAS(&st.tb, t, (t & ~0xFFFFu) | (uint32_t)r.x);
   __syncwarp();
+}
+
+// Segmented path, row end after tb_close and a barrier: exact b* and cge for
+// row_select.  All 32 lanes of one warp.
+__device__ __forceinline__ void tb_finish(RowState& st, int k, int lane) {
+  const int b0 = (int)(*(volatile uint32_t*)&st.tb & 0xFFFFu);
+  const int top = *(volatile int*)&st.top;
+  const int2 r = hist_scan(st, b0, top, k, lane);
   if (lane == 0) {
-    if (found > b0) st.bstar = found;
-    if (exact) st.cge = found >= 0 ? cge : S;
+    st.bstar = r.x >= 0 ? r.x : b0;
+    st.cge = r.y;
   }
   __syncwarp();
 }
@@ -205,9 +241,8 @@ __device__ __forceinline__ CandList single_list(const uint2* base, int n) {
   CandList c;
   c.base = base;
   c.stride = 0;
-  c.nseg = 1;
-  c.cnt[0] = n;
-  c.cnt[1] = c.cnt[2] = c.cnt[3] = 0;
+  c.c0 = n;
+  c.c1 = c.c2 = c.c3 = 0;
   return c;
 }
 
@@ -234,6 +269,39 @@ __device__ __forceinline__ void emit(RowState& st, uint2 e, int32_t* oidx, float
   oval[p] = __uint_as_float(e.x);
 }
 
+// Warp 0 of a group: over a 256-bucket histogram h (bucket 255 ranks
+// highest), the bucket dsel holding the remaining-th best entry, the count
+// above it and the count in it, written to st.dsel / st.above / st.hsel.
+__device__ __forceinline__ void pick_digit(const uint32_t* h, int remaining, RowState& st, int lane) {
+  uint32_t c[8];
+  uint32_t tot = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = h[255 - 8 * lane - j];
+    tot += c[j];
+  }
+  uint32_t incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - tot;
+  if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
+    uint32_t cum = excl;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (cum + c[j] >= (uint32_t)remaining) {
+        st.dsel = 255 - 8 * lane - j;
+        st.above = (int)cum;
+        st.hsel = (int)c[j];
+        break;
+      }
+      cum += c[j];
+    }
+  }
+}
+
 // One MSD radix step over the entries of `src` that pass its filter and
 // match (key & mask) == prefix: histogram of the 8-bit digit at `shift`,
 // then the digit dsel holding the remaining-th best entry, the number of
@@ -252,36 +320,7 @@ __device__ void radix_level(const Src& src, int n, uint64_t prefix, uint64_t mas
     if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
   }
   named_bar(bar, nthr);
-  if (tid < 32) {
-    const int lane = tid;
-    uint32_t c[8];
-    uint32_t tot = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      c[j] = h[255 - 8 * lane - j];
-      tot += c[j];
-    }
-    uint32_t incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t excl = incl - tot;
-    if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
-      uint32_t cum = excl;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (cum + c[j] >= (uint32_t)remaining) {
-          st.dsel = 255 - 8 * lane - j;
-          st.above = (int)cum;
-          st.hsel = (int)c[j];
-          break;
-        }
-        cum += c[j];
-      }
-    }
-  }
+  if (tid < 32) pick_digit(h, remaining, st, tid);
   named_bar(bar, nthr);
   dsel = st.dsel;
   above = st.above;
@@ -320,27 +359,111 @@ __device__ void radix_emit(const Src& src, int n, int need, RowState& st, int32_
   emit_at_least(src, n, prefix, mask, st, oidx, oval, tid, nthr, bar);
 }
 
+// Warp-aggregated output: lanes with `sel` write their entry at
+// consecutive output slots.  All 32 lanes of the warp call it.
+__device__ __forceinline__ void emit_warp(RowState& st, bool sel, uint2 e, int32_t* oidx, float* oval, int lane) {
+  const unsigned m = __ballot_sync(0xffffffffu, sel);
+  if (m == 0u) return;
+  int base = 0;
+  if (lane == __ffs(m) - 1) base = atomicAdd(&st.outpos, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+  if (sel) {
+    const int p = base + __popc(m & ((1u << lane) - 1u));
+    oidx[p] = (int32_t)e.y;
+    oval[p] = __uint_as_float(e.x);
+  }
+}
+
+// Warp-aggregated staging into shared memory (entries beyond `cap` are
+// counted but dropped).
+__device__ __forceinline__ void stage_warp(RowState& st, bool stg, uint2 e, uint2* stage, int cap, int lane) {
+  const unsigned m = __ballot_sync(0xffffffffu, stg);
+  if (m == 0u) return;
+  int base = 0;
+  if (lane == __ffs(m) - 1) base = atomicAdd(&st.stage_cnt, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+  const int p = base + __popc(m & ((1u << lane) - 1u));
+  if (stg && p < cap) stage[p] = e;
+}
+
+// Calls f(e, valid) for every entry of the list, 8 independent loads in
+// flight per thread; every thread of the group runs the same number of
+// calls (valid = false past the end) so that f may use warp collectives.
+template <class F>
+__device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nthr, F&& f) {
+  constexpr int kB = 8;
+  const int cnt[4] = {c.c0, c.c1, c.c2, c.c3};
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint2* seg = c.base + s * c.stride;
+    const int n = cnt[s];
+    for (int i0 = 0; i0 < n; i0 += nthr * kB) {
+      uint2 e[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int i = i0 + j * nthr + tid;
+        e[j] = (i < n) ? seg[i] : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < kB; ++j) f(e[j], i0 + j * nthr + tid < n);
+    }
+  }
+}
+
+// Sorts n <= cap staged entries by sel_key, largest first, in shared memory
+// (bitonic network over the next power of two; padding keys are 0).
+// Group-wide (nthr threads, barrier `bar`).
+static __device__ void stage_sort(uint2* stage, int n, int tid, int nthr, int bar) {
+  int P = 1;
+  while (P < n) P <<= 1;
+  uint64_t* kk = reinterpret_cast<uint64_t*>(stage);
+  for (int i = tid; i < P; i += nthr) kk[i] = (i < n) ? sel_key(stage[i]) : 0ull;
+  named_bar(bar, nthr);
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < (P >> 1); i += nthr) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint64_t x = kk[lo], y = kk[hi];
+        if ((x < y) == up) {
+          kk[lo] = y;
+          kk[hi] = x;
+        }
+      }
+      named_bar(bar, nthr);
+    }
+  }
+}
+
+__device__ __forceinline__ uint2 key_entry(uint64_t key) {
+  const uint32_t o = (uint32_t)(key >> 32);
+  const uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+  return make_uint2(u, ~(uint32_t)key);
+}
+
 // Final selection of one row: writes min(k, visible) entries to
 // oidx[0..k), oval[0..k) (any order), pads the rest with -1 / -inf, and
-// returns the number of real entries.  Group-wide call (nthr threads).
+// returns the number of real entries.  Group-wide call (nthr threads, a
+// multiple of 32).  Expects st.bstar / st.cge exact (no appends in flight).
 static __device__ __noinline__ int row_select(RowState& st, const CandList& cand, int k,
                                               int32_t* __restrict__ oidx, float* __restrict__ oval,
                                               uint2* __restrict__ stage, int stage_cap, int tid, int nthr, int bar,
                                               int* status) {
+  const int lane = tid & 31;
   named_bar(bar, nthr);
   const int n = cand.total(), bstar = st.bstar, cge = st.cge;
+  const int hb = (int)st.hist[bstar];
   named_bar(bar, nthr);
   if (tid == 0) {
     st.outpos = 0;
     st.stage_cnt = 0;
   }
+  named_bar(bar, nthr);
   if (cge < k) {
     // b* never moved: every visible key was appended (n == cge < k)
-    for (int i = tid; i < n; i += nthr) {
-      const uint2 e = cand.at(i);
-      oidx[i] = (int32_t)e.y;
-      oval[i] = __uint_as_float(e.x);
-    }
+    for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) { emit_warp(st, v, e, oidx, oval, lane); });
+    named_bar(bar, nthr);
     for (int i = n + tid; i < k; i += nthr) {
       oidx[i] = -1;
       oval[i] = __int_as_float(0xff800000);
@@ -348,35 +471,82 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
     named_bar(bar, nthr);
     return n;
   }
-  const int hb = (int)st.hist[bstar];
   const int need = k - (cge - hb);
-  named_bar(bar, nthr);
   // entries above the threshold bin are selected; the bin itself is staged
-  for (int i = tid; i < n; i += nthr) {
-    const uint2 e = cand.at(i);
-    const int b = score_bin(__uint_as_float(e.x));
-    if (b > bstar) {
-      emit(st, e, oidx, oval);
-    } else if (b == bstar) {
-      const int s = atomicAdd(&st.stage_cnt, 1);
-      if (s < stage_cap) stage[s] = e;
-    }
-  }
+  for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
+    const int b = v ? score_bin(__uint_as_float(e.x)) : -1;
+    emit_warp(st, b > bstar, e, oidx, oval, lane);
+    stage_warp(st, b == bstar, e, stage, stage_cap, lane);
+  });
   named_bar(bar, nthr);
   const int ns = st.stage_cnt;
   if (tid == 0 && (ns != hb || st.outpos != cge - hb)) report_error(status, DSA_ERR_INTERNAL, 1);
   if (ns <= stage_cap) {
-    radix_emit(StageSrc{stage}, ns, need, st, oidx, oval, tid, nthr, bar);
+    stage_sort(stage, ns, tid, nthr, bar);
+    const uint64_t* kk = reinterpret_cast<const uint64_t*>(stage);
+    const int base = cge - hb;
+    for (int i = tid; i < need; i += nthr) {
+      const uint2 e = key_entry(kk[i]);
+      oidx[base + i] = (int32_t)e.y;
+      oval[base + i] = __uint_as_float(e.x);
+    }
+    named_bar(bar, nthr);
     return k;
   }
-  // The threshold bin holds more entries than the stage: narrow it with
-  // radix steps over the candidate list until the selected sub-bucket fits.
+  // The threshold bin holds more entries than the stage.  Inside bins
+  // 1..1022 every score is a positive normal float with the same exponent
+  // and top 4 mantissa bits, so its next 8 bits (18..11) order the bin:
+  // one counting pass picks the sub-bucket holding the cut, one pass emits
+  // the sub-buckets above it and stages the cut sub-bucket.
+  if (bstar > 0 && bstar < kBins - 1) {
+    uint32_t* h = st.hist;
+    for (int i = tid; i < 256; i += nthr) h[i] = 0u;
+    named_bar(bar, nthr);
+    for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
+      if (v && score_bin(__uint_as_float(e.x)) == bstar) atomicAdd(&h[(e.x >> 11) & 255u], 1u);
+    });
+    named_bar(bar, nthr);
+    if (tid < 32) pick_digit(h, need, st, tid);
+    named_bar(bar, nthr);
+    const int dsel = st.dsel, above = st.above, hsel = st.hsel;
+    if (hsel <= stage_cap) {
+      named_bar(bar, nthr);
+      if (tid == 0) st.stage_cnt = 0;
+      named_bar(bar, nthr);
+      for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
+        const bool inb = v && score_bin(__uint_as_float(e.x)) == bstar;
+        const int dg = (int)((e.x >> 11) & 255u);
+        emit_warp(st, inb && dg > dsel, e, oidx, oval, lane);
+        stage_warp(st, inb && dg == dsel, e, stage, stage_cap, lane);
+      });
+      named_bar(bar, nthr);
+      const int base = st.outpos;
+      if (tid == 0 && (st.stage_cnt != hsel || base != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
+      stage_sort(stage, hsel, tid, nthr, bar);
+      const uint64_t* kk = reinterpret_cast<const uint64_t*>(stage);
+      for (int i = tid; i < need - above; i += nthr) {
+        const uint2 e = key_entry(kk[i]);
+        oidx[base + i] = (int32_t)e.y;
+        oval[base + i] = __uint_as_float(e.x);
+      }
+      named_bar(bar, nthr);
+      return k;
+    }
+    named_bar(bar, nthr);
+    if (tid == 0) {
+      st.outpos = cge - hb;  // nothing of the bin emitted yet
+      st.stage_cnt = 0;
+    }
+    named_bar(bar, nthr);
+  }
+  // Still too many (massive ties): radix steps over the whole 64-bit key.
   const BinSrc gsrc{cand, bstar};
+  const int n_all = n;
   uint64_t prefix = 0, mask = 0;
   int remaining = need;
   for (int shift = 56; shift >= 0; shift -= 8) {
     int dsel, above, hsel;
-    radix_level(gsrc, n, prefix, mask, shift, remaining, st, tid, nthr, bar, dsel, above, hsel);
+    radix_level(gsrc, n_all, prefix, mask, shift, remaining, st, tid, nthr, bar, dsel, above, hsel);
     remaining -= above;
     prefix |= (uint64_t)dsel << shift;
     mask |= (uint64_t)0xFFu << shift;
@@ -384,7 +554,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
     if (hsel <= stage_cap) {
       if (tid == 0) st.stage_cnt = 0;
       named_bar(bar, nthr);
-      for (int i = tid; i < n; i += nthr) {
+      for (int i = tid; i < n_all; i += nthr) {
         uint2 e;
         if (!gsrc.get(i, e)) continue;
         const uint64_t km = sel_key(e) & mask;
@@ -399,7 +569,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
       return k;
     }
   }
-  emit_at_least(gsrc, n, prefix, mask, st, oidx, oval, tid, nthr, bar);
+  emit_at_least(gsrc, n_all, prefix, mask, st, oidx, oval, tid, nthr, bar);
   return k;
 }
 
