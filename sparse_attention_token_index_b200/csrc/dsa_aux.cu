@@ -177,7 +177,7 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
 // ---------------------------------------------------------------------------
 struct MergeSmem {
   RowState st;
-  uint2 stage[2048];
+  uint2 stage[1024];
 };
 
 __global__ void __launch_bounds__(128) decode_merge_kernel(const int32_t* __restrict__ part_idx,
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const int32_t* __rest
     if (tid < 32) row_update(M.st, k, lane);
     named_bar(1, 128);
   }
-  row_select(M.st, single_list(cand, M.st.cnt), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k, M.stage, 2048, tid, 128, 1,
+  row_select(M.st, single_list(cand, M.st.cnt), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k, M.stage, 1024, tid, 128, 1,
              status);
 }
 

@@ -374,64 +374,93 @@ __device__ __forceinline__ void emit_warp(RowState& st, bool sel, uint2 e, int32
   }
 }
 
-// Warp-aggregated staging into shared memory (entries beyond `cap` are
-// counted but dropped).
-__device__ __forceinline__ void stage_warp(RowState& st, bool stg, uint2 e, uint2* stage, int cap, int lane) {
-  const unsigned m = __ballot_sync(0xffffffffu, stg);
-  if (m == 0u) return;
-  int base = 0;
-  if (lane == __ffs(m) - 1) base = atomicAdd(&st.stage_cnt, __popc(m));
-  base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
-  const int p = base + __popc(m & ((1u << lane) - 1u));
-  if (stg && p < cap) stage[p] = e;
+__device__ __forceinline__ int warp_excl_scan(int x, int lane, int& total) {
+  int p = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, p, o);
+    if (lane >= o) p += y;
+  }
+  total = __shfl_sync(0xffffffffu, p, 31);
+  return p - x;
 }
 
-// Calls f(e, valid) for every entry of the list, 8 independent loads in
-// flight per thread; every thread of the group runs the same number of
-// calls (valid = false past the end) so that f may use warp collectives.
+constexpr int kBatch = 8;
+
+// Calls f(e, valid) for every entry of the list, kBatch independent loads in
+// flight per thread; every thread of the group runs the same number of calls
+// (valid = false past the end) so that f may use warp collectives.
 template <class F>
 __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nthr, F&& f) {
-  constexpr int kB = 8;
   const int cnt[4] = {c.c0, c.c1, c.c2, c.c3};
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     const uint2* seg = c.base + s * c.stride;
     const int n = cnt[s];
-    for (int i0 = 0; i0 < n; i0 += nthr * kB) {
-      uint2 e[kB];
+    for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
+      uint2 e[kBatch];
 #pragma unroll
-      for (int j = 0; j < kB; ++j) {
+      for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * nthr + tid;
         e[j] = (i < n) ? seg[i] : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int j = 0; j < kB; ++j) f(e[j], i0 + j * nthr + tid < n);
+      for (int j = 0; j < kBatch; ++j) f(e[j], i0 + j * nthr + tid < n);
     }
   }
 }
 
-// Sorts n <= cap staged entries by sel_key, largest first, in shared memory
-// (bitonic network over the next power of two; padding keys are 0).
-// Group-wide (nthr threads, barrier `bar`).
-static __device__ void stage_sort(uint2* stage, int n, int tid, int nthr, int bar) {
-  int P = 1;
-  while (P < n) P <<= 1;
-  uint64_t* kk = reinterpret_cast<uint64_t*>(stage);
-  for (int i = tid; i < P; i += nthr) kk[i] = (i < n) ? sel_key(stage[i]) : 0ull;
-  named_bar(bar, nthr);
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < (P >> 1); i += nthr) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const uint64_t x = kk[lo], y = kk[hi];
-        if ((x < y) == up) {
-          kk[lo] = y;
-          kk[hi] = x;
+// Streams the candidate list in batches of kBatch entries per thread and
+// classifies each entry with cls(e) -> 0 drop, 1 emit to the output, 2 stage
+// into shared memory (entries beyond stage_cap are counted, not stored).
+// Output and stage slots are taken with one warp scan and one atomic per
+// warp and batch.  All nthr threads call it (nthr a multiple of 32).
+template <class Cls>
+__device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nthr, RowState& st, int32_t* oidx,
+                                              float* oval, uint2* stage, int stage_cap, Cls&& cls) {
+  const int lane = tid & 31;
+  const int cnt[4] = {c.c0, c.c1, c.c2, c.c3};
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint2* seg = c.base + s * c.stride;
+    const int n = cnt[s];
+    for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
+      uint2 e[kBatch];
+      int cat[kBatch];
+      int ne = 0, ns = 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int i = i0 + j * nthr + tid;
+        e[j] = (i < n) ? seg[i] : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int i = i0 + j * nthr + tid;
+        cat[j] = (i < n) ? cls(e[j]) : 0;
+        ne += cat[j] == 1;
+        ns += cat[j] == 2;
+      }
+      int te, ts;
+      int pe = warp_excl_scan(ne, lane, te);
+      int ps = warp_excl_scan(ns, lane, ts);
+      int be = 0, bs = 0;
+      if (lane == 0) {
+        if (te) be = atomicAdd(&st.outpos, te);
+        if (ts) bs = atomicAdd(&st.stage_cnt, ts);
+      }
+      be = __shfl_sync(0xffffffffu, be, 0) + pe;
+      bs = __shfl_sync(0xffffffffu, bs, 0) + ps;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (cat[j] == 1) {
+          oidx[be] = (int32_t)e[j].y;
+          oval[be] = __uint_as_float(e[j].x);
+          ++be;
+        } else if (cat[j] == 2) {
+          if (bs < stage_cap) stage[bs] = e[j];
+          ++bs;
         }
       }
-      named_bar(bar, nthr);
     }
   }
 }
@@ -442,15 +471,90 @@ __device__ __forceinline__ uint2 key_entry(uint64_t key) {
   return make_uint2(u, ~(uint32_t)key);
 }
 
+constexpr int kResolvePerThread = 8;  // staged entries per thread: stage_cap <= 8 * nthr
+
+// Emits the `need` best of the ns staged entries (need <= ns <= stage_cap).
+// Entries move into registers; MSD digit steps of 8 bits, starting at bit
+// `shift` of the 64-bit key (bits above it are equal for all entries or
+// already decided), drop or emit whole digit buckets until at most 128
+// entries remain undecided; those are ranked exactly by counting.
+// Group-wide (nthr threads, barrier `bar`).
+static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, int ns, int need, int shift, int32_t* oidx,
+                                           float* oval, int tid, int nthr, int bar) {
+  const int lane = tid & 31;
+  uint64_t key[kResolvePerThread];
+  bool live[kResolvePerThread];
+#pragma unroll
+  for (int j = 0; j < kResolvePerThread; ++j) {
+    const int i = j * nthr + tid;
+    live[j] = i < ns;
+    key[j] = live[j] ? sel_key(stage[i]) : 0ull;
+  }
+  int remaining = need, nlive = ns;
+  uint32_t* h = st.hist;
+  while (nlive > 128 && shift >= 0) {
+    named_bar(bar, nthr);
+    for (int i = tid; i < 256; i += nthr) h[i] = 0u;
+    named_bar(bar, nthr);
+#pragma unroll
+    for (int j = 0; j < kResolvePerThread; ++j)
+      if (live[j]) atomicAdd(&h[(key[j] >> shift) & 255u], 1u);
+    named_bar(bar, nthr);
+    if (tid < 32) pick_digit(h, remaining, st, tid);
+    named_bar(bar, nthr);
+    const int dsel = st.dsel, above = st.above, hsel = st.hsel;
+#pragma unroll
+    for (int j = 0; j < kResolvePerThread; ++j) {
+      const int d = live[j] ? (int)((key[j] >> shift) & 255u) : -1;
+      emit_warp(st, d > dsel, key_entry(key[j]), oidx, oval, lane);
+      live[j] = (d == dsel);
+    }
+    remaining -= above;
+    nlive = hsel;
+    shift -= 8;
+  }
+  // at most 128 undecided entries: compact them, rank each by counting
+  named_bar(bar, nthr);
+  if (tid == 0) st.stage_cnt = 0;
+  named_bar(bar, nthr);
+  uint64_t* kk = reinterpret_cast<uint64_t*>(stage);
+#pragma unroll
+  for (int j = 0; j < kResolvePerThread; ++j) {
+    const unsigned m = __ballot_sync(0xffffffffu, live[j]);
+    int base = 0;
+    if (m && lane == __ffs(m) - 1) base = atomicAdd(&st.stage_cnt, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, m ? __ffs(m) - 1 : 0);
+    if (live[j]) kk[base + __popc(m & ((1u << lane) - 1u))] = key[j];
+  }
+  named_bar(bar, nthr);
+  if (tid < nlive) {
+    const uint64_t mine = kk[tid];
+    int rank = 0;
+    for (int j = 0; j < nlive; ++j) rank += kk[j] > mine;
+    if (rank < remaining) {
+      const uint2 e = key_entry(mine);
+      const int p = atomicAdd(&st.outpos, 1);
+      oidx[p] = (int32_t)e.y;
+      oval[p] = __uint_as_float(e.x);
+    }
+  }
+  named_bar(bar, nthr);
+}
+
+// First key bit below a threshold bin's resolution: inside bins 1..1022 all
+// scores share sign, exponent and top 4 mantissa bits (key bits 63..51);
+// the clamped end bins share nothing.
+__device__ __forceinline__ int digit_shift_below(int bin) { return (bin > 0 && bin < kBins - 1) ? 43 : 56; }
+
 // Final selection of one row: writes min(k, visible) entries to
 // oidx[0..k), oval[0..k) (any order), pads the rest with -1 / -inf, and
 // returns the number of real entries.  Group-wide call (nthr threads, a
-// multiple of 32).  Expects st.bstar / st.cge exact (no appends in flight).
+// multiple of 32, stage_cap <= 8 * nthr).  Expects st.bstar / st.cge exact
+// (no appends in flight).
 static __device__ __noinline__ int row_select(RowState& st, const CandList& cand, int k,
                                               int32_t* __restrict__ oidx, float* __restrict__ oval,
                                               uint2* __restrict__ stage, int stage_cap, int tid, int nthr, int bar,
                                               int* status) {
-  const int lane = tid & 31;
   named_bar(bar, nthr);
   const int n = cand.total(), bstar = st.bstar, cge = st.cge;
   const int hb = (int)st.hist[bstar];
@@ -462,7 +566,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
   named_bar(bar, nthr);
   if (cge < k) {
     // b* never moved: every visible key was appended (n == cge < k)
-    for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) { emit_warp(st, v, e, oidx, oval, lane); });
+    classify_pass(cand, tid, nthr, st, oidx, oval, stage, 0, [](uint2) { return 1; });
     named_bar(bar, nthr);
     for (int i = n + tid; i < k; i += nthr) {
       oidx[i] = -1;
@@ -473,33 +577,24 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
   }
   const int need = k - (cge - hb);
   // entries above the threshold bin are selected; the bin itself is staged
-  for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
-    const int b = v ? score_bin(__uint_as_float(e.x)) : -1;
-    emit_warp(st, b > bstar, e, oidx, oval, lane);
-    stage_warp(st, b == bstar, e, stage, stage_cap, lane);
+  classify_pass(cand, tid, nthr, st, oidx, oval, stage, stage_cap, [bstar](uint2 e) {
+    const int b = score_bin(__uint_as_float(e.x));
+    return b > bstar ? 1 : (b == bstar ? 2 : 0);
   });
   named_bar(bar, nthr);
   const int ns = st.stage_cnt;
   if (tid == 0 && (ns != hb || st.outpos != cge - hb)) report_error(status, DSA_ERR_INTERNAL, 1);
   if (ns <= stage_cap) {
-    stage_sort(stage, ns, tid, nthr, bar);
-    const uint64_t* kk = reinterpret_cast<const uint64_t*>(stage);
-    const int base = cge - hb;
-    for (int i = tid; i < need; i += nthr) {
-      const uint2 e = key_entry(kk[i]);
-      oidx[base + i] = (int32_t)e.y;
-      oval[base + i] = __uint_as_float(e.x);
-    }
-    named_bar(bar, nthr);
+    stage_resolve(st, stage, ns, need, digit_shift_below(bstar), oidx, oval, tid, nthr, bar);
     return k;
   }
   // The threshold bin holds more entries than the stage.  Inside bins
-  // 1..1022 every score is a positive normal float with the same exponent
-  // and top 4 mantissa bits, so its next 8 bits (18..11) order the bin:
-  // one counting pass picks the sub-bucket holding the cut, one pass emits
-  // the sub-buckets above it and stages the cut sub-bucket.
+  // 1..1022 the score bits 18..11 order the bin: one counting pass picks the
+  // sub-bucket holding the cut, one pass emits the sub-buckets above it and
+  // stages the cut sub-bucket.
   if (bstar > 0 && bstar < kBins - 1) {
     uint32_t* h = st.hist;
+    named_bar(bar, nthr);
     for (int i = tid; i < 256; i += nthr) h[i] = 0u;
     named_bar(bar, nthr);
     for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
@@ -513,23 +608,14 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
       named_bar(bar, nthr);
       if (tid == 0) st.stage_cnt = 0;
       named_bar(bar, nthr);
-      for_each_cand(cand, tid, nthr, [&](uint2 e, bool v) {
-        const bool inb = v && score_bin(__uint_as_float(e.x)) == bstar;
+      classify_pass(cand, tid, nthr, st, oidx, oval, stage, stage_cap, [bstar, dsel](uint2 e) {
+        if (score_bin(__uint_as_float(e.x)) != bstar) return 0;
         const int dg = (int)((e.x >> 11) & 255u);
-        emit_warp(st, inb && dg > dsel, e, oidx, oval, lane);
-        stage_warp(st, inb && dg == dsel, e, stage, stage_cap, lane);
+        return dg > dsel ? 1 : (dg == dsel ? 2 : 0);
       });
       named_bar(bar, nthr);
-      const int base = st.outpos;
-      if (tid == 0 && (st.stage_cnt != hsel || base != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
-      stage_sort(stage, hsel, tid, nthr, bar);
-      const uint64_t* kk = reinterpret_cast<const uint64_t*>(stage);
-      for (int i = tid; i < need - above; i += nthr) {
-        const uint2 e = key_entry(kk[i]);
-        oidx[base + i] = (int32_t)e.y;
-        oval[base + i] = __uint_as_float(e.x);
-      }
-      named_bar(bar, nthr);
+      if (tid == 0 && (st.stage_cnt != hsel || st.outpos != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
+      stage_resolve(st, stage, hsel, need - above, 35, oidx, oval, tid, nthr, bar);
       return k;
     }
     named_bar(bar, nthr);
@@ -565,7 +651,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
         }
       }
       named_bar(bar, nthr);
-      radix_emit(StageSrc{stage}, hsel, remaining, st, oidx, oval, tid, nthr, bar);
+      stage_resolve(st, stage, hsel, remaining, shift - 8, oidx, oval, tid, nthr, bar);
       return k;
     }
   }
