@@ -139,3 +139,21 @@ def test_dense_full_size_sampled():
     rows = sorted(set([0, 1, 127, 128, 2046, 2047, 2048, 4095, 16383, T - 2, T - 1]
                       + rng.integers(0, T, 9).tolist()))
     _run_and_check(inp, 2048, rows=rows, what="dense 32K")
+
+
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_all_keys_identical(path):
+    # every score of a row is equal: the selection must be the k lowest key
+    # indices (more ties than the staging buffer holds)
+    T, N, k = 8, 3000, 100
+    H, d = (64, 128) if path == "tc" else (4, 16)
+    g = torch.Generator(device=DEV).manual_seed(41)
+    q = torch.randn(T, H, d, generator=g, device=DEV)
+    K = torch.randn(1, d, generator=g, device=DEV).expand(N, d).contiguous()
+    w = torch.rand(T, H, generator=g, device=DEV)
+    if path == "tc":
+        q, K = q.to(torch.bfloat16), K.to(torch.bfloat16)
+    idx, val = dsa.dsa_index_dense(q, w, K, k, check=True)
+    for t in range(T):
+        assert sorted(idx[t].tolist()) == list(range(k)), t
+        assert len(set(val[t].tolist())) == 1
