@@ -158,6 +158,32 @@ int dsa_index_decode(const void* Q, const float* w, const void* K,
                      size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Dense indexer that allocates nothing (the pages have no counterpart: this
+ * is an integration aid).  For callers that cannot hand the library a
+ * workspace — code running inside a host application that reserved all
+ * device memory up front (a serving engine sizing its KV cache to the whole
+ * GPU, say), or a loop where a late cudaMalloc may fail under memory pressure
+ * or stall the device.
+ *   Same inputs, outputs and results as dsa_index_dense with bf16 Q/K,
+ *   H = 64 and d = 128 (other shapes: DSA_ERR_UNSUPPORTED).  No workspace:
+ *   the scratch (a status word and per-CTA candidate lists) lives in a fixed
+ *   32 MiB array in device memory that every GPU loading this library holds
+ *   until the process exits.  Rows need 4 * round_up(N, 128) * 8 bytes per
+ *   CTA; the grid shrinks to fit, and N above about 1.04 million keys
+ *   returns DSA_ERR_WORKSPACE.
+ *   The first call on a device looks up that device's copy of the array
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   The call is synchronous: it waits for `stream` and returns the device
+ *   status of this call (DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_INTERNAL).
+ *   Every call on a device shares the one array: calls that overlap on the
+ *   GPU (other streams, other host threads) race; serialise them.
+ *   It calls no allocation routine (no cudaMalloc, no cudaFree).
+ * ---------------------------------------------------------------------- */
+int dsa_index_dense_static(const void* Q, const float* w, const void* K, int T,
+                           int N, int H, int d, int64_t q_pos0, int k,
+                           int32_t* idx, float* val, void* stream);
+
+/* ------------------------------------------------------------------------
  * Test aid: the full score matrix S [T, N] fp32 of the dense call (the same
  * kernel and epilogue arithmetic; entries with s > p_t hold -inf).
  * Needs T * N <= 2^26.  Uses the dense workspace.

@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     dsa_index_group,
     dsa_index_decode,
     dsa_debug_scores,
+    dsa_index_dense_static,
     dsa_check_status,
     dense_workspace_bytes,
     group_workspace_bytes,

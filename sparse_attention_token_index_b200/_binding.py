@@ -21,7 +21,7 @@ EXPORTED_SYMBOLS = (
     "dsa_index_dense_workspace_size", "dsa_index_dense",
     "dsa_index_group_workspace_size", "dsa_index_group",
     "dsa_index_decode_workspace_size", "dsa_index_decode",
-    "dsa_debug_scores",
+    "dsa_debug_scores", "dsa_index_dense_static",
 )
 
 
@@ -50,6 +50,8 @@ _SIGS = {
                                   _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_sz, _vp]),
     "dsa_debug_scores": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
                                   _vp, _vp, _c_sz, _vp]),
+    "dsa_index_dense_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _vp, _vp,
+                                        _vp]),
 }
 
 
@@ -257,3 +259,24 @@ def dsa_debug_scores(Q, w, K, q_pos0: Optional[int] = None, K_scale=None, worksp
     if check:
         dsa_check_status(ws, stream)
     return S
+
+
+def dsa_index_dense_static(Q: torch.Tensor, w: torch.Tensor, K: torch.Tensor, k: int, q_pos0: Optional[int] = None,
+                           out=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Dense indexer that allocates no device memory (bf16 Q/K, H = 64, d = 128).
+
+    For callers that cannot provide a workspace: the library's fixed scratch
+    array is used instead.  Synchronous; calls on one device must not
+    overlap.  ``out`` = (idx, val) preallocated by the caller, else
+    allocated here (by torch, outside the library).
+    """
+    _need_cuda(Q, w, K)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    if Q.dtype != torch.bfloat16 or K.dtype != torch.bfloat16:
+        raise TypeError("dsa_index_dense_static takes bf16 Q and K")
+    idx, val = _outputs(T, k, Q.device, out)
+    _check(lib().dsa_index_dense_static(_ptr(Q), _ptr(w), _ptr(K), T, N, H, d, q_pos0, k, _ptr(idx), _ptr(val),
+                                        _stream(stream)), "dsa_index_dense_static")
+    return idx, val
