@@ -88,8 +88,16 @@ struct Layout {
   }
 };
 
+// bf16 queries with bf16 or fp8 keys at H = 64, d = 128 run on the tensor
+// cores; fp8 keys are first widened to bf16 (exactly) in the workspace and
+// their per-key scale is applied to the score in the epilogue.
 bool use_tc(int H, int d, int q_dtype, int k_dtype) {
-  return q_dtype == DSA_DTYPE_BF16 && k_dtype == DSA_DTYPE_BF16 && H == 64 && d == 128;
+  return q_dtype == DSA_DTYPE_BF16 && (k_dtype == DSA_DTYPE_BF16 || k_dtype == DSA_DTYPE_FP8_E4M3) && H == 64 &&
+         d == 128;
+}
+
+bool needs_widen(int H, int d, int q_dtype, int k_dtype) {
+  return use_tc(H, d, q_dtype, k_dtype) && k_dtype == DSA_DTYPE_FP8_E4M3;
 }
 
 int check_common(int H, int d, int k, int q_dtype, int k_dtype) {
@@ -106,6 +114,15 @@ int simt_grid(const DeviceInfo& di, int64_t tasks) {
   int64_t g = (tasks + 1) / 2;
   const int64_t cap = (int64_t)di.sms * 4;
   return (int)(g < cap ? (g < 1 ? 1 : g) : cap);
+}
+
+// Offset of the widened (bf16) copy of fp8 keys, taken first in every plan.
+size_t take_widen(Layout& L, int64_t n_keys, int H, int d, int q_dtype, int k_dtype) {
+  return needs_widen(H, d, q_dtype, k_dtype) ? L.take((size_t)n_keys * d * 2) : 0;
+}
+
+int widen_keys(const void* K, int64_t n_keys, int d, uint8_t* ws, size_t off, cudaStream_t st) {
+  return launch_e4m3_to_bf16(static_cast<const uint8_t*>(K), n_keys * d, ws + off, st);
 }
 
 // Dense / proxy-scan workspace pieces.
@@ -133,6 +150,8 @@ DensePlan plan_dense(const DeviceInfo& di, int T, int N, int H, int d, int q_dty
   return p;
 }
 
+// K / k_dtype: for the tensor-core path the keys as bf16 (fp8 keys already
+// widened) with K_scale their per-key scale or null.
 int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, const float* w, const void* K,
                    const float* K_scale, int n_rows, int N, int H, int d, int64_t pos_base, int64_t pos_mul,
                    int64_t pos_add, int64_t pos_clamp, int k, int q_dtype, int k_dtype, int32_t* idx, float* val,
@@ -148,6 +167,7 @@ int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, cons
     TcArgs a;
     memset(&a, 0, sizeof(a));
     a.kind = 0;
+    a.k_scale = K_scale;
     a.n_rows = n_rows;
     a.n_units = (n_rows + 3) / 4;
     a.k = k;
@@ -248,6 +268,7 @@ int dsa_index_dense_workspace_size(int T, int N, int H, int d, int k, int q_dtyp
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   Layout L;
+  take_widen(L, N, H, d, q_dtype, k_dtype);
   *bytes = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L).total;
   return DSA_OK;
 }
@@ -261,11 +282,18 @@ int dsa_index_dense(const void* Q, const float* w, const void* K, const float* K
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   Layout L;
+  const size_t wo = take_widen(L, N, H, d, q_dtype, k_dtype);
   DensePlan p = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L);
   if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, N, d, ws, wo, st)) != DSA_OK) return r;
+    return run_dense_rows(di, p, Q, w, ws + wo, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype,
+                          DSA_DTYPE_BF16, idx, val, ws, nullptr, 0, st);
+  }
   return run_dense_rows(di, p, Q, w, K, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype, k_dtype,
-                        idx, val, static_cast<uint8_t*>(workspace), nullptr, 0,
-                        static_cast<cudaStream_t>(stream));
+                        idx, val, ws, nullptr, 0, st);
 }
 
 int dsa_debug_scores(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
@@ -279,6 +307,7 @@ int dsa_debug_scores(const void* Q, const float* w, const void* K, const float* 
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   Layout L;
+  const size_t wo = take_widen(L, N, H, d, q_dtype, k_dtype);
   DensePlan p = plan_dense(di, T, N, H, d, q_dtype, k_dtype, L);
   // the top-1 outputs of this run go to scratch behind the plan
   const size_t oi = L.take((size_t)T * sizeof(int32_t));
@@ -287,7 +316,14 @@ int dsa_debug_scores(const void* Q, const float* w, const void* K, const float* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((r = launch_fill_scores(S, (int64_t)T * N, st)) != DSA_OK) return r;
-  return run_dense_rows(di, p, Q, w, K, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype, k_dtype,
+  const void* Kuse = K;
+  int kd = k_dtype;
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, N, d, ws, wo, st)) != DSA_OK) return r;
+    Kuse = ws + wo;
+    kd = DSA_DTYPE_BF16;
+  }
+  return run_dense_rows(di, p, Q, w, Kuse, K_scale, T, N, H, d, q_pos0, 1, 0, (int64_t)T - 1, k, q_dtype, kd,
                         reinterpret_cast<int32_t*>(ws + oi), reinterpret_cast<float*>(ws + ov), ws, S, N, st);
 }
 
@@ -299,6 +335,7 @@ int dsa_debug_scores(const void* Q, const float* w, const void* K, const float* 
 namespace {
 
 struct GroupPlan {
+  size_t widen_off;
   int ng;
   size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off;
   DensePlan scan;       // proxy scan
@@ -311,6 +348,7 @@ struct GroupPlan {
 int plan_group(const DeviceInfo& di, int T, int N, int H, int d, int k, int G, int B, int q_dtype, int k_dtype,
                GroupPlan& gp) {
   Layout L;
+  gp.widen_off = take_widen(L, N, H, d, q_dtype, k_dtype);
   gp.ng = (T + G - 1) / G;
   gp.qbar_off = L.take((size_t)gp.ng * H * d * elt_size(q_dtype));
   gp.wbar_off = L.take((size_t)gp.ng * H * sizeof(float));
@@ -322,7 +360,7 @@ int plan_group(const DeviceInfo& di, int T, int N, int H, int d, int k, int G, i
   gp.ref_cap = ((int64_t)B + 127) / 128 * 128;
   gp.ref_grid = 0;
   if (use_tc(H, d, q_dtype, k_dtype)) {
-    gp.kg_off = L.take((size_t)gp.ng * B * d * elt_size(k_dtype));
+    gp.kg_off = L.take((size_t)gp.ng * B * d * 2);  // gathered bank keys, bf16
     const int mblocks = (G + 3) / 4;
     const int64_t units = (int64_t)gp.ng * mblocks;
     gp.ref_grid = units < di.sms ? (int)units : di.sms;
@@ -372,6 +410,12 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   float* wbar = proxy_w ? proxy_w : reinterpret_cast<float*>(ws + gp.wbar_off);
   int32_t* bi = bank_idx ? bank_idx : reinterpret_cast<int32_t*>(ws + gp.bidx_off);
   float* bv = bank_val ? bank_val : reinterpret_cast<float*>(ws + gp.bval_off);
+  // 0. fp8 keys: exact bf16 copy, the per-key scale goes to the epilogue
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, N, d, ws, gp.widen_off, st)) != DSA_OK) return r;
+    K = ws + gp.widen_off;
+    k_dtype = DSA_DTYPE_BF16;
+  }
   // 1. proxies
   if ((r = launch_proxy_mean(Q, w, T, H, d, group, q_dtype, qbar, wbar, st)) != DSA_OK) return r;
   // 2. one full-prefix scan per proxy: bank = its top-`bank` keys
@@ -392,6 +436,7 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   TcArgs a;
   memset(&a, 0, sizeof(a));
   a.kind = 2;
+  a.k_scale = K_scale;
   a.n_rows = T;
   a.mblocks = (group + 3) / 4;
   a.n_units = gp.ng * a.mblocks;
@@ -416,6 +461,7 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
 namespace {
 
 struct DecodePlan {
+  size_t widen_off;
   bool tc;
   int splits, tiles_per_split;
   int grid;
@@ -423,8 +469,8 @@ struct DecodePlan {
   size_t cand_off, pidx_off, pval_off, pcnt_off, mscr_off, total;
 };
 
-void plan_decode(const DeviceInfo& di, int B, int total_q, int max_keys, int H, int d, int k, int q_dtype,
-                 int k_dtype, DecodePlan& p) {
+void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, int max_keys, int H, int d, int k,
+                 int q_dtype, int k_dtype, DecodePlan& p) {
   p.tc = use_tc(H, d, q_dtype, k_dtype);
   const int tiles_max = (max_keys + 127) / 128;
   // choose the split count minimising (rounds of units) x (tiles per unit + a
@@ -446,6 +492,7 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int max_keys, int H, 
   p.tiles_per_split = (tiles_max + best_s - 1) / best_s;
   p.cand_cap = (int64_t)p.tiles_per_split * 128;
   Layout L;
+  p.widen_off = take_widen(L, total_keys, H, d, q_dtype, k_dtype);
   if (p.tc) {
     const int64_t units = (int64_t)B * p.splits;
     p.grid = units < di.sms ? (int)units : di.sms;
@@ -475,7 +522,7 @@ int dsa_index_decode_workspace_size(int B, int total_q, int max_keys, int H, int
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   DecodePlan p;
-  plan_decode(di, B, total_q, max_keys, H, d, k, q_dtype, k_dtype, p);
+  plan_decode(di, B, total_q, (int64_t)B * max_keys, max_keys, H, d, k, q_dtype, k_dtype, p);
   *bytes = p.total;
   return DSA_OK;
 }
@@ -493,10 +540,14 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   DecodePlan p;
-  plan_decode(di, B, total_q, max_keys, H, d, k, q_dtype, k_dtype, p);
+  plan_decode(di, B, total_q, total_keys, max_keys, H, d, k, q_dtype, k_dtype, p);
   if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, total_keys, d, ws, p.widen_off, st)) != DSA_OK) return r;
+    K = ws + p.widen_off;
+  }
   int* status = reinterpret_cast<int*>(ws);
   int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
   float* pval = reinterpret_cast<float*>(ws + p.pval_off);
@@ -510,6 +561,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
     TcArgs a;
     memset(&a, 0, sizeof(a));
     a.kind = 1;
+    a.k_scale = K_scale;
     a.n_rows = total_q;
     a.n_units = B * p.splits;
     a.k = k;

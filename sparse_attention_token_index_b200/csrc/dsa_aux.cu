@@ -221,6 +221,36 @@ int launch_decode_merge(const int32_t* part_idx, const float* part_val, const in
 }
 
 // ---------------------------------------------------------------------------
+// fp8 e4m3 keys -> bf16 (every e4m3 value is exactly a bf16 value), 16 keys'
+// bytes per thread per step.
+// ---------------------------------------------------------------------------
+__global__ void e4m3_to_bf16_kernel(const uint4* __restrict__ src, int64_t n16, uint4* __restrict__ dst) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = src[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float a = e4m3_to_f32((uint8_t)(w[j] >> (16 * h)));
+        const float b = e4m3_to_f32((uint8_t)(w[j] >> (16 * h + 8)));
+        const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+        o[2 * j + h] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+    }
+    dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream) {
+  e4m3_to_bf16_kernel<<<148 * 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(src), n / 16,
+                                                    static_cast<uint4*>(dst));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 __global__ void fill_neg_inf_kernel(float* S, int64_t n) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     S[i] = __int_as_float(0xff800000);

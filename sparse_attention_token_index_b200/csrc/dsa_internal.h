@@ -18,6 +18,7 @@ namespace dsa {
 //           positions.
 struct TcArgs {
   int kind;
+  const float* k_scale;     // per-key scale (fp8 keys), or null
   int n_rows;
   int n_units;
   int k;
@@ -90,5 +91,7 @@ int launch_decode_merge(const int32_t* part_idx, const float* part_val, const in
                         int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
                         cudaStream_t stream);
 int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
+// Exact e4m3 -> bf16 copy of n bytes (n a multiple of 16, both 16-byte aligned).
+int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream);
 
 }  // namespace dsa

@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (a.kind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
+      const float* kscale = a.k_scale;  // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0
+      const int u_key_row0 = u.key_row0;
       if (has_q) {
         if (tid == 0) tb_retire(st);
         named_bar(bar, 128);
@@ -375,6 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kmap != nullptr) kpos = in_range ? (int64_t)kmap[key] : -1;
           const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
           float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+          if (kscale != nullptr && in_range) score *= kscale[a.kind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && kpos >= 0 && kpos <= pos;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;

@@ -246,14 +246,6 @@ __device__ __forceinline__ CandList single_list(const uint2* base, int n) {
   return c;
 }
 
-struct StageSrc {
-  const uint2* p;
-  __device__ __forceinline__ bool get(int i, uint2& e) const {
-    e = p[i];
-    return true;
-  }
-};
-
 struct BinSrc {
   CandList c;
   int bin;
@@ -338,25 +330,6 @@ __device__ void emit_at_least(const Src& src, int n, uint64_t prefix, uint64_t m
     if ((sel_key(e) & mask) >= prefix) emit(st, e, oidx, oval);
   }
   named_bar(bar, nthr);
-}
-
-// Selects the `need` best entries (by sel_key) among the entries of `src`
-// that pass its filter, and emits them.  All nthr threads of the group call
-// it; the group synchronises on named barrier `bar`.
-template <class Src>
-__device__ void radix_emit(const Src& src, int n, int need, RowState& st, int32_t* oidx, float* oval, int tid,
-                           int nthr, int bar) {
-  uint64_t prefix = 0, mask = 0;
-  int remaining = need;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    int dsel, above, hsel;
-    radix_level(src, n, prefix, mask, shift, remaining, st, tid, nthr, bar, dsel, above, hsel);
-    remaining -= above;
-    prefix |= (uint64_t)dsel << shift;
-    mask |= (uint64_t)0xFFu << shift;
-    if (hsel == remaining) break;
-  }
-  emit_at_least(src, n, prefix, mask, st, oidx, oval, tid, nthr, bar);
 }
 
 // Warp-aggregated output: lanes with `sel` write their entry at

@@ -79,3 +79,8 @@ def test_decode_full_size_sampled():
     # 32 caches x 131072 keys, 2 queries each, k = 2048; 8 sampled rows
     inp = make_decode_inputs(device=DEV)
     _check(inp, 2048, rows=[0, 1, 17, 30, 41, 50, 62, 63], what="decode 32x128K")
+
+
+def test_decode_fp8_keys_tensor_core():
+    inp = make_decode_inputs(device=DEV, lengths=[1200, 300, 77], m=[2, 3, 1], seed=36, k_dtype="fp8")
+    _check(inp, 96, what="decode fp8 tc")

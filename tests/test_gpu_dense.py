@@ -157,3 +157,21 @@ def test_all_keys_identical(path):
     for t in range(T):
         assert sorted(idx[t].tolist()) == list(range(k)), t
         assert len(set(val[t].tolist())) == 1
+
+
+def test_fp8_keys_tensor_core():
+    # e4m3 keys with a per-key scale at H = 64, d = 128: keys widened exactly
+    # to bf16, the scale applied to the score
+    inp = make_dense_inputs("fp8_256k", device=DEV, T=400, N=900)
+    assert inp.k.dtype == torch.uint8
+    _run_and_check(inp, 128, what="fp8 tc")
+
+
+def test_fp8_debug_scores_tensor_core():
+    inp = make_dense_inputs("fp8_256k", device=DEV, T=200, N=300)
+    S = dsa.dsa_debug_scores(inp.q, inp.w, inp.k, q_pos0=inp.q_pos0, K_scale=inp.k_scale, check=True)
+    K, ks = _keys(inp)
+    ref = O.score_rows(_f64(inp.q), _f64(inp.w), O.key_values(K, ks))
+    pos = inp.q_pos0 + np.arange(200)
+    ref = np.where(np.arange(300)[None, :] <= pos[:, None], ref, -np.inf)
+    check_scores(S.cpu().numpy(), ref, what="fp8 tc")

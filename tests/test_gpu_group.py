@@ -127,3 +127,26 @@ def test_group_full_size_sampled():
                     check_row(gi[t], gv[t], S[cand], k, what=f"refine t={t}", idx_map=cand)
                 else:
                     check_row(gi[t], gv[t], ps[cand], k, what=f"reuse t={t}", idx_map=cand)
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+def test_group_fp8_keys(mode):
+    inp = make_dense_inputs("fp8_256k", device=DEV, T=256, N=512)
+    idx, val, bidx, bval, pq, pw = dsa.dsa_index_group(inp.q, inp.w, inp.k, 32, 64, 128, mode=mode,
+                                                       q_pos0=inp.q_pos0, K_scale=inp.k_scale, return_bank=True,
+                                                       return_proxy=True, check=True)
+    Kd = O.key_values(inp.k.cpu().numpy(), inp.k_scale.cpu().numpy())
+    gq, gw = _f64(pq), _f64(pw)
+    bi, bv = bidx.cpu().numpy(), bval.cpu().numpy()
+    gi, gv = idx.cpu().numpy(), val.cpu().numpy()
+    q, w = _f64(inp.q), _f64(inp.w)
+    for g in range(4):
+        L = inp.q_pos0 + (g + 1) * 64 - 1
+        ps = O.score_rows(gq[g:g + 1], gw[g:g + 1], Kd[:L + 1])[0]
+        check_row(bi[g], bv[g], ps, 128, what=f"fp8 bank g={g}")
+        bank = bi[g][bi[g] >= 0].astype(np.int64)
+        for t in range(g * 64, (g + 1) * 64, 9):
+            p = inp.q_pos0 + t
+            cand = bank[bank <= p]
+            S = (O.score_rows(q[t:t + 1], w[t:t + 1], Kd[:p + 1])[0] if mode == 0 else ps)
+            check_row(gi[t], gv[t], S[cand], 32, what=f"fp8 member t={t}", idx_map=cand)
