@@ -16,37 +16,65 @@ namespace dsa {
 // proxy: qbar[g] = mean of q over the group's members (fp32 sum, then
 // rounded to the input type), wbar[g] = mean of w (fp32).
 // ---------------------------------------------------------------------------
+// Each thread owns 8 consecutive elements (one 16-byte load per member row
+// for bf16 queries), summed over the members in order in fp32.
 __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __restrict__ w, int T, int H, int d,
                                   int G, int q_dtype, void* __restrict__ qbar, float* __restrict__ wbar) {
-  const int g = blockIdx.x;
+  const int g = blockIdx.y;
   const int r0 = g * G, r1 = min(T, r0 + G);
-  const float inv_n = 1.0f / (float)(r1 - r0);
+  const float n = (float)(r1 - r0);
   const int64_t hd = (int64_t)H * d;
-  for (int64_t e = threadIdx.x; e < hd; e += blockDim.x) {
-    float s = 0.f;
-    for (int r = r0; r < r1; ++r) {
-      const int64_t i = (int64_t)r * hd + e;
-      s += (q_dtype == DSA_DTYPE_FP32) ? static_cast<const float*>(Q)[i]
-                                       : __bfloat162float(static_cast<const __nv_bfloat16*>(Q)[i]);
+  const int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (e0 < hd) {
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (q_dtype == DSA_DTYPE_BF16 && e0 + 8 <= hd) {
+      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+      for (int r = r0; r < r1; ++r) {
+        const uint4 v = *reinterpret_cast<const uint4*>(q + (int64_t)r * hd + e0);
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(p[j]);
+          s[2 * j] += f.x;
+          s[2 * j + 1] += f.y;
+        }
+      }
+      uint4 o;
+      __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) po[j] = __floats2bfloat162_rn(s[2 * j] / n, s[2 * j + 1] / n);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(qbar) + (int64_t)g * hd + e0) = o;
+    } else {
+      for (int j = 0; j < 8 && e0 + j < hd; ++j) {
+        float a = 0.f;
+        for (int r = r0; r < r1; ++r) {
+          const int64_t i = (int64_t)r * hd + e0 + j;
+          a += (q_dtype == DSA_DTYPE_FP32) ? static_cast<const float*>(Q)[i]
+                                           : __bfloat162float(static_cast<const __nv_bfloat16*>(Q)[i]);
+        }
+        const float m = a / n;
+        if (q_dtype == DSA_DTYPE_FP32)
+          static_cast<float*>(qbar)[(int64_t)g * hd + e0 + j] = m;
+        else
+          static_cast<__nv_bfloat16*>(qbar)[(int64_t)g * hd + e0 + j] = __float2bfloat16_rn(m);
+      }
     }
-    const float m = s / (float)(r1 - r0);
-    if (q_dtype == DSA_DTYPE_FP32)
-      static_cast<float*>(qbar)[(int64_t)g * hd + e] = m;
-    else
-      static_cast<__nv_bfloat16*>(qbar)[(int64_t)g * hd + e] = __float2bfloat16_rn(m);
   }
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    float s = 0.f;
-    for (int r = r0; r < r1; ++r) s += w[(int64_t)r * H + h];
-    wbar[(int64_t)g * H + h] = s / (float)(r1 - r0);
+  if (blockIdx.x == 0) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+      float a = 0.f;
+      for (int r = r0; r < r1; ++r) a += w[(int64_t)r * H + h];
+      wbar[(int64_t)g * H + h] = a / n;
+    }
   }
-  (void)inv_n;
 }
 
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
                       float* wbar, cudaStream_t stream) {
   const int ng = (T + G - 1) / G;
-  proxy_mean_kernel<<<ng, 256, 0, stream>>>(Q, w, T, H, d, G, q_dtype, qbar, wbar);
+  const int64_t chunks = ((int64_t)H * d + 7) / 8;
+  const dim3 grid((unsigned)((chunks + 127) / 128), (unsigned)ng);
+  proxy_mean_kernel<<<grid, 128, 0, stream>>>(Q, w, T, H, d, G, q_dtype, qbar, wbar);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -171,52 +199,78 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
 }
 
 // ---------------------------------------------------------------------------
-// decode merge: per query row, the union of its splits' top-k lists goes
-// through the streaming filter into a contiguous scratch list, then the
-// exact selection.
+// decode merge: per query row, its splits' top-k lists are compacted into one
+// contiguous list while their histogram is built (one pass, batched loads),
+// the exact threshold bin is read off the histogram, and the row is selected.
 // ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 256;
+constexpr int kMergeStage = 2048;
+
 struct MergeSmem {
   RowState st;
-  uint2 stage[1024];
+  uint2 stage[kMergeStage];
+  int base[257];  // prefix sums of the splits' counts
 };
 
-__global__ void __launch_bounds__(128) decode_merge_kernel(const int32_t* __restrict__ part_idx,
-                                                           const float* __restrict__ part_val,
-                                                           const int* __restrict__ part_cnt, int splits, int k,
-                                                           int32_t* __restrict__ out_idx, float* __restrict__ out_val,
-                                                           uint2* __restrict__ scratch, int* status) {
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32_t* __restrict__ part_idx,
+                                                                     const float* __restrict__ part_val,
+                                                                     const int* __restrict__ part_cnt, int splits,
+                                                                     int k, int32_t* __restrict__ out_idx,
+                                                                     float* __restrict__ out_val,
+                                                                     uint2* __restrict__ scratch, int* status) {
   __shared__ MergeSmem M;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
-  row_reset(M.st, tid, 128);
-  uint2* cand = scratch + (int64_t)row * splits * k;
-  named_bar(1, 128);
-  for (int s = 0; s < splits; ++s) {
-    const int64_t o = ((int64_t)row * splits + s);
-    const int c = part_cnt[o];
-    for (int i0 = 0; i0 < c; i0 += 128) {
-      const int i = i0 + tid;
-      const bool valid = i < c;
-      float v = 0.f;
-      uint32_t id = 0;
-      if (valid) {
-        v = part_val[o * k + i];
-        id = (uint32_t)part_idx[o * k + i];
-      }
-      row_append(M.st, cand, v, id, valid, lane);
+  RowState& st = M.st;
+  row_reset(st, tid, kMergeThreads);
+  if (tid == 0) {
+    int acc = 0;
+    for (int s = 0; s < splits; ++s) {
+      M.base[s] = acc;
+      acc += part_cnt[(int64_t)row * splits + s];
     }
-    named_bar(1, 128);
-    if (tid < 32) row_update(M.st, k, lane);
-    named_bar(1, 128);
+    M.base[splits] = acc;
   }
-  row_select(M.st, single_list(cand, M.st.cnt), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k, M.stage, 1024, tid, 128, 1,
-             status);
+  __syncthreads();
+  uint2* cand = scratch + (int64_t)row * splits * k;
+  for (int s = 0; s < splits; ++s) {
+    const int64_t o = ((int64_t)row * splits + s) * k;
+    const int c = M.base[s + 1] - M.base[s], b0 = M.base[s];
+    for (int i0 = 0; i0 < c; i0 += kMergeThreads * 4) {
+      uint2 e[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * kMergeThreads + tid;
+        e[j] = (i < c) ? make_uint2(__float_as_uint(part_val[o + i]), (uint32_t)part_idx[o + i]) : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + j * kMergeThreads + tid;
+        if (i < c) {
+          cand[b0 + i] = e[j];
+          atomicAdd(&st.hist[score_bin(__uint_as_float(e[j].x))], 1u);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int2 r = hist_scan(st, 0, kBins - 1, k, lane);
+    if (lane == 0) {
+      st.bstar = r.x >= 0 ? r.x : 0;
+      st.cge = r.y;
+    }
+  }
+  __syncthreads();
+  row_select(st, single_list(cand, M.base[splits]), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k,
+             M.stage, kMergeStage, tid, kMergeThreads, 1, status);
 }
 
 int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
                         int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
                         cudaStream_t stream) {
-  decode_merge_kernel<<<total_q, 128, 0, stream>>>(part_idx, part_val, part_cnt, splits, k, out_idx, out_val,
-                                                    scratch, status);
+  if (splits > 256) return DSA_ERR_UNSUPPORTED;
+  decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(part_idx, part_val, part_cnt, splits, k, out_idx,
+                                                              out_val, scratch, status);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

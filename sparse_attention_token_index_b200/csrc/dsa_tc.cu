@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     while (*(volatile int*)&S.epi_done < 4 && !*abort_flag) {
 #pragma unroll 1
       for (int q = 0; q < kQB; ++q) tb_raise(S.rows[q], a.k, lane);
-      __nanosleep(200);
+      __nanosleep(1000);
     }
   } else {
     // ---------------- epilogue: warpgroup `slot` follows query `slot` ----------------
