@@ -137,7 +137,10 @@ struct DensePlan {
 DensePlan plan_dense(const DeviceInfo& di, int T, int N, int H, int d, int q_dtype, int k_dtype, Layout& L) {
   DensePlan p;
   p.tc = use_tc(H, d, q_dtype, k_dtype);
-  p.cand_cap = ((int64_t)N + 127) / 128 * 128;
+  // candidate lists: a multiple of 4 tiles of 128 keys, so that a team of
+  // 1, 2 or 4 warpgroups splits them into equal per-warp segments that each
+  // hold every key of the tiles that warp owns
+  p.cand_cap = ((int64_t)N + 511) / 512 * 512;
   if (p.tc) {
     const int units = (T + 3) / 4;
     p.grid = units < di.sms ? units : di.sms;
@@ -357,7 +360,7 @@ int plan_group(const DeviceInfo& di, int T, int N, int H, int d, int k, int G, i
   gp.scan = plan_dense(di, gp.ng, N, H, d, q_dtype, k_dtype, L);
   gp.kg_off = 0;
   gp.ref_cand_off = 0;
-  gp.ref_cap = ((int64_t)B + 127) / 128 * 128;
+  gp.ref_cap = ((int64_t)B + 511) / 512 * 512;
   gp.ref_grid = 0;
   if (use_tc(H, d, q_dtype, k_dtype)) {
     gp.kg_off = L.take((size_t)gp.ng * B * d * 2);  // gathered bank keys, bf16
@@ -490,7 +493,7 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
   }
   p.splits = best_s;
   p.tiles_per_split = (tiles_max + best_s - 1) / best_s;
-  p.cand_cap = (int64_t)p.tiles_per_split * 128;
+  p.cand_cap = (int64_t)((p.tiles_per_split + 3) / 4 * 4) * 128;
   Layout L;
   p.widen_off = take_widen(L, total_keys, H, d, q_dtype, k_dtype);
   if (p.tc) {

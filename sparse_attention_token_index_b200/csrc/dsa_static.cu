@@ -82,9 +82,10 @@ extern "C" int dsa_index_dense_static(const void* Q, const float* w, const void*
     return DSA_ERR_CUDA;
   if (major != 10) return DSA_ERR_DEVICE;
 
-  // Each CTA of the kernel keeps 4 candidate lists of round_up(N, 128)
-  // entries; the grid shrinks to what the fixed scratch holds.
-  const int64_t cap = ((int64_t)N + 127) / 128 * 128;
+  // Each CTA of the kernel keeps 4 candidate lists of round_up(N, 512)
+  // entries (whole groups of 4 key tiles); the grid shrinks to what the
+  // fixed scratch holds.
+  const int64_t cap = ((int64_t)N + 511) / 512 * 512;
   const size_t per_cta = (size_t)4 * cap * sizeof(uint2);
   const int units = (T + 3) / 4;
   const int64_t fit = (int64_t)((kStaticScratchBytes - 256) / per_cta);

@@ -307,42 +307,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __nanosleep(1000);
     }
   } else {
-    // ---------------- epilogue: warpgroup `slot` follows query `slot` ----------------
-    // Per tile a warp waits for its accumulator, pulls its 32 key rows x 64
-    // heads out of TMEM, frees the buffer, scores, and appends survivors of
-    // the threshold to its own candidate segment.  No barrier inside the
-    // tile loop: warp 0 of the group raises the threshold every few tiles
-    // from the shared histogram alone.
+    // ---------------- epilogue: 16 warps in four warpgroups ----------------
+    // A unit of nq queries gives each query a team of 4/nq warpgroups (one
+    // for nq >= 3, the last warpgroup idle when nq == 3); team member m takes
+    // the tiles jt with jt % team == m, so the per-tile latency of a short
+    // unit (decode, tails) overlaps across the team.  Per tile a warp waits
+    // for its accumulator, pulls its 32 key rows x 64 heads out of TMEM,
+    // frees the buffer, scores, and appends survivors of the threshold to its
+    // own candidate segment; warps not on the tile only release it.  No
+    // barrier inside the tile loop: the threshold warp raises the thresholds.
     const int slot = warp >> 2, lq = warp & 3, tid = threadIdx.x & 127;
-    const int bar = 1 + slot;
-    RowState& st = S.rows[slot];
-    const int64_t seg_stride = a.cand_cap / 4;
-    uint2* const cand0 = a.cand + ((int64_t)blockIdx.x * kQB + slot) * a.cand_cap;
-    uint2* const my_seg = cand0 + lq * seg_stride;
-    const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[slot]);
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
     uint32_t eph = 0u;  // bit b: phase of accumulator buffer b
     int buf = 0;
     UnitInfo u;
     bool ok = true;
     for (int round = 0; ok && unit_at(a, round, u); ++round) {
+      // team layout of this unit
+      const int team = u.nq == 1 ? 4 : (u.nq == 2 ? 2 : 1);
+      const int q = team == 1 ? slot : (team == 2 ? (slot & 1) : 0);
+      const int member = team == 1 ? 0 : (team == 2 ? (slot >> 1) : slot);
+      const bool active = q < u.nq;
+      const int tbar = team == 1 ? 1 + slot : (team == 2 ? 5 + q : 7);
+      const int tthr = 128 * team;
+      const int ttid = member * 128 + tid;
+      RowState& st = S.rows[q];
+      const int nseg = 4 * team;
+      const int64_t seg_stride = a.cand_cap / nseg;
+      uint2* const cand0 = a.cand + ((int64_t)blockIdx.x * kQB + q) * a.cand_cap;
+      uint2* const my_seg = cand0 + (member * 4 + lq) * seg_stride;
+      const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[q]);
       // per-unit scalars (kept in registers through the tile loop)
-      const bool has_q = slot < u.nq;
-      const int64_t row = (int64_t)u.row0 + slot;
-      const int64_t pos = has_q ? slot_pos(a, u, slot) : -1;
+      const int64_t row = (int64_t)u.row0 + q;
+      const int64_t pos = active ? slot_pos(a, u, q) : -1;
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (a.kind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
       const float* kscale = a.k_scale;  // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0
       const int u_key_row0 = u.key_row0;
-      if (has_q) {
-        if (tid == 0) tb_retire(st);
-        named_bar(bar, 128);
-        row_reset(st, tid, 128);
-        if (tid < kHeads) S.w[slot][tid] = a.w[row * kHeads + tid];
+      if (active) {
+        if (ttid == 0) tb_retire(st);
+        named_bar(tbar, tthr);
+        row_reset(st, ttid, tthr);
+        if (ttid < kHeads) S.w[q][ttid] = a.w[row * kHeads + ttid];
+        named_bar(tbar, tthr);
+        if (ttid == 0) tb_open(st);
       }
-      named_bar(bar, 128);
-      if (has_q && tid == 0) tb_open(st);
       int count = 0;  // my segment's fill
       for (int jt = 0; jt < ntiles; ++jt) {
         if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30)) {
@@ -350,9 +360,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         tc_fence_after();
+        const bool mine = active && (jt % team) == member;
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
-        const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + slot * kHeads);
-        if (has_q) {
+        const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
+        if (mine) {
           float v[32];
           tmem_ld_32x32b_x32(col, v);
           tmem_ld_wait();
@@ -370,7 +381,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         eph ^= 1u << buf;
         buf ^= 1;
-        if (has_q) {
+        if (mine) {
           const int key = key0 + jt * kTileKeys;  // local key index
           const bool in_range = key < nkeys;
           int64_t kpos = key;
@@ -384,35 +395,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
         }
       }
-      // the whole group agrees on success before any further barrier
-      ok = group_and(bar, 128, ok);
-      if (!ok) break;
-      if (has_q) {
-        if (lane == 0) st.seg_cnt[lq] = count;
-        if (tid == 0) tb_close(st);
-        named_bar(bar, 128);
-        if (lq == 0) tb_finish(st, a.k, lane);
-        named_bar(bar, 128);
-        CandList cl;
-        cl.base = cand0;
-        cl.stride = seg_stride;
-        cl.c0 = st.seg_cnt[0];
-        cl.c1 = st.seg_cnt[1];
-        cl.c2 = st.seg_cnt[2];
-        cl.c3 = st.seg_cnt[3];
-        int32_t* oi;
-        float* ov;
-        if (a.kind != 1) {
-          oi = a.out_idx + row * a.out_ld;
-          ov = a.out_val + row * a.out_ld;
-        } else {
-          const int64_t o = row * a.splits + u.seq_split;
-          oi = a.out_idx + o * a.out_ld;
-          ov = a.out_val + o * a.out_ld;
-        }
-        const int cnt = row_select(st, cl, a.k, oi, ov, S.stage[slot], kStageCap, tid, 128, bar, a.status);
-        if (a.kind == 1 && tid == 0) a.out_cnt[row * a.splits + u.seq_split] = cnt;
+      if (!active) {
+        ok = group_and(1 + slot, 128, ok);
+        continue;
       }
+      // the whole team agrees on success before any further barrier
+      ok = group_and(tbar, tthr, ok);
+      if (!ok) break;
+      if (lane == 0) st.seg_cnt[member * 4 + lq] = count;
+      if (ttid == 0) tb_close(st);
+      named_bar(tbar, tthr);
+      if (ttid < 32) tb_finish(st, a.k, lane);
+      named_bar(tbar, tthr);
+      CandList cl;
+      cl.base = cand0;
+      cl.stride = seg_stride;
+      cl.nseg = nseg;
+      cl.cnt = st.seg_cnt;
+      int32_t* oi;
+      float* ov;
+      if (a.kind != 1) {
+        oi = a.out_idx + row * a.out_ld;
+        ov = a.out_val + row * a.out_ld;
+      } else {
+        const int64_t o = row * a.splits + u.seq_split;
+        oi = a.out_idx + o * a.out_ld;
+        ov = a.out_val + o * a.out_ld;
+      }
+      const int cnt = row_select(st, cl, a.k, oi, ov, S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
+      if (a.kind == 1 && ttid == 0) a.out_cnt[row * a.splits + u.seq_split] = cnt;
     }
     if (tid == 0) atomicAdd(&S.epi_done, 1);
   }

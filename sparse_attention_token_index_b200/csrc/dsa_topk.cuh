@@ -23,7 +23,7 @@ namespace dsa {
 struct RowState {
   uint32_t hist[kBins];
   int cnt;         // single-list path: entries appended
-  int seg_cnt[4];  // segmented path: entries per segment (set at row end)
+  int seg_cnt[16]; // segmented path: entries per segment (set at row end)
   int bstar;       // threshold bin
   int cge;         // appended entries whose bin >= bstar (exact at select time)
   int seen;        // single-list path: cnt at the last update
@@ -37,20 +37,25 @@ struct RowState {
 
 constexpr uint32_t kTbActive = 1u << 16;
 
-// Candidate list: up to four segments of `stride` entries each, c0..c3 used
-// (scalars, so that the list lives in registers).
+// Candidate list: nseg segments of `stride` entries each; cnt[s] (shared
+// memory) entries used in segment s.
 struct CandList {
   const uint2* base;
   int64_t stride;
-  int c0, c1, c2, c3;
-  __device__ __forceinline__ int total() const { return c0 + c1 + c2 + c3; }
+  int nseg;
+  const int* cnt;
+  __device__ __forceinline__ int total() const {
+    int n = 0;
+    for (int s = 0; s < nseg; ++s) n += cnt[s];
+    return n;
+  }
   __device__ __forceinline__ uint2 at(int i) const {
-    if (i < c0) return base[i];
-    i -= c0;
-    if (i < c1) return base[stride + i];
-    i -= c1;
-    if (i < c2) return base[2 * stride + i];
-    return base[3 * stride + (i - c2)];
+    int s = 0;
+    while (s + 1 < nseg && i >= cnt[s]) {
+      i -= cnt[s];
+      ++s;
+    }
+    return base[s * stride + i];
   }
 };
 
@@ -62,7 +67,7 @@ __device__ __forceinline__ void row_reset(RowState& st, int tid, int nthr) {
     st.cge = 0;
     st.seen = 0;
     st.top = 0;
-    for (int s = 0; s < 4; ++s) st.seg_cnt[s] = 0;
+    for (int s = 0; s < 16; ++s) st.seg_cnt[s] = 0;
   }
 }
 
@@ -237,12 +242,13 @@ __device__ __forceinline__ void row_update(RowState& st, int k, int lane) {
   __syncwarp();
 }
 
-__device__ __forceinline__ CandList single_list(const uint2* base, int n) {
+// One contiguous list whose length is *n (shared memory).
+__device__ __forceinline__ CandList single_list(const uint2* base, const int* n) {
   CandList c;
   c.base = base;
   c.stride = 0;
-  c.c0 = n;
-  c.c1 = c.c2 = c.c3 = 0;
+  c.nseg = 1;
+  c.cnt = n;
   return c;
 }
 
@@ -365,11 +371,9 @@ constexpr int kBatch = 8;
 // (valid = false past the end) so that f may use warp collectives.
 template <class F>
 __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nthr, F&& f) {
-  const int cnt[4] = {c.c0, c.c1, c.c2, c.c3};
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
+  for (int s = 0; s < c.nseg; ++s) {
     const uint2* seg = c.base + s * c.stride;
-    const int n = cnt[s];
+    const int n = c.cnt[s];
     for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
       uint2 e[kBatch];
 #pragma unroll
@@ -392,11 +396,9 @@ template <class Cls>
 __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nthr, RowState& st, int32_t* oidx,
                                               float* oval, uint2* stage, int stage_cap, Cls&& cls) {
   const int lane = tid & 31;
-  const int cnt[4] = {c.c0, c.c1, c.c2, c.c3};
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
+  for (int s = 0; s < c.nseg; ++s) {
     const uint2* seg = c.base + s * c.stride;
-    const int n = cnt[s];
+    const int n = c.cnt[s];
     for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
       uint2 e[kBatch];
       int cat[kBatch];
