@@ -241,7 +241,9 @@ class Decode(Workload):
         self.alg_bytes = (i.k.numel() * i.k.element_size() + i.q.numel() * i.q.element_size()
                           + i.w.numel() * 4 + i.q.shape[0] * self.k * 8)
         self.rows = i.q.shape[0]
-        self.ko, self.qo = i.k_offsets.to(device), i.q_offsets.to(device)
+        self.ko = i.k_offsets.to(device, torch.int64)
+        self.qo = i.q_offsets.to(device, torch.int32)
+        self.total_keys = int(i.k_offsets[-1])
         self.host_src = [i.q, i.w, i.k]
         self.launches_per_step = 2
 
@@ -263,7 +265,7 @@ class Decode(Workload):
 
     def call(self, q, w, k):
         import sparse_attention_token_index_b200 as dsa
-        dsa.dsa_index_decode(q, w, k, self.k, self.inp.k_offsets, self.inp.q_offsets, max_keys=self.cfg["Nb"],
+        dsa.dsa_index_decode(q, w, k, self.k, self.ko, self.qo, max_keys=self.cfg["Nb"], total_keys=self.total_keys,
                              out=self.out, workspace=self.ws)
 
     def oracle_sample(self, budget_s=15.0, seed=0):

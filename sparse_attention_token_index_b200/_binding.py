@@ -14,7 +14,8 @@ DSA_GROUP_REFINE = 0
 DSA_GROUP_REUSE = 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_HERE, "libdsa_index.so")
+# DSA_LIB overrides the in-tree library (to compare builds)
+lib_path = os.environ.get("DSA_LIB") or os.path.join(_HERE, "libdsa_index.so")
 
 EXPORTED_SYMBOLS = (
     "dsa_status_string", "dsa_version", "dsa_check_status",
@@ -216,28 +217,35 @@ def dsa_index_group(Q, w, K, k: int, group: int, bank: int, mode: int = DSA_GROU
 
 
 def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.Tensor,
-                     max_keys: Optional[int] = None, K_scale=None, out=None, workspace=None, stream=None,
-                     check: bool = False):
+                     max_keys: Optional[int] = None, total_keys: Optional[int] = None, K_scale=None, out=None,
+                     workspace=None, stream=None, check: bool = False):
     """Decode indexer over B key caches; offsets are [B+1] (host or device).
 
-    Returns (idx [sum m_b, k], val) with key indices local to each sequence.
+    With device offsets (int64 / int32) and ``max_keys`` / ``total_keys``
+    given, the call does no host-side work on the offsets (no copies, no
+    synchronisation).  Returns (idx [sum m_b, k], val) with key indices
+    local to each sequence.
     """
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
-    ko_host = k_offsets.to("cpu", torch.int64)
-    if max_keys is None:
-        max_keys = int((ko_host[1:] - ko_host[:-1]).max())
-    total_keys = int(ko_host[-1])
-    ko = k_offsets.to(Q.device, torch.int64).contiguous()
-    qo = q_offsets.to(Q.device, torch.int32).contiguous()
+    if max_keys is None or total_keys is None:
+        ko_host = k_offsets.to("cpu", torch.int64)
+        if max_keys is None:
+            max_keys = int((ko_host[1:] - ko_host[:-1]).max())
+        if total_keys is None:
+            total_keys = int(ko_host[-1])
+    ko = k_offsets if (k_offsets.is_cuda and k_offsets.dtype == torch.int64) else \
+        k_offsets.to(Q.device, torch.int64).contiguous()
+    qo = q_offsets if (q_offsets.is_cuda and q_offsets.dtype == torch.int32) else \
+        q_offsets.to(Q.device, torch.int32).contiguous()
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     nb = decode_workspace_bytes(B, total_q, max_keys, H, d, k, qd, kd)
     ws = _workspace(nb, Q.device, workspace)
     idx, val = _outputs(total_q, k, Q.device, out)
     _check(lib().dsa_index_decode(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), _ptr(ko), _ptr(qo), B, total_q,
-                                  total_keys, max_keys, H, d, k, qd, kd, _ptr(idx), _ptr(val), _ptr(ws), ws.numel(),
-                                  _stream(stream)), "dsa_index_decode")
+                                  int(total_keys), int(max_keys), H, d, k, qd, kd, _ptr(idx), _ptr(val), _ptr(ws),
+                                  ws.numel(), _stream(stream)), "dsa_index_decode")
     if check:
         dsa_check_status(ws, stream)
     return idx, val

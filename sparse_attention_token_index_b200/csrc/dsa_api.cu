@@ -466,41 +466,50 @@ namespace {
 struct DecodePlan {
   size_t widen_off;
   bool tc;
-  int splits, tiles_per_split;
   int grid;
   int64_t cand_cap;
+  int splits, tiles_per_split;
   size_t cand_off, pidx_off, pval_off, pcnt_off, mscr_off, total;
 };
 
 void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, int max_keys, int H, int d, int k,
                  int q_dtype, int k_dtype, DecodePlan& p) {
+  memset(&p, 0, sizeof(p));
   p.tc = use_tc(H, d, q_dtype, k_dtype);
-  const int tiles_max = (max_keys + 127) / 128;
-  // choose the split count minimising (rounds of units) x (tiles per unit + a
-  // fixed per-unit cost of about 4 tiles)
-  int best_s = 1;
-  double best_cost = 1e300;
-  for (int s = 1; s <= 256 && s <= tiles_max; ++s) {
-    const int tps = (tiles_max + s - 1) / s;
-    const int s_eff = (tiles_max + tps - 1) / tps;
-    const int64_t units = (int64_t)B * s_eff;
-    const int64_t rounds = (units + di.sms - 1) / di.sms;
-    const double cost = (double)rounds * (tps + 4) + 0.01 * s_eff;
-    if (cost < best_cost) {
-      best_cost = cost;
-      best_s = s_eff;
-    }
-  }
-  p.splits = best_s;
-  p.tiles_per_split = (tiles_max + best_s - 1) / best_s;
-  p.cand_cap = (int64_t)((p.tiles_per_split + 3) / 4 * 4) * 128;
   Layout L;
   p.widen_off = take_widen(L, total_keys, H, d, q_dtype, k_dtype);
+  const int tiles_max = (max_keys + 127) / 128;
   if (p.tc) {
+    // split each cache into s pieces, s minimising (rounds of units over the
+    // grid) x (tiles per unit + a per-unit cost of about 4 tiles)
+    int best_s = 1;
+    double best_cost = 1e300;
+    for (int s = 1; s <= 256 && s <= tiles_max; ++s) {
+      const int tps = (tiles_max + s - 1) / s;
+      const int s_eff = (tiles_max + tps - 1) / tps;
+      const int64_t units = (int64_t)B * s_eff;
+      const int64_t rounds = (units + di.sms - 1) / di.sms;
+      const double cost = (double)rounds * (tps + 4) + 0.01 * s_eff;
+      if (cost < best_cost) {
+        best_cost = cost;
+        best_s = s_eff;
+      }
+    }
+    p.splits = best_s;
+    p.tiles_per_split = (tiles_max + best_s - 1) / best_s;
+    p.cand_cap = (int64_t)((p.tiles_per_split + 3) / 4 * 4) * 128;
     const int64_t units = (int64_t)B * p.splits;
     p.grid = units < di.sms ? (int)units : di.sms;
     p.cand_off = L.take((size_t)p.grid * 4 * p.cand_cap * sizeof(uint2));
   } else {
+    int s = (int)((2 * (int64_t)di.sms * 2 + total_q - 1) / total_q);
+    if (s < 1) s = 1;
+    if (s > 256) s = 256;
+    if (s > tiles_max) s = tiles_max;
+    const int kps = (int)((((int64_t)max_keys + s - 1) / s + 127) / 128 * 128);
+    p.tiles_per_split = kps / 128;
+    p.splits = (int)(((int64_t)max_keys + kps - 1) / kps);
+    p.cand_cap = kps;
     p.grid = simt_grid(di, (int64_t)total_q * p.splits);
     p.cand_off = L.take((size_t)p.grid * 2 * p.cand_cap * sizeof(uint2));
   }

@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32
     }
   }
   __syncthreads();
-  row_select(st, single_list(cand, &M.base[splits]), k, out_idx + (int64_t)row * k, out_val + (int64_t)row * k,
+  row_select(st, single_list(cand, &M.base[splits]), k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k),
              M.stage, kMergeStage, tid, kMergeThreads, 1, status);
 }
 

@@ -12,7 +12,8 @@ namespace dsa {
 //           pos_base + min(r * pos_mul + pos_add, pos_clamp) and sees keys
 //           0..pos (dense: pos_mul 1, pos_add 0; group proxies: pos_mul G,
 //           pos_add G-1 so the proxy scans its group's last member's prefix).
-//   kind 1: decode segments; unit v = (sequence v / splits, split v % splits).
+//   kind 1: decode segments; unit v = (sequence v / splits, split v % splits);
+//           each leaves a partial top-k list that decode_merge combines.
 //   kind 2: group refine; unit v = (group v / mblocks, member block v % mblocks);
 //           keys are the group's gathered bank rows, key_map gives their
 //           positions.

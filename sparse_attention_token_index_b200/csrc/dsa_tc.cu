@@ -67,7 +67,8 @@ struct UnitInfo {
   int tile0;         // first key tile (local to the key range)
   int ntiles;        // tiles streamed
   int nkeys;         // keys in the range (local index < nkeys is valid)
-  int seq_split;     // decode: split index; refine: group index
+  int seq_split;     // decode: sequence; refine: group index
+  int partial;       // decode: leaves a partial list
 };
 
 __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
@@ -77,11 +78,12 @@ __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
 }
 
 // Zig-zag, longest-first static schedule over the persistent grid.
+template <int kKind>
 __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u) {
   const int G = gridDim.x, c = blockIdx.x;
   const int v = round * G + ((round & 1) ? (G - 1 - c) : c);
   if (v >= a.n_units) return false;
-  if (a.kind == 0) {
+  if constexpr (kKind == 0) {
     const int unit = a.n_units - 1 - v;
     u.row0 = unit * kQB;
     u.nq = min(kQB, a.n_rows - u.row0);
@@ -91,13 +93,14 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     u.ntiles = (int)(maxpos / kTileKeys) + 1;
     u.nkeys = (int)(maxpos + 1);
     u.seq_split = -1;
-  } else if (a.kind == 1) {
+    u.partial = 0;
+  } else if constexpr (kKind == 1) {
     const int b = v / a.splits, sp = v % a.splits;
     const int64_t k0 = a.k_off[b], k1 = a.k_off[b + 1];
     const int q0 = a.q_off[b], q1 = a.q_off[b + 1];
-    const int nb = (int)(k1 - k0), mb = q1 - q0;
+    const int nb = (int)(k1 - k0);
     u.row0 = q0;
-    u.nq = mb;
+    u.nq = q1 - q0;
     const int tiles_b = (nb + kTileKeys - 1) / kTileKeys;
     const int t0 = min(tiles_b, sp * a.tiles_per_split);
     const int t1 = min(tiles_b, t0 + a.tiles_per_split);
@@ -106,6 +109,12 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     u.ntiles = t1 - t0;
     u.nkeys = nb;
     u.seq_split = sp;
+    u.partial = 1;
+    if (u.nq < 1 || u.nq > kQB || u.nq > nb) {  // 1 <= m_b <= min(4, N_b) is required
+      if (threadIdx.x == 0) report_error(a.status, DSA_ERR_INTERNAL, 3);
+      u.nq = 0;
+      u.ntiles = 0;
+    }
   } else {
     // group refine: members of group g against the group's gathered bank
     const int unit = a.n_units - 1 - v;
@@ -120,14 +129,16 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     u.ntiles = u.nq > 0 ? (nbk + kTileKeys - 1) / kTileKeys : 0;
     u.nkeys = nbk;
     u.seq_split = g;
+    u.partial = 0;
   }
   return true;
 }
 
 // Causal position of query `slot` of a unit (slot < u.nq), in key-index units.
+template <int kKind>
 __device__ __forceinline__ int64_t slot_pos(const TcArgs& a, const UnitInfo& u, int slot) {
-  if (a.kind == 0) return prefill_pos(a, u.row0 + slot);
-  if (a.kind == 1) return (int64_t)u.nkeys - u.nq + slot;
+  if constexpr (kKind == 0) return prefill_pos(a, u.row0 + slot);
+  if constexpr (kKind == 1) return (int64_t)u.nkeys - u.nq + slot;
   return a.pos_base + u.row0 + slot;
 }
 
@@ -179,7 +190,7 @@ __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ul
   }
 }
 
-template <bool kDebug>
+template <bool kDebug, int kKind>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_index_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ TcArgs a) {
@@ -224,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t armed = 0u, armed_ph = 0u;  // bit s: stage s armed / its phase
       bool ok = true;
       UnitInfo u;
-      for (int round = 0; ok && unit_at(a, round, u); ++round) {
+      for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
         if (qi > 0 && !(ok = mbar_wait(&S.q_empty, (qi - 1) & 1, abort_flag, a.status, 10))) break;
         mbar_arrive_expect_tx(&S.q_full, (uint32_t)(u.nq * 2 * kQHeadBlockBytes));
         for (int q = 0; q < u.nq; ++q)
@@ -261,7 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       UnitInfo u;
       const uint32_t q_addr = smem_u32(S.q);
-      for (int round = 0; ok && unit_at(a, round, u); ++round) {
+      for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
         if (!(ok = mbar_wait(&S.q_full, qi & 1, abort_flag, a.status, 20))) break;
         ++qi;
         tc_fence_after();
@@ -322,7 +333,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int buf = 0;
     UnitInfo u;
     bool ok = true;
-    for (int round = 0; ok && unit_at(a, round, u); ++round) {
+    for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
       // team layout of this unit
       const int team = u.nq == 1 ? 4 : (u.nq == 2 ? 2 : 1);
       const int q = team == 1 ? slot : (team == 2 ? (slot & 1) : 0);
@@ -339,10 +350,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[q]);
       // per-unit scalars (kept in registers through the tile loop)
       const int64_t row = (int64_t)u.row0 + q;
-      const int64_t pos = active ? slot_pos(a, u, q) : -1;
+      const int64_t pos = active ? slot_pos<kKind>(a, u, q) : -1;
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
-      const int32_t* kmap = (a.kind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
+      const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
       const float* kscale = a.k_scale;  // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0
       const int u_key_row0 = u.key_row0;
       if (active) {
@@ -388,7 +399,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kmap != nullptr) kpos = in_range ? (int64_t)kmap[key] : -1;
           const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
           float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
-          if (kscale != nullptr && in_range) score *= kscale[a.kind == 1 ? (int64_t)u_key_row0 + key : kpos];
+          if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && kpos >= 0 && kpos <= pos;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
@@ -412,18 +423,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cl.stride = seg_stride;
       cl.nseg = nseg;
       cl.cnt = st.seg_cnt;
-      int32_t* oi;
-      float* ov;
-      if (a.kind != 1) {
-        oi = a.out_idx + row * a.out_ld;
-        ov = a.out_val + row * a.out_ld;
-      } else {
+      cl.l2 = false;
+      if constexpr (kKind == 1) {
+        // decode: this split's local top-k, combined later by decode_merge
         const int64_t o = row * a.splits + u.seq_split;
-        oi = a.out_idx + o * a.out_ld;
-        ov = a.out_val + o * a.out_ld;
+        const int cnt = row_select(st, cl, a.k, row_out(a.out_idx + o * a.out_ld, a.out_val + o * a.out_ld),
+                                   S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
+        if (ttid == 0) a.out_cnt[o] = cnt;
+      } else {
+        row_select(st, cl, a.k, row_out(a.out_idx + row * a.out_ld, a.out_val + row * a.out_ld), S.stage[q],
+                   kStageCap, ttid, tthr, tbar, a.status);
       }
-      const int cnt = row_select(st, cl, a.k, oi, ov, S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
-      if (a.kind == 1 && ttid == 0) a.out_cnt[row * a.splits + u.seq_split] = cnt;
     }
     if (tid == 0) atomicAdd(&S.epi_done, 1);
   }
@@ -434,23 +444,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem_base, 512);
 }
 
-template <bool kDebug>
+template <bool kDebug, int kKind>
 static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid, cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(tc_index_kernel<kDebug>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_index_kernel<kDebug, kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kTcSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
     configured = true;
   }
-  tc_index_kernel<kDebug><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
+  tc_index_kernel<kDebug, kKind><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream) {
-  return a.dbg_scores != nullptr ? launch_tc<true>(tmQ, tmK, a, grid, stream)
-                                 : launch_tc<false>(tmQ, tmK, a, grid, stream);
+  if (a.dbg_scores != nullptr) return a.kind == 0 ? launch_tc<true, 0>(tmQ, tmK, a, grid, stream) : DSA_ERR_UNSUPPORTED;
+  switch (a.kind) {
+    case 0: return launch_tc<false, 0>(tmQ, tmK, a, grid, stream);
+    case 1: return launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
+    case 2: return launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
+    default: return DSA_ERR_INVALID_ARG;
+  }
 }
 
 size_t tc_smem_bytes() { return kTcSmemBytes; }

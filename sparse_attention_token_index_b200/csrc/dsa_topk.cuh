@@ -40,22 +40,26 @@ constexpr uint32_t kTbActive = 1u << 16;
 // Candidate list: nseg segments of `stride` entries each; cnt[s] (shared
 // memory) entries used in segment s.
 struct CandList {
-  const uint2* base;
+  const uint2* __restrict__ base;
   int64_t stride;
   int nseg;
   const int* cnt;
+  bool l2;  // entries written by other CTAs: read them through L2
+  // counts may live in shared or global memory (written by other CTAs):
+  // read them with volatile loads
+  __device__ __forceinline__ int count(int s) const { return *(volatile const int*)(cnt + s); }
   __device__ __forceinline__ int total() const {
     int n = 0;
-    for (int s = 0; s < nseg; ++s) n += cnt[s];
+    for (int s = 0; s < nseg; ++s) n += count(s);
     return n;
   }
   __device__ __forceinline__ uint2 at(int i) const {
     int s = 0;
-    while (s + 1 < nseg && i >= cnt[s]) {
-      i -= cnt[s];
+    while (s + 1 < nseg && i >= count(s)) {
+      i -= count(s);
       ++s;
     }
-    return base[s * stride + i];
+    return l2 ? __ldcg(base + s * stride + i) : base[s * stride + i];
   }
 };
 
@@ -249,6 +253,7 @@ __device__ __forceinline__ CandList single_list(const uint2* base, const int* n)
   c.stride = 0;
   c.nseg = 1;
   c.cnt = n;
+  c.l2 = false;
   return c;
 }
 
@@ -261,10 +266,35 @@ struct BinSrc {
   }
 };
 
-__device__ __forceinline__ void emit(RowState& st, uint2 e, int32_t* oidx, float* oval) {
+// Where a row's selection goes: separate index / score arrays, or packed
+// {score bits, index} pairs (partial lists that are merged later).
+struct RowOut {
+  int32_t* __restrict__ idx;
+  float* __restrict__ val;
+  uint2* __restrict__ pair;
+  __device__ __forceinline__ void put(int p, uint2 e) const {
+    if (pair != nullptr) {
+      pair[p] = e;
+    } else {
+      idx[p] = (int32_t)e.y;
+      val[p] = __uint_as_float(e.x);
+    }
+  }
+  __device__ __forceinline__ void pad(int p) const {
+    if (pair != nullptr) {
+      pair[p] = make_uint2(0xff800000u, 0xffffffffu);
+    } else {
+      idx[p] = -1;
+      val[p] = __int_as_float(0xff800000);
+    }
+  }
+};
+
+__device__ __forceinline__ RowOut row_out(int32_t* idx, float* val) { return RowOut{idx, val, nullptr}; }
+
+__device__ __forceinline__ void emit(RowState& st, uint2 e, const RowOut& out) {
   const int p = atomicAdd(&st.outpos, 1);
-  oidx[p] = (int32_t)e.y;
-  oval[p] = __uint_as_float(e.x);
+  out.put(p, e);
 }
 
 // Warp 0 of a group: over a 256-bucket histogram h (bucket 255 ranks
@@ -328,28 +358,26 @@ __device__ void radix_level(const Src& src, int n, uint64_t prefix, uint64_t mas
 
 // Emits every entry of `src` (passing its filter) with (key & mask) >= prefix.
 template <class Src>
-__device__ void emit_at_least(const Src& src, int n, uint64_t prefix, uint64_t mask, RowState& st, int32_t* oidx,
-                              float* oval, int tid, int nthr, int bar) {
+__device__ void emit_at_least(const Src& src, int n, uint64_t prefix, uint64_t mask, RowState& st, const RowOut& out,
+                              int tid, int nthr, int bar) {
   for (int i = tid; i < n; i += nthr) {
     uint2 e;
     if (!src.get(i, e)) continue;
-    if ((sel_key(e) & mask) >= prefix) emit(st, e, oidx, oval);
+    if ((sel_key(e) & mask) >= prefix) emit(st, e, out);
   }
   named_bar(bar, nthr);
 }
 
 // Warp-aggregated output: lanes with `sel` write their entry at
 // consecutive output slots.  All 32 lanes of the warp call it.
-__device__ __forceinline__ void emit_warp(RowState& st, bool sel, uint2 e, int32_t* oidx, float* oval, int lane) {
+__device__ __forceinline__ void emit_warp(RowState& st, bool sel, uint2 e, const RowOut& out, int lane) {
   const unsigned m = __ballot_sync(0xffffffffu, sel);
   if (m == 0u) return;
   int base = 0;
   if (lane == __ffs(m) - 1) base = atomicAdd(&st.outpos, __popc(m));
   base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
   if (sel) {
-    const int p = base + __popc(m & ((1u << lane) - 1u));
-    oidx[p] = (int32_t)e.y;
-    oval[p] = __uint_as_float(e.x);
+    out.put(base + __popc(m & ((1u << lane) - 1u)), e);
   }
 }
 
@@ -373,13 +401,13 @@ template <class F>
 __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nthr, F&& f) {
   for (int s = 0; s < c.nseg; ++s) {
     const uint2* seg = c.base + s * c.stride;
-    const int n = c.cnt[s];
+    const int n = c.count(s);
     for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
       uint2 e[kBatch];
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * nthr + tid;
-        e[j] = (i < n) ? seg[i] : make_uint2(0u, 0u);
+        e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) f(e[j], i0 + j * nthr + tid < n);
@@ -393,12 +421,12 @@ __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nt
 // Output and stage slots are taken with one warp scan and one atomic per
 // warp and batch.  All nthr threads call it (nthr a multiple of 32).
 template <class Cls>
-__device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nthr, RowState& st, int32_t* oidx,
-                                              float* oval, uint2* stage, int stage_cap, Cls&& cls) {
+__device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nthr, RowState& st, const RowOut& out,
+                                              uint2* stage, int stage_cap, Cls&& cls) {
   const int lane = tid & 31;
   for (int s = 0; s < c.nseg; ++s) {
     const uint2* seg = c.base + s * c.stride;
-    const int n = c.cnt[s];
+    const int n = c.count(s);
     for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
       uint2 e[kBatch];
       int cat[kBatch];
@@ -406,7 +434,7 @@ __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nt
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * nthr + tid;
-        e[j] = (i < n) ? seg[i] : make_uint2(0u, 0u);
+        e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
@@ -428,8 +456,7 @@ __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nt
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         if (cat[j] == 1) {
-          oidx[be] = (int32_t)e[j].y;
-          oval[be] = __uint_as_float(e[j].x);
+          out.put(be, e[j]);
           ++be;
         } else if (cat[j] == 2) {
           if (bs < stage_cap) stage[bs] = e[j];
@@ -454,8 +481,8 @@ constexpr int kResolvePerThread = 8;  // staged entries per thread: stage_cap <=
 // already decided), drop or emit whole digit buckets until at most 128
 // entries remain undecided; those are ranked exactly by counting.
 // Group-wide (nthr threads, barrier `bar`).
-static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, int ns, int need, int shift, int32_t* oidx,
-                                           float* oval, int tid, int nthr, int bar) {
+static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, int ns, int need, int shift,
+                                                  const RowOut out, int tid, int nthr, int bar) {
   const int lane = tid & 31;
   uint64_t key[kResolvePerThread];
   bool live[kResolvePerThread];
@@ -481,7 +508,7 @@ static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, in
 #pragma unroll
     for (int j = 0; j < kResolvePerThread; ++j) {
       const int d = live[j] ? (int)((key[j] >> shift) & 255u) : -1;
-      emit_warp(st, d > dsel, key_entry(key[j]), oidx, oval, lane);
+      emit_warp(st, d > dsel, key_entry(key[j]), out, lane);
       live[j] = (d == dsel);
     }
     remaining -= above;
@@ -508,9 +535,7 @@ static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, in
     for (int j = 0; j < nlive; ++j) rank += kk[j] > mine;
     if (rank < remaining) {
       const uint2 e = key_entry(mine);
-      const int p = atomicAdd(&st.outpos, 1);
-      oidx[p] = (int32_t)e.y;
-      oval[p] = __uint_as_float(e.x);
+      out.put(atomicAdd(&st.outpos, 1), e);
     }
   }
   named_bar(bar, nthr);
@@ -522,12 +547,11 @@ static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, in
 __device__ __forceinline__ int digit_shift_below(int bin) { return (bin > 0 && bin < kBins - 1) ? 43 : 56; }
 
 // Final selection of one row: writes min(k, visible) entries to
-// oidx[0..k), oval[0..k) (any order), pads the rest with -1 / -inf, and
+// out[0..k) (any order), pads the rest with -1 / -inf, and
 // returns the number of real entries.  Group-wide call (nthr threads, a
 // multiple of 32, stage_cap <= 8 * nthr).  Expects st.bstar / st.cge exact
 // (no appends in flight).
-static __device__ __noinline__ int row_select(RowState& st, const CandList& cand, int k,
-                                              int32_t* __restrict__ oidx, float* __restrict__ oval,
+static __device__ __noinline__ int row_select(RowState& st, const CandList cand, int k, const RowOut out,
                                               uint2* __restrict__ stage, int stage_cap, int tid, int nthr, int bar,
                                               int* status) {
   named_bar(bar, nthr);
@@ -541,18 +565,15 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
   named_bar(bar, nthr);
   if (cge < k) {
     // b* never moved: every visible key was appended (n == cge < k)
-    classify_pass(cand, tid, nthr, st, oidx, oval, stage, 0, [](uint2) { return 1; });
+    classify_pass(cand, tid, nthr, st, out, stage, 0, [](uint2) { return 1; });
     named_bar(bar, nthr);
-    for (int i = n + tid; i < k; i += nthr) {
-      oidx[i] = -1;
-      oval[i] = __int_as_float(0xff800000);
-    }
+    for (int i = n + tid; i < k; i += nthr) out.pad(i);
     named_bar(bar, nthr);
     return n;
   }
   const int need = k - (cge - hb);
   // entries above the threshold bin are selected; the bin itself is staged
-  classify_pass(cand, tid, nthr, st, oidx, oval, stage, stage_cap, [bstar](uint2 e) {
+  classify_pass(cand, tid, nthr, st, out, stage, stage_cap, [bstar](uint2 e) {
     const int b = score_bin(__uint_as_float(e.x));
     return b > bstar ? 1 : (b == bstar ? 2 : 0);
   });
@@ -560,7 +581,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
   const int ns = st.stage_cnt;
   if (tid == 0 && (ns != hb || st.outpos != cge - hb)) report_error(status, DSA_ERR_INTERNAL, 1);
   if (ns <= stage_cap) {
-    stage_resolve(st, stage, ns, need, digit_shift_below(bstar), oidx, oval, tid, nthr, bar);
+    stage_resolve(st, stage, ns, need, digit_shift_below(bstar), out, tid, nthr, bar);
     return k;
   }
   // The threshold bin holds more entries than the stage.  Inside bins
@@ -583,14 +604,14 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
       named_bar(bar, nthr);
       if (tid == 0) st.stage_cnt = 0;
       named_bar(bar, nthr);
-      classify_pass(cand, tid, nthr, st, oidx, oval, stage, stage_cap, [bstar, dsel](uint2 e) {
+      classify_pass(cand, tid, nthr, st, out, stage, stage_cap, [bstar, dsel](uint2 e) {
         if (score_bin(__uint_as_float(e.x)) != bstar) return 0;
         const int dg = (int)((e.x >> 11) & 255u);
         return dg > dsel ? 1 : (dg == dsel ? 2 : 0);
       });
       named_bar(bar, nthr);
       if (tid == 0 && (st.stage_cnt != hsel || st.outpos != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
-      stage_resolve(st, stage, hsel, need - above, 35, oidx, oval, tid, nthr, bar);
+      stage_resolve(st, stage, hsel, need - above, 35, out, tid, nthr, bar);
       return k;
     }
     named_bar(bar, nthr);
@@ -620,17 +641,17 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList& cand
         if (!gsrc.get(i, e)) continue;
         const uint64_t km = sel_key(e) & mask;
         if (km > prefix) {
-          emit(st, e, oidx, oval);
+          emit(st, e, out);
         } else if (km == prefix) {
           stage[atomicAdd(&st.stage_cnt, 1)] = e;
         }
       }
       named_bar(bar, nthr);
-      stage_resolve(st, stage, hsel, remaining, shift - 8, oidx, oval, tid, nthr, bar);
+      stage_resolve(st, stage, hsel, remaining, shift - 8, out, tid, nthr, bar);
       return k;
     }
   }
-  emit_at_least(gsrc, n_all, prefix, mask, st, oidx, oval, tid, nthr, bar);
+  emit_at_least(gsrc, n_all, prefix, mask, st, out, tid, nthr, bar);
   return k;
 }
 
