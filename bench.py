@@ -54,8 +54,10 @@ class Workload:
 
     pairs: score pairs the metric counts per step (group modes: the
     dense-equivalent causal pairs); alg_pairs: pairs actually scored;
-    bound / alg_flops / alg_bytes: the roofline of the dominant kernel."""
+    bound / alg_flops / alg_bytes: the roofline of the dominant kernel (the
+    scoring kernel), summed over its launches in one step."""
     launches_per_step = 1
+    kernel_launches_per_step = 1   # launches of the scoring kernel (the dominant one)
     bound = "tensor"
     alg_bytes = 0
 
@@ -176,6 +178,7 @@ class Group(Workload):
         i = self.inp
         self.host_src = [i.q, i.w, i.k] + ([i.k_scale] if i.k_scale is not None else [])
         self.launches_per_step = (5 if mode == 0 else 3) + (1 if c["k_dtype"] == "fp8" else 0)
+        self.kernel_launches_per_step = 2 if mode == 0 else 1
 
     def describe(self):
         c = self.cfg
@@ -237,9 +240,10 @@ class Decode(Workload):
         self.pairs = self.alg_pairs = c["B"] * sum(c["Nb"] - m + j + 1 for j in range(m))
         self.alg_flops = self.alg_pairs * 2 * c["H"] * c["d"]
         i = self.inp
-        # compulsory HBM bytes: every cached key once, the queries, weights and outputs
+        # compulsory HBM bytes of the scoring kernel: every cached key once,
+        # the queries and weights (the merge kernel writes the outputs)
         self.alg_bytes = (i.k.numel() * i.k.element_size() + i.q.numel() * i.q.element_size()
-                          + i.w.numel() * 4 + i.q.shape[0] * self.k * 8)
+                          + i.w.numel() * 4)
         self.rows = i.q.shape[0]
         self.ko = i.k_offsets.to(device, torch.int64)
         self.qo = i.q_offsets.to(device, torch.int32)
@@ -376,12 +380,19 @@ def _barrier(dist):
         dist.barrier()
 
 
-def _max_over_ranks(dist, x):
+def _max_over_ranks(dist, x, device="cuda"):
+    """The slowest rank's time: every rank takes part, every rank gets it."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, world, steps, slowest_ms):
+    """Whole-job throughput of N replicas: the units all ranks processed in
+    the timed steps over the slowest rank's time (units per second)."""
+    return units_per_rank_step * world * steps / (slowest_ms / 1e3)
 
 
 def run_reference(args):
@@ -447,6 +458,10 @@ def main():
 
     clk = ClockSampler(local)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # the library records an event pair around each scoring-kernel launch
+    # on this stream (events created here, before the timed region)
+    n_kernel = wl.kernel_launches_per_step * args.steps
+    dsa.dsa_kernel_timer_start(n_kernel)
     _barrier(dist)
     torch.cuda.synchronize()
     clk.start()
@@ -457,36 +472,40 @@ def main():
     torch.cuda.synchronize()
     _barrier(dist)
     clocks = clk.stop()
+    kernel_ms, kernel_n = dsa.dsa_kernel_timer_stop()
+    if kernel_n != n_kernel:
+        raise RuntimeError(f"timed {kernel_n} scoring-kernel launches, expected {n_kernel}")
     wl.check()
     per = [e0.elapsed_time(e1) for e0, e1 in ev]  # ms per launch
     total_ms = ev[0][0].elapsed_time(ev[-1][1])
     total_ms = _max_over_ranks(dist, total_ms)
+    kernel_ms = _max_over_ranks(dist, kernel_ms)
     ms_step = total_ms / args.steps
-    pairs = wl.pairs * world
-    value = pairs * args.steps / (total_ms / 1e3) / 1e9
-    alg_value = wl.alg_pairs * world * args.steps / (total_ms / 1e3) / 1e9
-    rows_s = wl.rows * world * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(wl.pairs, world, args.steps, total_ms) / 1e9
+    alg_value = whole_job_rate(wl.alg_pairs, world, args.steps, total_ms) / 1e9
+    rows_s = whole_job_rate(wl.rows, world, args.steps, total_ms)
 
     pk = _peaks()
-    avg_launch = sum(per) / len(per)
-    single = wl.launches_per_step == 1
-    scope = ("the step is one launch of the dominant kernel" if single else
-             f"step-level: {wl.launches_per_step} launches per step timed together (a lower bound for the "
-             f"dominant kernel; its share is in the ncu launch list)")
+    avg_launch = kernel_ms / kernel_n                     # ms per scoring-kernel launch
+    scope = (f"kernel time from CUDA events around each of the {kernel_n} scoring-kernel launches in the timed "
+             f"region ({wl.kernel_launches_per_step} per step, {kernel_ms / args.steps:.4f} ms of the "
+             f"{ms_step:.4f} ms step)")
+    per_launch_flops = wl.alg_flops / wl.kernel_launches_per_step
+    per_launch_bytes = wl.alg_bytes / wl.kernel_launches_per_step
     if wl.bound == "tensor":
-        achieved = wl.alg_flops / (avg_launch / 1e3) / 1e12
+        achieved = per_launch_flops / (avg_launch / 1e3) / 1e12
         peak = pk["bf16_sus"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None,
+                "traffic": None, "alg_per_launch": per_launch_flops, "kernel_ms": avg_launch,
                 "note": f"algorithmic 2*H*d flop per scored pair; peak = {pk['src']} sustained cuBLAS bf16 "
                         f"(kernel timed inside a back-to-back loop); frac of burst peak "
                         f"{achieved / pk['bf16']:.3f}; {scope}"}
     else:
-        achieved = wl.alg_bytes / (avg_launch / 1e3) / 1e9
+        achieved = per_launch_bytes / (avg_launch / 1e3) / 1e9
         peak = pk["hbm"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": None,
-                "note": f"algorithmic bytes = cached keys once + queries + weights + outputs; peak = {pk['src']} "
+                "traffic": None, "alg_per_launch": per_launch_bytes, "kernel_ms": avg_launch,
+                "note": f"algorithmic bytes = cached keys once + queries + weights; peak = {pk['src']} "
                         f"copy bandwidth; {scope}"}
     traffic_file = os.path.join(ROOT, "profiles", f"{args.config}_traffic.json")
     if os.path.exists(traffic_file):
@@ -509,7 +528,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = _max_over_ranks(dist, e0.elapsed_time(e1))
-        e2e = {"value": wl.pairs * world * n_e2e / (e2e_ms / 1e3) / 1e9, "unit": "Gpairs/s",
+        e2e = {"value": whole_job_rate(wl.pairs, world, n_e2e, e2e_ms) / 1e9, "unit": "Gpairs/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "note": "pinned host inputs copied in, indexer run, idx/val copied out, every step"}
 

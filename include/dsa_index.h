@@ -144,7 +144,11 @@ int dsa_index_group(const void* Q, const float* w, const void* K,
  *   total_keys: k_offsets[B] (host value: rows of K; tensor copies never
  *          read beyond it).
  *   max_keys: an upper bound on every N_b (host value; sizes the split of
- *          each cache over the GPU's multiprocessors and the workspace).
+ *          each cache over the GPU's multiprocessors and the workspace);
+ *          max_keys <= total_keys.
+ *   On the tensor-core path (bf16 q, bf16 or fp8 k, H = 64, d = 128) K
+ *   rows are addressed with 32-bit coordinates: total_keys above
+ *   2^31 - 256 returns DSA_ERR_UNSUPPORTED.
  * ---------------------------------------------------------------------- */
 int dsa_index_decode_workspace_size(int B, int total_q, int max_keys, int H,
                                     int d, int k, int q_dtype, int k_dtype,
@@ -168,8 +172,8 @@ int dsa_index_decode(const void* Q, const float* w, const void* K,
  *   H = 64 and d = 128 (other shapes: DSA_ERR_UNSUPPORTED).  No workspace:
  *   the scratch (a status word and per-CTA candidate lists) lives in a fixed
  *   32 MiB array in device memory that every GPU loading this library holds
- *   until the process exits.  Rows need 4 * round_up(N, 128) * 8 bytes per
- *   CTA; the grid shrinks to fit, and N above about 1.04 million keys
+ *   until the process exits.  Each CTA needs 4 * round_up(N, 512) * 8 bytes
+ *   of it; the grid shrinks to fit, and N above about 1.04 million keys
  *   returns DSA_ERR_WORKSPACE.
  *   The first call on a device looks up that device's copy of the array
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
@@ -192,6 +196,30 @@ int dsa_debug_scores(const void* Q, const float* w, const void* K,
                      const float* K_scale, int T, int N, int H, int d,
                      int64_t q_pos0, int q_dtype, int k_dtype, float* S,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Kernel timer (instrumentation; the pages describe no counterpart).
+ *
+ * dsa_kernel_timer_start arms a process-wide timer: each later launch of the
+ * scoring kernel (tensor-core or fp32 CUDA-core; made by dsa_index_dense,
+ * dsa_index_group, dsa_index_decode, dsa_index_dense_static or
+ * dsa_debug_scores) records a CUDA event pair around itself on the caller's
+ * stream, for the first max_launches launches; later ones are not timed.
+ * The proxy, gather, rank, merge and widening kernels are never timed.  The
+ * events are created here, so arm the timer outside a timed region and
+ * outside CUDA graph capture.
+ *
+ * dsa_kernel_timer_stop disarms it, waits for the recorded events, writes the
+ * summed duration of the timed launches in milliseconds to *total_ms and
+ * their number to *launches, and destroys the events.
+ *
+ * Both return DSA_OK; DSA_ERR_INVALID_ARG for max_launches outside
+ * [1, 2^20], a start while armed, a stop while disarmed or a null pointer;
+ * DSA_ERR_CUDA if creating or reading an event fails.  Launches from several
+ * host threads are counted in the order they take a slot.
+ * ---------------------------------------------------------------------- */
+int dsa_kernel_timer_start(int max_launches);
+int dsa_kernel_timer_stop(float* total_ms, int* launches);
 
 #ifdef __cplusplus
 }

@@ -23,6 +23,8 @@ from ._binding import (  # noqa: F401
     dsa_index_decode,
     dsa_debug_scores,
     dsa_index_dense_static,
+    dsa_kernel_timer_start,
+    dsa_kernel_timer_stop,
     dsa_check_status,
     dense_workspace_bytes,
     group_workspace_bytes,

@@ -23,6 +23,7 @@ EXPORTED_SYMBOLS = (
     "dsa_index_group_workspace_size", "dsa_index_group",
     "dsa_index_decode_workspace_size", "dsa_index_decode",
     "dsa_debug_scores", "dsa_index_dense_static",
+    "dsa_kernel_timer_start", "dsa_kernel_timer_stop",
 )
 
 
@@ -53,6 +54,8 @@ _SIGS = {
                                   _vp, _vp, _c_sz, _vp]),
     "dsa_index_dense_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _vp, _vp,
                                         _vp]),
+    "dsa_kernel_timer_start": (_c_int, [_c_int]),
+    "dsa_kernel_timer_stop": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int)]),
 }
 
 
@@ -288,3 +291,15 @@ def dsa_index_dense_static(Q: torch.Tensor, w: torch.Tensor, K: torch.Tensor, k:
     _check(lib().dsa_index_dense_static(_ptr(Q), _ptr(w), _ptr(K), T, N, H, d, q_pos0, k, _ptr(idx), _ptr(val),
                                         _stream(stream)), "dsa_index_dense_static")
     return idx, val
+
+
+def dsa_kernel_timer_start(max_launches: int) -> None:
+    """Arm the library's scoring-kernel timer for up to ``max_launches`` launches."""
+    _check(lib().dsa_kernel_timer_start(int(max_launches)), "dsa_kernel_timer_start")
+
+
+def dsa_kernel_timer_stop() -> Tuple[float, int]:
+    """Disarm the timer; (summed kernel milliseconds, timed launches)."""
+    ms, n = ctypes.c_float(0.0), _c_int(0)
+    _check(lib().dsa_kernel_timer_stop(ctypes.byref(ms), ctypes.byref(n)), "dsa_kernel_timer_stop")
+    return float(ms.value), int(n.value)

@@ -546,9 +546,11 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
-  if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1) return DSA_ERR_INVALID_ARG;
+  if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1 || max_keys > total_keys) return DSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  // the tensor-core kernel addresses key rows with 32-bit TMA coordinates
+  if (use_tc(H, d, q_dtype, k_dtype) && total_keys > ((int64_t)1 << 31) - 256) return DSA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   DecodePlan p;

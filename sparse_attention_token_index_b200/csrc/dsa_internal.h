@@ -47,6 +47,14 @@ struct TcArgs {
   int T;
 };
 
+// Event pair for timing one scoring-kernel launch (dsa_timer.cu); both null
+// unless dsa_kernel_timer_start armed the timer and a slot is left.
+struct TimerSlot {
+  cudaEvent_t start = nullptr;
+  cudaEvent_t end = nullptr;
+};
+TimerSlot timer_acquire();
+
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream);
 size_t tc_smem_bytes();

@@ -114,8 +114,12 @@ int launch_simt_index(const SimtArgs& a, int grid, cudaStream_t stream) {
         cudaSuccess)
       return DSA_ERR_CUDA;
   }
+  const TimerSlot ts = timer_acquire();
+  if (ts.start) cudaEventRecord(ts.start, stream);
   simt_index_kernel<<<grid, kSimtThreads, smem, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (ts.end) cudaEventRecord(ts.end, stream);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace dsa

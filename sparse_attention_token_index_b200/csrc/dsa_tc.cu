@@ -459,13 +459,20 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream) {
-  if (a.dbg_scores != nullptr) return a.kind == 0 ? launch_tc<true, 0>(tmQ, tmK, a, grid, stream) : DSA_ERR_UNSUPPORTED;
-  switch (a.kind) {
-    case 0: return launch_tc<false, 0>(tmQ, tmK, a, grid, stream);
-    case 1: return launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
-    case 2: return launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
-    default: return DSA_ERR_INVALID_ARG;
-  }
+  if (a.kind < 0 || a.kind > 2 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
+  const TimerSlot ts = timer_acquire();
+  if (ts.start) cudaEventRecord(ts.start, stream);
+  int r;
+  if (a.dbg_scores != nullptr)
+    r = launch_tc<true, 0>(tmQ, tmK, a, grid, stream);
+  else if (a.kind == 0)
+    r = launch_tc<false, 0>(tmQ, tmK, a, grid, stream);
+  else if (a.kind == 1)
+    r = launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
+  else
+    r = launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
+  if (ts.end) cudaEventRecord(ts.end, stream);
+  return r;
 }
 
 size_t tc_smem_bytes() { return kTcSmemBytes; }

@@ -74,3 +74,22 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(2, 64, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         dsa.dsa_index_dense(q, torch.zeros(2, 64), torch.zeros(4, 128, dtype=torch.bfloat16), 2)
+
+
+def test_kernel_timer_host_checks(L):
+    ms, n = ctypes.c_float(0.0), ctypes.c_int(0)
+    # stop while disarmed, null outputs, and out-of-range counts are refused
+    # before any CUDA call
+    assert L.dsa_kernel_timer_stop(ctypes.byref(ms), ctypes.byref(n)) == -1
+    assert L.dsa_kernel_timer_stop(None, None) == -1
+    assert L.dsa_kernel_timer_start(0) == -1
+    assert L.dsa_kernel_timer_start((1 << 20) + 1) == -1
+
+
+def test_decode_host_checks(L):
+    ok = ctypes.c_void_p(4096)
+    f = L.dsa_index_decode
+    # max_keys above total_keys
+    assert f(ok, ok, ok, None, ok, ok, 1, 2, 100, 101, 64, 128, 16, 0, 0, ok, ok, ok, 1 << 20, None) == -1
+    # more keys than 32-bit TMA row coordinates reach (tensor-core shape)
+    assert f(ok, ok, ok, None, ok, ok, 1, 2, 1 << 31, 1 << 20, 64, 128, 16, 0, 0, ok, ok, ok, 1 << 20, None) == -2
