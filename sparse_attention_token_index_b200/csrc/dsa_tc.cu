@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------- epilogue: 16 warps in four warpgroups ----------------
     // A unit of nq queries gives each query a team of 4/nq warpgroups (one
     // for nq >= 3, the last warpgroup idle when nq == 3); team member m takes
-    // the tiles jt with jt % team == m, so the per-tile latency of a short
+    // the tiles jt with jt mod team == m (team is 1, 2 or 4), so the per-tile latency of a short
     // unit (decode, tails) overlaps across the team.  Per tile a warp waits
     // for its accumulator, pulls its 32 key rows x 64 heads out of TMEM,
     // frees the buffer, scores, and appends survivors of the threshold to its
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[q]);
       // per-unit scalars (kept in registers through the tile loop)
       const int64_t row = (int64_t)u.row0 + q;
-      const int64_t pos = active ? slot_pos<kKind>(a, u, q) : -1;
+      const int pos = active ? (int)slot_pos<kKind>(a, u, q) : -1;  // key positions fit in int (N <= INT_MAX)
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         tc_fence_after();
-        const bool mine = active && (jt % team) == member;
+        const bool mine = active && (jt & (team - 1)) == member;
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
         if (mine) {
@@ -401,13 +401,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (mine) {
           const int key = key0 + jt * kTileKeys;  // local key index
           const bool in_range = key < nkeys;
-          int64_t kpos = key;
-          if (kmap != nullptr) kpos = in_range ? (int64_t)kmap[key] : -1;
+          int kpos = key;
+          if (kmap != nullptr) kpos = in_range ? kmap[key] : -1;
           const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
           float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
           if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
-          const bool valid = in_range && kpos >= 0 && kpos <= pos;
+          const bool valid = in_range && (unsigned)kpos <= (unsigned)pos;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
           row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
         }
