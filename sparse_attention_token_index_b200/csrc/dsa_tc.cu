@@ -200,8 +200,11 @@ template <bool kDebug, int kKind>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_index_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ TcArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  TcSmem& S = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // 1024-byte aligned (128B-swizzled TMA tiles) by a byte offset from the
+  // __shared__ array itself, so every access through S stays a shared-memory
+  // access (a detour through an integer address would make them generic)
+  TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &S.abort_flag;
 
