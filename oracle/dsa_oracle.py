@@ -294,3 +294,51 @@ def decode(q, w, K, k_offsets, q_offsets, k, k_scale=None, return_scores=False):
     if return_scores:
         res["scores"] = scores
     return res
+
+
+def decode_group(q, w, K, k_offsets, q_offsets, k, bank, mode, k_scale=None, qbar=None, wbar=None,
+                 bank_override=None):
+    """PIVOT in decode: the new queries of one sequence form the group.
+
+    The PIVOT abstract names the queries decoded together in one
+    multi-token-prediction step as a natural group.  Sequence b (keys
+    K[k_offsets[b]:k_offsets[b+1]], N_b of them; query rows
+    q_offsets[b]..q_offsets[b+1]-1, m_b of them, query j at position
+    N_b - m_b + j) is one group of G = m_b: its proxy is the members' mean,
+    the proxy scans keys 0..N_b - 1 (the prefix of its last query), the bank is
+    the proxy's top-`bank`, and every query refines or reuses exactly as in
+    ``group``.  Indices are local to the sequence.
+
+    ``qbar`` [B, H, d] / ``wbar`` [B, H] replace the float64 means (a proxy as
+    another implementation rounded it); ``bank_override`` {b: bank indices}
+    replaces the proxy's bank.  Returns idx/val/count over all query rows and
+    bank_idx/bank_val/bank_scores {b: ...}.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    ko = np.asarray(k_offsets, dtype=np.int64)
+    qo = np.asarray(q_offsets, dtype=np.int64)
+    B = ko.shape[0] - 1
+    M = int(qo[-1])
+    out_i = np.full((M, k), -1, dtype=np.int64)
+    out_v = np.full((M, k), -np.inf, dtype=np.float64)
+    cnt = np.zeros(M, dtype=np.int64)
+    res = {"bank_idx": {}, "bank_val": {}, "bank_scores": {}}
+    Kall = np.asarray(K)
+    sc = None if k_scale is None else np.asarray(k_scale)
+    for b in range(B):
+        k0, k1 = int(ko[b]), int(ko[b + 1])
+        r0, r1 = int(qo[b]), int(qo[b + 1])
+        Nb, mb = k1 - k0, r1 - r0
+        r = group(q[r0:r1], w[r0:r1], Kall[k0:k1], k, mb, bank, mode, q_pos0=Nb - mb,
+                  k_scale=None if sc is None else sc[k0:k1],
+                  qbar=None if qbar is None else np.asarray(qbar)[b:b + 1],
+                  wbar=None if wbar is None else np.asarray(wbar)[b:b + 1],
+                  bank_override=None if bank_override is None or b not in bank_override
+                  else {0: bank_override[b]})
+        res["bank_idx"][b], res["bank_val"][b] = r["bank_idx"][0], r["bank_val"][0]
+        res["bank_scores"][b] = r["bank_scores"][0]
+        for j in range(mb):
+            out_i[r0 + j], out_v[r0 + j], cnt[r0 + j] = r["idx"][j], r["val"][j], r["count"][j]
+    res.update(idx=out_i, val=out_v, count=cnt)
+    return res

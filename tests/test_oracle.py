@@ -268,11 +268,52 @@ def pin_decode_matches_dense(O):
         assert np.array_equal(r["idx"][qo[b]:qo[b + 1]], dn["idx"]), b
 
 
+def pin_decode_group_hand(O):
+    g = _load("decode_group_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["K"], float)
+    for mode, key in ((O.REFINE, "refine"), (O.REUSE, "reuse")):
+        r = O.decode_group(q, w, K, g["k_offsets"], g["q_offsets"], g["k"], g["bank"], mode)
+        for b in range(2):
+            assert np.array_equal(r["bank_idx"][b], g["bank_idx"][b]), (key, b, r["bank_idx"][b])
+            assert np.array_equal(r["bank_val"][b], g["bank_val"][b]), (key, b, r["bank_val"][b])
+        assert np.array_equal(r["idx"], np.array(g[key + "_idx"])), (key, r["idx"])
+        assert np.array_equal(r["val"], np.array(g[key + "_val"])), (key, r["val"])
+    d = O.decode(q, w, K, g["k_offsets"], g["q_offsets"], g["k"])
+    assert np.array_equal(d["idx"], np.array(g["decode_idx"])) and np.array_equal(d["val"], g["decode_val"])
+
+
+def pin_decode_group_invariants(O):
+    rng = np.random.default_rng(11)
+    lengths, ms = [9, 6, 14, 5], [2, 1, 3, 4]
+    H, d, k = 2, 3, 3
+    q = rng.standard_normal((sum(ms), H, d))
+    w = rng.uniform(0, 1, (sum(ms), H))
+    K = rng.standard_normal((sum(lengths), d))
+    ko = np.concatenate([[0], np.cumsum(lengths)])
+    qo = np.concatenate([[0], np.cumsum(ms)])
+    dec = O.decode(q, w, K, ko, qo, k)
+    # a bank as large as every cache makes Refine the decode indexer
+    r = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE)
+    assert np.array_equal(r["idx"], dec["idx"]) and np.array_equal(r["val"], dec["val"])
+    rf = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE)
+    ru = O.decode_group(q, w, K, ko, qo, k, 4, O.REUSE)
+    for b in range(4):
+        last = qo[b + 1] - 1
+        # the last query may see the whole bank: Reuse gives it the proxy's top-k
+        n = ru["count"][last]
+        assert np.array_equal(ru["idx"][last][:n], ru["bank_idx"][b][:k]), b
+        if ms[b] == 1:
+            # one query: the proxy is the query, so all three agree
+            assert np.array_equal(rf["idx"][last], dec["idx"][last]), b
+            assert np.array_equal(ru["idx"][last], dec["idx"][last]), b
+            assert np.allclose(ru["val"][last], dec["val"][last], rtol=1e-12), b
+
+
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
         pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
-        pin_decode_matches_dense]
+        pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -380,10 +421,47 @@ def _m_decode_first_positions(mp):
     mp.setattr(O, "decode", bad)
 
 
+def _m_decode_group_first_positions(mp):
+    # the group's queries placed at the first m_b positions of their cache
+    real_group = O.group
+
+    def bad(q, w, K, k, G, bank, mode, q_pos0=0, **kw):
+        return real_group(q, w, K, k, G, bank, mode, q_pos0=0, **kw)
+    real = O.decode_group
+
+    def dg(*a, **kw):
+        with pytest.MonkeyPatch.context() as m2:
+            m2.setattr(O, "group", bad)
+            return real(*a, **kw)
+    mp.setattr(O, "decode_group", dg)
+
+
+def _m_decode_group_scan_first_member(mp):
+    # the proxy scans only its first member's prefix: the cache cut at N_b - m_b + 1
+    real = O.decode_group
+
+    def dg(q, w, K, k_offsets, q_offsets, k, bank, mode, **kw):
+        ko, qo = np.asarray(k_offsets), np.asarray(q_offsets)
+        out_i = np.full((int(qo[-1]), k), -1, dtype=np.int64)
+        out_v = np.full((int(qo[-1]), k), -np.inf)
+        res = {"bank_idx": {}, "bank_val": {}, "count": np.zeros(int(qo[-1]), dtype=np.int64)}
+        for b in range(len(ko) - 1):
+            Nb, mb = int(ko[b + 1] - ko[b]), int(qo[b + 1] - qo[b])
+            r = real(q[qo[b]:qo[b + 1]], w[qo[b]:qo[b + 1]], K[ko[b]:ko[b] + Nb - mb + 1], [0, Nb - mb + 1],
+                     [0, mb], k, bank, mode)
+            out_i[qo[b]:qo[b + 1]], out_v[qo[b]:qo[b + 1]] = r["idx"], r["val"]
+            res["bank_idx"][b], res["bank_val"][b] = r["bank_idx"][0], r["bank_val"][0]
+            res["count"][qo[b]:qo[b + 1]] = r["count"]
+        res.update(idx=out_i, val=out_v)
+        return res
+    mp.setattr(O, "decode_group", dg)
+
+
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
-           _m_proxy_first_member, _m_decode_first_positions]
+           _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
+           _m_decode_group_scan_first_member]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
