@@ -177,7 +177,8 @@ class Group(Workload):
         self.rows = self.T
         i = self.inp
         self.host_src = [i.q, i.w, i.k] + ([i.k_scale] if i.k_scale is not None else [])
-        self.launches_per_step = (5 if mode == 0 else 3) + (1 if c["k_dtype"] == "fp8" else 0)
+        # proxy mean, proxy scan, then Refine: bank gather + re-scoring; Reuse: bank ranking
+        self.launches_per_step = (4 if mode == 0 else 3) + (1 if c["k_dtype"] == "fp8" else 0)
         self.kernel_launches_per_step = 2 if mode == 0 else 1
 
     def describe(self):
@@ -380,6 +381,32 @@ def _barrier(dist):
         dist.barrier()
 
 
+def _kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("dsa_tc.cu", "dsa_topk.cuh", "dsa_common.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_token_index_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(config):
+    """ncu DRAM bytes per scoring-kernel launch from profiles/, or None when
+    there is no capture for this workload or the kernel changed since."""
+    p = os.path.join(ROOT, "profiles", f"{config}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                a, b = line.split("=", 1)
+                kv[a.strip()] = b.strip()
+    if kv.get("kernel_source") != _kernel_source_hash():
+        return None
+    return int(kv["bytes_per_launch"])
+
+
 def _max_over_ranks(dist, x, device="cuda"):
     """The slowest rank's time: every rank takes part, every rank gets it."""
     if dist is None:
@@ -507,10 +534,7 @@ def main():
                 "traffic": None, "alg_per_launch": per_launch_bytes, "kernel_ms": avg_launch,
                 "note": f"algorithmic bytes = cached keys once + queries + weights; peak = {pk['src']} "
                         f"copy bandwidth; {scope}"}
-    traffic_file = os.path.join(ROOT, "profiles", f"{args.config}_traffic.json")
-    if os.path.exists(traffic_file):
-        with open(traffic_file) as f:
-            roof["traffic"] = json.load(f).get("bytes_per_launch")
+    roof["traffic"] = _traffic(args.config)
 
     e2e = None
     if not args.no_e2e:

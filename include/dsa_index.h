@@ -115,8 +115,11 @@ int dsa_index_dense(const void* Q, const float* w, const void* K,
  *          wbar[g] = mean of the members' w (fp32).  The proxy scans keys
  *          0..L_g, L_g = position of the group's last member.
  *   bank_idx [ng, B] int32, bank_val [ng, B] fp32: optional outputs (NULL to
- *          skip) — the bank in the proxy's ranking order (Reuse needs that
- *          order; for Refine it is a set).  Unused slots: -1 / -inf.
+ *          skip) — the bank in the proxy's ranking order (score descending,
+ *          lower key first).  Unused slots: -1 / -inf.  Asking for them
+ *          costs a sort of every group's bank; without them Refine does not
+ *          rank the bank (it re-scores it as a set) and Reuse ranks only the
+ *          bank's top k + G - 1 entries, the only ones a member can take.
  *   proxy_q [ng, H, d] (q_dtype), proxy_w [ng, H] fp32: optional outputs.
  * ---------------------------------------------------------------------- */
 int dsa_index_group_workspace_size(int T, int N, int H, int d, int k,

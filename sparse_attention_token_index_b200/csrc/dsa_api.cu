@@ -425,10 +425,14 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   if ((r = run_dense_rows(di, gp.scan, qbar, wbar, K, K_scale, gp.ng, N, H, d, q_pos0, group, group - 1,
                           (int64_t)T - 1, bank, q_dtype, k_dtype, bi, bv, ws, nullptr, 0, st)) != DSA_OK)
     return r;
-  // 3. rank the bank; Reuse finishes here
-  if ((r = launch_bank_rank_reuse(bi, bv, gp.ng, bank, group, T, q_pos0, k, idx, val, mode == DSA_GROUP_REUSE,
-                                  st)) != DSA_OK)
-    return r;
+  // 3. Reuse ranks the bank and finishes here.  Refine uses the bank as a
+  // set; it is ranked only when the caller asked for it.
+  const bool want_bank = bank_idx != nullptr || bank_val != nullptr;
+  if (mode == DSA_GROUP_REUSE || want_bank) {
+    if ((r = launch_bank_rank_reuse(bi, bv, gp.ng, bank, group, T, q_pos0, k, idx, val, mode == DSA_GROUP_REUSE,
+                                    want_bank, st)) != DSA_OK)
+      return r;
+  }
   if (mode == DSA_GROUP_REUSE) return DSA_OK;
   // 4. Refine: members re-score their group's bank on tensor cores
   void* Kg = ws + gp.kg_off;

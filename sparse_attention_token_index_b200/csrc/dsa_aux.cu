@@ -104,67 +104,150 @@ int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, i
 
 // ---------------------------------------------------------------------------
 // bank ranking + Reuse.  One CTA per group; the bank (at most 16384 entries)
-// is sorted in shared memory as 64-bit keys (order-preserving score bits,
-// inverted key index), largest first.
+// is held in shared memory as 64-bit keys (order-preserving score bits,
+// inverted key index: larger key = higher rank, unique per entry).
+//   M == B: the whole bank is sorted, largest first, and written back.
+//   M <  B: only the M highest keys are needed (Reuse without a bank output:
+//           member t drops at most G - 1 bank keys, those of its own group
+//           above p_t, so its first k lie among the top k + G - 1).  An MSD
+//           radix select on 8-bit digits finds the M-th key, the M keys at or
+//           above it are compacted and only they are sorted.
 // ---------------------------------------------------------------------------
 constexpr int kRankThreads = 512;
 
 __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* __restrict__ bank_idx,
                                                                        float* __restrict__ bank_val, int B, int P,
-                                                                       int G, int T, int64_t q_pos0, int k,
-                                                                       int32_t* __restrict__ out_idx,
+                                                                       int M, int PM, int G, int T, int64_t q_pos0,
+                                                                       int k, int32_t* __restrict__ out_idx,
                                                                        float* __restrict__ out_val, int do_reuse) {
-  extern __shared__ uint64_t keys[];
-  const int g = blockIdx.x;
+  extern __shared__ uint64_t keys[];  // [P] the bank; then [PM] its top M when M < B
+  __shared__ uint32_t hist[256];
+  __shared__ int sh_digit, sh_above, sh_in, sh_cnt;
+  const int g = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   int32_t* bi = bank_idx + (int64_t)g * B;
   float* bv = bank_val + (int64_t)g * B;
-  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+  if (tid == 0) sh_cnt = 0;
+  int mine = 0;
+  for (int i = tid; i < P; i += blockDim.x) {
     uint64_t key = 0;
     if (i < B && bi[i] >= 0) key = sel_key(make_uint2(__float_as_uint(bv[i]), (uint32_t)bi[i]));
     keys[i] = key;
+    mine += key != 0;
   }
   __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
+  if (mine) atomicAdd(&sh_cnt, mine);
+  __syncthreads();
+  const int nvalid = sh_cnt;
+  __syncthreads();  // every thread has read the count before sh_cnt is reused
+  uint64_t* rk = keys;  // the array that gets sorted, R entries
+  int R = P;
+  if (M < B) {
+    uint64_t prefix = 0, mask = 0;
+    if (nvalid > M) {
+      int remaining = M;
+      for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < P; i += blockDim.x) {
+          const uint64_t key = keys[i];
+          if (key != 0 && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+          // digit holding the remaining-th largest, scanning from digit 255 down
+          uint32_t c[8], tot = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            c[j] = hist[255 - 8 * lane - j];
+            tot += c[j];
+          }
+          uint32_t incl = tot;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const uint32_t excl = incl - tot;
+          if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
+            uint32_t cum = excl;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (cum + c[j] >= (uint32_t)remaining) {
+                sh_digit = 255 - 8 * lane - j;
+                sh_above = (int)cum;
+                sh_in = (int)c[j];
+                break;
+              }
+              cum += c[j];
+            }
+          }
+        }
+        __syncthreads();
+        const int dsel = sh_digit, above = sh_above, in = sh_in;
+        __syncthreads();
+        remaining -= above;
+        prefix |= (uint64_t)dsel << shift;
+        mask |= (uint64_t)0xFFu << shift;
+        if (in == remaining) break;  // the whole digit bucket is in: keys with (key & mask) >= prefix
+      }
+    }
+    // compact the top min(M, nvalid) keys (any order), then sort only them
+    uint64_t* top = keys + P;
+    if (tid == 0) sh_cnt = 0;
+    __syncthreads();
+    for (int i = tid; i < P; i += blockDim.x) {
+      const uint64_t key = keys[i];
+      if (key != 0 && (key & mask) >= prefix) top[atomicAdd(&sh_cnt, 1)] = key;
+    }
+    __syncthreads();
+    for (int i = sh_cnt + tid; i < PM; i += blockDim.x) top[i] = 0;
+    __syncthreads();
+    rk = top;
+    R = PM;
+  }
+  for (int size = 2; size <= R; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (P >> 1); i += blockDim.x) {
+      for (int i = tid; i < (R >> 1); i += blockDim.x) {
         const int lo = 2 * i - (i & (stride - 1));
         const int hi = lo + stride;
         const bool up = (lo & size) == 0;
-        const uint64_t x = keys[lo], y = keys[hi];
+        const uint64_t x = rk[lo], y = rk[hi];
         if ((x < y) == up) {
-          keys[lo] = y;
-          keys[hi] = x;
+          rk[lo] = y;
+          rk[hi] = x;
         }
       }
       __syncthreads();
     }
   }
-  // ranked bank back to global (empty slots last: -1 / -inf)
-  for (int i = threadIdx.x; i < B; i += blockDim.x) {
-    const uint64_t key = keys[i];
-    if (key == 0) {
-      bi[i] = -1;
-      bv[i] = __int_as_float(0xff800000);
-    } else {
-      const uint32_t o = (uint32_t)(key >> 32);
-      const uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
-      bi[i] = (int32_t)(~(uint32_t)key);
-      bv[i] = __uint_as_float(u);
+  if (M == B) {
+    // ranked bank back to global (empty slots last: -1 / -inf)
+    for (int i = tid; i < B; i += blockDim.x) {
+      const uint64_t key = keys[i];
+      if (key == 0) {
+        bi[i] = -1;
+        bv[i] = __int_as_float(0xff800000);
+      } else {
+        const uint32_t o = (uint32_t)(key >> 32);
+        const uint32_t u = (o & 0x80000000u) ? (o & 0x7fffffffu) : ~o;
+        bi[i] = (int32_t)(~(uint32_t)key);
+        bv[i] = __uint_as_float(u);
+      }
     }
   }
   if (!do_reuse) return;
-  __syncthreads();
+  const int NR = M < R ? M : R;  // ranked entries a member may take from
   // Reuse: warp per member, first k ranked keys with position <= p_t
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int r0 = g * G, r1 = min(T, r0 + G);
   for (int r = r0 + warp; r < r1; r += nw) {
     const int64_t p = q_pos0 + r;
     int32_t* oi = out_idx + (int64_t)r * k;
     float* ov = out_val + (int64_t)r * k;
     int cnt = 0;
-    for (int i0 = 0; i0 < B && cnt < k; i0 += 32) {
+    for (int i0 = 0; i0 < NR && cnt < k; i0 += 32) {
       const int i = i0 + lane;
-      uint64_t key = (i < B) ? keys[i] : 0;
+      uint64_t key = (i < NR) ? rk[i] : 0;
       const int32_t kidx = (int32_t)(~(uint32_t)key);
       const bool keep = key != 0 && (int64_t)kidx <= p;
       const unsigned m = __ballot_sync(0xffffffffu, keep);
@@ -185,15 +268,25 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
 }
 
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T, int64_t q_pos0,
-                           int k, int32_t* out_idx, float* out_val, int do_reuse, cudaStream_t stream) {
+                           int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all, cudaStream_t stream) {
   int P = 1;
   while (P < bank_size) P <<= 1;
   if (P > 16384) return DSA_ERR_UNSUPPORTED;
-  const size_t smem = (size_t)P * sizeof(uint64_t);
+  int M = bank_size, PM = 0;
+  if (!rank_all) {
+    const int64_t m = (int64_t)k + G - 1;
+    if (m < bank_size) {
+      PM = 1;
+      while (PM < m) PM <<= 1;
+      if ((size_t)(P + PM) * sizeof(uint64_t) <= 200 * 1024) M = (int)m;
+      else PM = 0;
+    }
+  }
+  const size_t smem = (size_t)(P + PM) * sizeof(uint64_t);
   if (smem > 48 * 1024 && cudaFuncSetAttribute(bank_rank_reuse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)smem) != cudaSuccess)
     return DSA_ERR_CUDA;
-  bank_rank_reuse_kernel<<<ng, kRankThreads, smem, stream>>>(bank_idx, bank_val, bank_size, P, G, T, q_pos0, k,
+  bank_rank_reuse_kernel<<<ng, kRankThreads, smem, stream>>>(bank_idx, bank_val, bank_size, P, M, PM, G, T, q_pos0, k,
                                                              out_idx, out_val, do_reuse);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

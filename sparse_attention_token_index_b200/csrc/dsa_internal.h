@@ -93,8 +93,10 @@ int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G,
                       float* wbar, cudaStream_t stream);
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
                        void* Kg, cudaStream_t stream);
+// rank_all: sort and write back the whole bank; otherwise only the top
+// k + G - 1 entries are ranked (enough for Reuse) and the bank is not written.
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,
-                           int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse,
+                           int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all,
                            cudaStream_t stream);
 int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
                         int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,

@@ -101,6 +101,27 @@ def test_group_size_one_matches_dense():
             assert set(a[t].tolist()) == set(b[t].tolist()), (mode, t)
 
 
+def _same_rows(a_idx, a_val, b_idx, b_val):
+    # equal row sets (outputs are sets): sort each row by index on the device
+    ai, ap = torch.sort(a_idx, dim=1)
+    bi, bp = torch.sort(b_idx, dim=1)
+    assert torch.equal(ai, bi)
+    assert torch.equal(torch.gather(a_val, 1, ap), torch.gather(b_val, 1, bp))
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("shape", [(640, 640, 64, 256, 64), (100, 700, 6, 48, 16), (300, 300, 64, 2048, 100)],
+                         ids=["G64", "G6", "bank-ge-prefix"])
+def test_group_without_bank_output(mode, shape):
+    # without a bank output Refine skips the ranking and Reuse ranks only the
+    # top k + G - 1 bank entries: member outputs equal the fully ranked path's
+    T, N, G, B, k = shape
+    inp = make_dense_inputs("group_bf16_128k", device=DEV, T=T, N=N, seed=25)
+    fi, fv, _, _, _, _ = _run_group(inp, k, G, B, mode)
+    pi, pv = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0, check=True)
+    _same_rows(fi, fv, pi, pv)
+
+
 def test_group_full_size_sampled():
     # the 128K group workload (G = 64, B = 8192, k = 2048), sampled groups
     inp = make_dense_inputs("group_bf16_128k", device=DEV)
@@ -108,6 +129,10 @@ def test_group_full_size_sampled():
     T = inp.q.shape[0]
     for mode in (0, 1):
         idx, val, bidx, bval, pq, pw = _run_group(inp, k, G, B, mode)
+        # the bench's call (no bank output) gives the same member sets
+        pi, pv = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0, check=True)
+        _same_rows(idx, val, pi, pv)
+        del pi, pv
         K = _f64(inp.k)
         gq, gw = _f64(pq), _f64(pw)
         bi, bv = bidx.cpu().numpy(), bval.cpu().numpy()
