@@ -228,6 +228,7 @@ class Group(Workload):
 class Decode(Workload):
     name = "decode_bf16_32x128k"
     bound = "hbm"
+    alg_bytes_note = "cached keys once + queries + weights"
 
     def __init__(self, device, size=None):
         from synthetic import CONFIGS, make_decode_inputs
@@ -293,9 +294,77 @@ class Decode(Workload):
         return self._oracle_loop(budget_s, one)
 
 
+class DecodeGroup(Decode):
+    """PIVOT in decode: each sequence's new queries form one group (bank 8192)."""
+    bank = 8192
+    alg_bytes_note = "cached keys once + proxies (+ Refine: gathered bank keys, queries, weights)"
+
+    def __init__(self, device, size=None, mode=0):
+        super().__init__(device, size)
+        c = self.cfg
+        self.mode = mode
+        m, nb = c["m"], c["Nb"]
+        # proxy scan over every cache, then (Refine) each query over the bank
+        self.alg_pairs = c["B"] * nb + (c["B"] * m * min(self.bank, nb) if mode == 0 else 0)
+        self.alg_flops = self.alg_pairs * 2 * c["H"] * c["d"]
+        i = self.inp
+        # compulsory HBM bytes of the scoring kernels: every cached key once and
+        # the proxies; Refine adds its gathered bank keys and its queries
+        self.alg_bytes = i.k.numel() * i.k.element_size() + c["B"] * c["H"] * (c["d"] * 2 + 4)
+        if mode == 0:
+            self.alg_bytes += c["B"] * min(self.bank, nb) * c["d"] * 2 + i.q.numel() * 2 + i.w.numel() * 4
+        self.kernel_launches_per_step = 2 if mode == 0 else 1
+        # proxy mean, scan, merge, then Refine: gather + re-scoring; Reuse: ranking
+        self.launches_per_step = 5 if mode == 0 else 4
+
+    def describe(self):
+        d = super().describe()
+        m = "Refine" if self.mode == 0 else "Reuse"
+        d["workload"] = d["workload"].replace("decode,", f"decode group ({m}, bank {self.bank}, group = a sequence's "
+                                                           f"new queries),")
+        d["bank"], d["mode"] = self.bank, m
+        d["metric_pairs"] = "dense-equivalent decode pairs (alg_pairs = proxy scan + bank re-scoring)"
+        return d
+
+    def setup(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        c = self.cfg
+        self.ws = torch.zeros(dsa.decode_group_workspace_bytes(c["B"], i.q.shape[0], c["Nb"], c["H"], c["d"],
+                                                               self.k, self.bank, 0, 0),
+                              dtype=torch.uint8, device=i.q.device)
+        self.out = (torch.empty((i.q.shape[0], self.k), dtype=torch.int32, device=i.q.device),
+                    torch.empty((i.q.shape[0], self.k), dtype=torch.float32, device=i.q.device))
+
+    def call(self, q, w, k):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_decode_group(q, w, k, self.k, self.ko, self.qo, self.bank, mode=self.mode,
+                                   max_keys=self.cfg["Nb"], total_keys=self.total_keys, out=self.out,
+                                   workspace=self.ws)
+
+    def oracle_sample(self, budget_s=15.0, seed=0):
+        from oracle import dsa_oracle as O
+        i = self.inp
+        c = self.cfg
+        rng = np.random.default_rng(seed)
+        m, nb = c["m"], c["Nb"]
+
+        def one(_):
+            # one whole sequence: proxy scan + its queries; counted like the
+            # GPU arm (the queries' dense-equivalent pairs)
+            b = int(rng.integers(0, c["B"]))
+            K = _f64(i.k[b * nb:(b + 1) * nb])
+            O.decode_group(_f64(i.q[b * m:(b + 1) * m]), _f64(i.w[b * m:(b + 1) * m]), K, [0, nb], [0, m],
+                           self.k, self.bank, self.mode)
+            return sum(nb - m + j + 1 for j in range(m))
+        return self._oracle_loop(budget_s, one)
+
+
 WORKLOADS = {
     "dense_bf16_32k": lambda dev, size: Dense(dev, size),
     "decode_bf16_32x128k": lambda dev, size: Decode(dev, size),
+    "decode_bf16_32x128k_group_refine": lambda dev, size: DecodeGroup(dev, size, 0),
+    "decode_bf16_32x128k_group_reuse": lambda dev, size: DecodeGroup(dev, size, 1),
     "group_bf16_128k_refine": lambda dev, size: Group(dev, size, "group_bf16_128k", 0),
     "group_bf16_128k_reuse": lambda dev, size: Group(dev, size, "group_bf16_128k", 1),
     "dense_bf16_128k": lambda dev, size: Dense(dev, size or 131072, name="group_bf16_128k"),
@@ -532,7 +601,7 @@ def main():
         peak = pk["hbm"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": None, "alg_per_launch": per_launch_bytes, "kernel_ms": avg_launch,
-                "note": f"algorithmic bytes = cached keys once + queries + weights; peak = {pk['src']} "
+                "note": f"algorithmic bytes = {wl.alg_bytes_note}; peak = {pk['src']} "
                         f"copy bandwidth; {scope}"}
     roof["traffic"] = _traffic(args.config)
 

@@ -165,6 +165,39 @@ int dsa_index_decode(const void* Q, const float* w, const void* K,
                      size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * PIVOT in decode (PIVOT abstract: the queries decoded together in one
+ * multi-token-prediction step form a natural group).  Sequence b's m_b new
+ * queries are one group:
+ *   proxy   qbar[b] = mean of its queries' q (fp32 mean, rounded to q_dtype),
+ *           wbar[b] = mean of their w (fp32); the proxy sits at the last
+ *           query's position N_b - 1 and scans keys 0..N_b - 1;
+ *   bank    the proxy's top-`bank` keys (indices local to the sequence);
+ *   mode    DSA_GROUP_REFINE: query j (position N_b - m_b + j) re-scores the
+ *           bank keys <= its position with its own q, w and keeps its top-k;
+ *           DSA_GROUP_REUSE: it keeps the first k bank keys <= its position
+ *           in the proxy's ranking, valued by the proxy score.
+ *   Arguments as for dsa_index_decode (1 <= m_b <= min(4, N_b), device
+ *   offsets, local output indices), plus bank (k <= bank <= 16384), mode and
+ *   the optional outputs bank_idx/bank_val [B, bank] (ranked, -1 / -inf
+ *   padded; asking for them costs a sort of every bank) and proxy_q
+ *   [B, H, d] (q_dtype) / proxy_w [B, H] fp32.  Tensor-core shape only (bf16
+ *   q, bf16 or fp8 k, H = 64, d = 128); other shapes DSA_ERR_UNSUPPORTED.
+ * ---------------------------------------------------------------------- */
+int dsa_index_decode_group_workspace_size(int B, int total_q, int max_keys,
+                                          int H, int d, int k, int bank,
+                                          int q_dtype, int k_dtype,
+                                          size_t* bytes);
+int dsa_index_decode_group(const void* Q, const float* w, const void* K,
+                           const float* K_scale, const int64_t* k_offsets,
+                           const int32_t* q_offsets, int B, int total_q,
+                           int64_t total_keys, int max_keys, int H, int d,
+                           int k, int bank, int mode, int q_dtype,
+                           int k_dtype, int32_t* idx, float* val,
+                           int32_t* bank_idx, float* bank_val, void* proxy_q,
+                           float* proxy_w, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dense indexer that allocates nothing (the pages have no counterpart: this
  * is an integration aid).  For callers that cannot hand the library a
  * workspace — code running inside a host application that reserved all

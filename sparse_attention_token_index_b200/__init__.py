@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     dsa_index_dense,
     dsa_index_group,
     dsa_index_decode,
+    dsa_index_decode_group,
     dsa_debug_scores,
     dsa_index_dense_static,
     dsa_kernel_timer_start,
@@ -29,5 +30,6 @@ from ._binding import (  # noqa: F401
     dense_workspace_bytes,
     group_workspace_bytes,
     decode_workspace_bytes,
+    decode_group_workspace_bytes,
     EXPORTED_SYMBOLS,
 )

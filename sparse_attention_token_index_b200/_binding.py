@@ -24,6 +24,7 @@ EXPORTED_SYMBOLS = (
     "dsa_index_decode_workspace_size", "dsa_index_decode",
     "dsa_debug_scores", "dsa_index_dense_static",
     "dsa_kernel_timer_start", "dsa_kernel_timer_stop",
+    "dsa_index_decode_group_workspace_size", "dsa_index_decode_group",
 )
 
 
@@ -55,6 +56,10 @@ _SIGS = {
     "dsa_index_dense_static": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _vp, _vp,
                                         _vp]),
     "dsa_kernel_timer_start": (_c_int, [_c_int]),
+    "dsa_index_decode_group_workspace_size": (_c_int, [_c_int] * 9 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_decode_group": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                        _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _c_sz, _vp]),
     "dsa_kernel_timer_stop": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int)]),
 }
 
@@ -232,16 +237,7 @@ def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
-    if max_keys is None or total_keys is None:
-        ko_host = k_offsets.to("cpu", torch.int64)
-        if max_keys is None:
-            max_keys = int((ko_host[1:] - ko_host[:-1]).max())
-        if total_keys is None:
-            total_keys = int(ko_host[-1])
-    ko = k_offsets if (k_offsets.is_cuda and k_offsets.dtype == torch.int64) else \
-        k_offsets.to(Q.device, torch.int64).contiguous()
-    qo = q_offsets if (q_offsets.is_cuda and q_offsets.dtype == torch.int32) else \
-        q_offsets.to(Q.device, torch.int32).contiguous()
+    ko, qo, max_keys, total_keys = _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys)
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     nb = decode_workspace_bytes(B, total_q, max_keys, H, d, k, qd, kd)
     ws = _workspace(nb, Q.device, workspace)
@@ -252,6 +248,66 @@ def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.
     if check:
         dsa_check_status(ws, stream)
     return idx, val
+
+
+def decode_group_workspace_bytes(B, total_q, max_keys, H, d, k, bank, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_decode_group_workspace_size(B, total_q, max_keys, H, d, k, bank, q_dtype, k_dtype,
+                                                       ctypes.byref(n)), "dsa_index_decode_group_workspace_size")
+    return int(n.value)
+
+
+def _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys):
+    if max_keys is None or total_keys is None:
+        ko_host = k_offsets.to("cpu", torch.int64)
+        if max_keys is None:
+            max_keys = int((ko_host[1:] - ko_host[:-1]).max())
+        if total_keys is None:
+            total_keys = int(ko_host[-1])
+    ko = k_offsets if (k_offsets.is_cuda and k_offsets.dtype == torch.int64) else \
+        k_offsets.to(Q.device, torch.int64).contiguous()
+    qo = q_offsets if (q_offsets.is_cuda and q_offsets.dtype == torch.int32) else \
+        q_offsets.to(Q.device, torch.int32).contiguous()
+    return ko, qo, int(max_keys), int(total_keys)
+
+
+def dsa_index_decode_group(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.Tensor, bank: int,
+                           mode: int = DSA_GROUP_REFINE, max_keys: Optional[int] = None,
+                           total_keys: Optional[int] = None, K_scale=None, out=None, return_bank: bool = False,
+                           return_proxy: bool = False, workspace=None, stream=None, check: bool = False):
+    """PIVOT in decode: each sequence's new queries form one group.
+
+    Returns (idx [sum m_b, k], val) with indices local to each sequence and,
+    on request, (bank_idx [B, bank], bank_val) in the proxy's ranking order
+    and (proxy_q [B, H, d], proxy_w [B, H]).
+    """
+    _need_cuda(Q, w, K, K_scale)
+    total_q, H, d = Q.shape
+    B = k_offsets.numel() - 1
+    ko, qo, max_keys, total_keys = _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    nb = decode_group_workspace_bytes(B, total_q, max_keys, H, d, k, bank, qd, kd)
+    ws = _workspace(nb, Q.device, workspace)
+    idx, val = _outputs(total_q, k, Q.device, out)
+    bi = bv = pq = pw = None
+    if return_bank:
+        bi = torch.empty((B, bank), dtype=torch.int32, device=Q.device)
+        bv = torch.empty((B, bank), dtype=torch.float32, device=Q.device)
+    if return_proxy:
+        pq = torch.empty((B, H, d), dtype=Q.dtype, device=Q.device)
+        pw = torch.empty((B, H), dtype=torch.float32, device=Q.device)
+    _check(lib().dsa_index_decode_group(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), _ptr(ko), _ptr(qo), B, total_q,
+                                        total_keys, max_keys, H, d, k, bank, int(mode), qd, kd, _ptr(idx),
+                                        _ptr(val), _ptr(bi), _ptr(bv), _ptr(pq), _ptr(pw), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "dsa_index_decode_group")
+    if check:
+        dsa_check_status(ws, stream)
+    res = [idx, val]
+    if return_bank:
+        res += [bi, bv]
+    if return_proxy:
+        res += [pq, pw]
+    return tuple(res)
 
 
 def dsa_debug_scores(Q, w, K, q_pos0: Optional[int] = None, K_scale=None, workspace=None, stream=None,

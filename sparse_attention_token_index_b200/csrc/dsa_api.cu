@@ -525,6 +525,46 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
   p.total = L.off;
 }
 
+// Tensor-core decode scan of `rows` query rows (q_offsets == nullptr: one row
+// per sequence) followed by the merge of the splits' partial lists into
+// idx / val [rows, k].  K is bf16 (fp8 keys already widened).
+int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void* K, const float* K_scale,
+                  const int64_t* k_offsets, const int32_t* q_offsets, int B, int rows, int64_t total_keys, int H,
+                  int d, int k, int32_t* idx, float* val, uint8_t* ws, cudaStream_t st) {
+  int r;
+  int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
+  float* pval = reinterpret_cast<float*>(ws + p.pval_off);
+  int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
+  int* status = reinterpret_cast<int*>(ws);
+  CUtensorMap tmQ, tmK;
+  if ((r = make_map_bf16(&tmQ, Q, (uint64_t)rows * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  // rows: the whole key array; a tile running past its sequence's end is
+  // masked per key, and rows past the array's end read as zeros
+  if ((r = make_map_bf16(&tmK, K, (uint64_t)total_keys, (uint64_t)d, 128)) != DSA_OK) return r;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 1;
+  a.k_scale = K_scale;
+  a.n_rows = rows;
+  a.n_units = B * p.splits;
+  a.k = k;
+  a.w = w;
+  a.out_idx = pidx;
+  a.out_val = pval;
+  a.out_ld = k;
+  a.out_cnt = pcnt;
+  a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+  a.cand_cap = p.cand_cap;
+  a.status = status;
+  a.k_off = k_offsets;
+  a.q_off = q_offsets;
+  a.splits = p.splits;
+  a.tiles_per_split = p.tiles_per_split;
+  if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
+  return launch_decode_merge(pidx, pval, pcnt, rows, p.splits, k, idx, val,
+                             reinterpret_cast<uint2*>(ws + p.mscr_off), status, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -566,37 +606,13 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
     if ((r = widen_keys(K, total_keys, d, ws, p.widen_off, st)) != DSA_OK) return r;
     K = ws + p.widen_off;
   }
+  if (p.tc)
+    return run_decode_tc(p, Q, w, K, K_scale, k_offsets, q_offsets, B, total_q, total_keys, H, d, k, idx, val, ws, st);
   int* status = reinterpret_cast<int*>(ws);
   int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
   float* pval = reinterpret_cast<float*>(ws + p.pval_off);
   int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
-  if (p.tc) {
-    CUtensorMap tmQ, tmK;
-    if ((r = make_map_bf16(&tmQ, Q, (uint64_t)total_q * H, (uint64_t)d, 64)) != DSA_OK) return r;
-    // rows: the whole key array; a tile running past its sequence's end is
-    // masked per key, and rows past the array's end read as zeros
-    if ((r = make_map_bf16(&tmK, K, (uint64_t)total_keys, (uint64_t)d, 128)) != DSA_OK) return r;
-    TcArgs a;
-    memset(&a, 0, sizeof(a));
-    a.kind = 1;
-    a.k_scale = K_scale;
-    a.n_rows = total_q;
-    a.n_units = B * p.splits;
-    a.k = k;
-    a.w = w;
-    a.out_idx = pidx;
-    a.out_val = pval;
-    a.out_ld = k;
-    a.out_cnt = pcnt;
-    a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
-    a.cand_cap = p.cand_cap;
-    a.status = status;
-    a.k_off = k_offsets;
-    a.q_off = q_offsets;
-    a.splits = p.splits;
-    a.tiles_per_split = p.tiles_per_split;
-    if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
-  } else {
+  {
     SimtArgs a;
     memset(&a, 0, sizeof(a));
     a.kind = 1;
@@ -626,6 +642,135 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
   }
   return launch_decode_merge(pidx, pval, pcnt, total_q, p.splits, k, idx, val,
                              reinterpret_cast<uint2*>(ws + p.mscr_off), status, st);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// PIVOT in decode: each sequence's new queries are one group.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct DecodeGroupPlan {
+  DecodePlan scan;  // the proxies' cache scan: one row per sequence, k = bank
+  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off, ref_cand_off, total;
+  int ref_grid;
+  int64_t ref_cap;
+};
+
+void plan_decode_group(const DeviceInfo& di, int B, int64_t total_keys, int max_keys, int H, int d, int bank,
+                       int q_dtype, int k_dtype, DecodeGroupPlan& gp) {
+  plan_decode(di, B, B, total_keys, max_keys, H, d, bank, q_dtype, k_dtype, gp.scan);
+  Layout L;
+  L.off = gp.scan.total;
+  gp.qbar_off = L.take((size_t)B * H * d * 2);
+  gp.wbar_off = L.take((size_t)B * H * sizeof(float));
+  gp.bidx_off = L.take((size_t)B * bank * sizeof(int32_t));
+  gp.bval_off = L.take((size_t)B * bank * sizeof(float));
+  gp.kg_off = L.take((size_t)B * bank * d * 2);
+  // refine: one unit per sequence (m_b <= 4 queries), candidate lists as for
+  // the prefill refine (whole groups of 4 key tiles)
+  gp.ref_cap = ((int64_t)bank + 511) / 512 * 512;
+  gp.ref_grid = B < di.sms ? B : di.sms;
+  gp.ref_cand_off = L.take((size_t)gp.ref_grid * 4 * gp.ref_cap * sizeof(uint2));
+  gp.total = L.off;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_index_decode_group_workspace_size(int B, int total_q, int max_keys, int H, int d, int k, int bank,
+                                          int q_dtype, int k_dtype, size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (B < 1 || total_q < 1 || max_keys < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  DecodeGroupPlan gp;
+  plan_decode_group(di, B, (int64_t)B * max_keys, max_keys, H, d, bank, q_dtype, k_dtype, gp);
+  *bytes = gp.total;
+  return DSA_OK;
+}
+
+int dsa_index_decode_group(const void* Q, const float* w, const void* K, const float* K_scale,
+                           const int64_t* k_offsets, const int32_t* q_offsets, int B, int total_q, int64_t total_keys,
+                           int max_keys, int H, int d, int k, int bank, int mode, int q_dtype, int k_dtype,
+                           int32_t* idx, float* val, int32_t* bank_idx, float* bank_val, void* proxy_q,
+                           float* proxy_w, void* workspace, size_t workspace_bytes, void* stream) {
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
+  if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1 || max_keys > total_keys) return DSA_ERR_INVALID_ARG;
+  if (bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  if ((proxy_q && !aligned16(proxy_q)) || (proxy_w && !aligned16(proxy_w))) return DSA_ERR_INVALID_ARG;
+  if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (total_keys > ((int64_t)1 << 31) - 256) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  DecodeGroupPlan gp;
+  plan_decode_group(di, B, total_keys, max_keys, H, d, bank, q_dtype, k_dtype, gp);
+  if (workspace_bytes < gp.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* qbar = proxy_q ? proxy_q : ws + gp.qbar_off;
+  float* wbar = proxy_w ? proxy_w : reinterpret_cast<float*>(ws + gp.wbar_off);
+  int32_t* bi = bank_idx ? bank_idx : reinterpret_cast<int32_t*>(ws + gp.bidx_off);
+  float* bv = bank_val ? bank_val : reinterpret_cast<float*>(ws + gp.bval_off);
+  // 0. fp8 keys: exact bf16 copy, the per-key scale goes to the epilogue
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, total_keys, d, ws, gp.scan.widen_off, st)) != DSA_OK) return r;
+    K = ws + gp.scan.widen_off;
+  }
+  // 1. proxies: the mean of each sequence's new queries
+  if ((r = launch_proxy_mean(Q, w, total_q, H, d, 1, q_dtype, qbar, wbar, st, q_offsets, B)) != DSA_OK) return r;
+  // 2. one scan of each cache by its proxy, which sits at the last query's
+  // position N_b - 1: bank = its top-`bank` keys (local indices)
+  if ((r = run_decode_tc(gp.scan, qbar, wbar, K, K_scale, k_offsets, nullptr, B, B, total_keys, H, d, bank, bi, bv,
+                         ws, st)) != DSA_OK)
+    return r;
+  // 3. Reuse ranks the bank and finishes here; Refine ranks it only for the
+  // caller's bank output.  A sequence's queries drop at most 3 bank keys
+  // (m_b <= 4), so Reuse needs the top k + 3.
+  const bool want_bank = bank_idx != nullptr || bank_val != nullptr;
+  if (mode == DSA_GROUP_REUSE || want_bank) {
+    if ((r = launch_bank_rank_reuse(bi, bv, B, bank, 4, total_q, 0, k, idx, val, mode == DSA_GROUP_REUSE, want_bank,
+                                    st, q_offsets, k_offsets)) != DSA_OK)
+      return r;
+  }
+  if (mode == DSA_GROUP_REUSE) return DSA_OK;
+  // 4. Refine: each sequence's queries re-score its bank on tensor cores
+  void* Kg = ws + gp.kg_off;
+  if ((r = launch_bank_gather(K, DSA_DTYPE_BF16, d, bi, B, bank, Kg, st, k_offsets)) != DSA_OK) return r;
+  CUtensorMap tmQ, tmK;
+  if ((r = make_map_bf16(&tmQ, Q, (uint64_t)total_q * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)B * bank, (uint64_t)d, 128)) != DSA_OK) return r;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 2;
+  a.k_scale = K_scale;
+  a.n_rows = total_q;
+  a.mblocks = 1;
+  a.n_units = B;
+  a.k = k;
+  a.w = w;
+  a.out_idx = idx;
+  a.out_val = val;
+  a.out_ld = k;
+  a.cand = reinterpret_cast<uint2*>(ws + gp.ref_cand_off);
+  a.cand_cap = gp.ref_cap;
+  a.status = reinterpret_cast<int*>(ws);
+  a.key_map = bi;
+  a.bank = bank;
+  a.T = total_q;
+  a.k_off = k_offsets;
+  a.q_off = q_offsets;
+  return launch_tc_index(tmQ, tmK, a, gp.ref_grid, st);
 }
 
 }  // extern "C"

@@ -18,10 +18,13 @@ namespace dsa {
 // ---------------------------------------------------------------------------
 // Each thread owns 8 consecutive elements (one 16-byte load per member row
 // for bf16 queries), summed over the members in order in fp32.
+// Group g is rows gG .. min(T, (g+1)G) - 1, or seg[g] .. seg[g+1] - 1 when
+// seg (per-group row offsets, e.g. a decode batch's query offsets) is given.
 __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __restrict__ w, int T, int H, int d,
-                                  int G, int q_dtype, void* __restrict__ qbar, float* __restrict__ wbar) {
+                                  int G, const int32_t* __restrict__ seg, int q_dtype, void* __restrict__ qbar,
+                                  float* __restrict__ wbar) {
   const int g = blockIdx.y;
-  const int r0 = g * G, r1 = min(T, r0 + G);
+  const int r0 = seg ? seg[g] : g * G, r1 = seg ? seg[g + 1] : min(T, r0 + G);
   const float n = (float)(r1 - r0);
   const int64_t hd = (int64_t)H * d;
   const int64_t e0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
@@ -70,35 +73,39 @@ __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __res
 }
 
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
-                      float* wbar, cudaStream_t stream) {
-  const int ng = (T + G - 1) / G;
+                      float* wbar, cudaStream_t stream, const int32_t* seg, int nseg) {
+  const int ng = seg ? nseg : (T + G - 1) / G;
   const int64_t chunks = ((int64_t)H * d + 7) / 8;
   const dim3 grid((unsigned)((chunks + 127) / 128), (unsigned)ng);
-  proxy_mean_kernel<<<grid, 128, 0, stream>>>(Q, w, T, H, d, G, q_dtype, qbar, wbar);
+  proxy_mean_kernel<<<grid, 128, 0, stream>>>(Q, w, T, H, d, G, seg, q_dtype, qbar, wbar);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
-// bank gather: Kg[g*B + j, :] = K[bank[g*B + j], :] (zero rows for -1).
-// Rows are copied 16 bytes per thread.
+// bank gather: Kg[g*B + j, :] = K[base_g + bank[g*B + j], :] (zero rows for
+// -1), base_g = row_off[g] when the bank holds indices local to a sequence
+// (decode), else 0.  Rows are copied 16 bytes per thread.
 // ---------------------------------------------------------------------------
 __global__ void bank_gather_kernel(const uint4* __restrict__ K, int row_vecs, const int32_t* __restrict__ bank,
-                                   int64_t n_rows, uint4* __restrict__ Kg) {
+                                   int64_t n_rows, int bank_size, const int64_t* __restrict__ row_off,
+                                   uint4* __restrict__ Kg) {
   const int64_t total = n_rows * row_vecs;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / row_vecs;
     const int c = (int)(i - r * row_vecs);
     const int32_t src = bank[r];
-    Kg[i] = src >= 0 ? K[(int64_t)src * row_vecs + c] : make_uint4(0u, 0u, 0u, 0u);
+    const int64_t base = row_off ? row_off[r / bank_size] : 0;
+    Kg[i] = src >= 0 ? K[(base + src) * row_vecs + c] : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size, void* Kg,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, const int64_t* row_off) {
   const int elt = (k_dtype == DSA_DTYPE_FP32) ? 4 : (k_dtype == DSA_DTYPE_BF16 ? 2 : 1);
   const int row_vecs = d * elt / 16;
   bank_gather_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), row_vecs, bank,
-                                                   (int64_t)ng * bank_size, static_cast<uint4*>(Kg));
+                                                   (int64_t)ng * bank_size, bank_size, row_off,
+                                                   static_cast<uint4*>(Kg));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -119,7 +126,9 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
                                                                        float* __restrict__ bank_val, int B, int P,
                                                                        int M, int PM, int G, int T, int64_t q_pos0,
                                                                        int k, int32_t* __restrict__ out_idx,
-                                                                       float* __restrict__ out_val, int do_reuse) {
+                                                                       float* __restrict__ out_val, int do_reuse,
+                                                                       const int32_t* __restrict__ q_off,
+                                                                       const int64_t* __restrict__ k_off) {
   extern __shared__ uint64_t keys[];  // [P] the bank; then [PM] its top M when M < B
   __shared__ uint32_t hist[256];
   __shared__ int sh_digit, sh_above, sh_in, sh_cnt;
@@ -238,10 +247,13 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
   }
   if (!do_reuse) return;
   const int NR = M < R ? M : R;  // ranked entries a member may take from
-  // Reuse: warp per member, first k ranked keys with position <= p_t
-  const int r0 = g * G, r1 = min(T, r0 + G);
+  // Reuse: warp per member, first k ranked keys with position <= p_t.  A
+  // decode group (q_off / k_off given) is sequence g: members q_off[g] ..
+  // q_off[g+1] - 1, member j at N_g - m_g + j with local key indices.
+  const int r0 = q_off ? q_off[g] : g * G, r1 = q_off ? q_off[g + 1] : min(T, r0 + G);
+  const int64_t p0 = q_off ? (k_off[g + 1] - k_off[g]) - (r1 - r0) - r0 : q_pos0;
   for (int r = r0 + warp; r < r1; r += nw) {
-    const int64_t p = q_pos0 + r;
+    const int64_t p = p0 + r;
     int32_t* oi = out_idx + (int64_t)r * k;
     float* ov = out_val + (int64_t)r * k;
     int cnt = 0;
@@ -268,7 +280,8 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
 }
 
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T, int64_t q_pos0,
-                           int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all, cudaStream_t stream) {
+                           int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all, cudaStream_t stream,
+                           const int32_t* q_off, const int64_t* k_off) {
   int P = 1;
   while (P < bank_size) P <<= 1;
   if (P > 16384) return DSA_ERR_UNSUPPORTED;
@@ -287,7 +300,7 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
                                                (int)smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   bank_rank_reuse_kernel<<<ng, kRankThreads, smem, stream>>>(bank_idx, bank_val, bank_size, P, M, PM, G, T, q_pos0, k,
-                                                             out_idx, out_val, do_reuse);
+                                                             out_idx, out_val, do_reuse, q_off, k_off);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

@@ -16,7 +16,10 @@ namespace dsa {
 //           each leaves a partial top-k list that decode_merge combines.
 //   kind 2: group refine; unit v = (group v / mblocks, member block v % mblocks);
 //           keys are the group's gathered bank rows, key_map gives their
-//           positions.
+//           positions.  With k_off / q_off set, group g is decode sequence g
+//           (queries q_off[g].., at N_g - m_g + j; key_map local indices).
+//   Decode units with q_off == nullptr have one query row per sequence
+//   (row b: the proxies of a decode group scan).
 struct TcArgs {
   int kind;
   const float* k_scale;     // per-key scale (fp8 keys), or null
@@ -89,15 +92,20 @@ int launch_simt_index(const SimtArgs& a, int grid, cudaStream_t stream);
 size_t simt_smem_bytes(int H, int d);
 
 // Auxiliary kernels.
+// Groups of G consecutive rows, or (seg given) rows seg[g] .. seg[g+1]-1 of
+// nseg groups.
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
-                      float* wbar, cudaStream_t stream);
+                      float* wbar, cudaStream_t stream, const int32_t* seg = nullptr, int nseg = 0);
+// row_off (decode): bank indices are local to sequence g, whose rows start at row_off[g].
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
-                       void* Kg, cudaStream_t stream);
+                       void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr);
 // rank_all: sort and write back the whole bank; otherwise only the top
 // k + G - 1 entries are ranked (enough for Reuse) and the bank is not written.
+// q_off / k_off (decode): group g is sequence g with members q_off[g] ..
+// q_off[g+1]-1 at positions N_g - m_g + j (local key indices).
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,
                            int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all,
-                           cudaStream_t stream);
+                           cudaStream_t stream, const int32_t* q_off = nullptr, const int64_t* k_off = nullptr);
 int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
                         int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
                         cudaStream_t stream);

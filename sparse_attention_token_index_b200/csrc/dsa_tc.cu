@@ -67,8 +67,9 @@ struct UnitInfo {
   int tile0;         // first key tile (local to the key range)
   int ntiles;        // tiles streamed
   int nkeys;         // keys in the range (local index < nkeys is valid)
-  int seq_split;     // decode: sequence; refine: group index
+  int seq_split;     // decode: split; refine: group index
   int partial;       // decode: leaves a partial list
+  int pos0;          // refine: causal position of the unit's first query
 };
 
 __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
@@ -97,7 +98,8 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
   } else if constexpr (kKind == 1) {
     const int b = v / a.splits, sp = v % a.splits;
     const int64_t k0 = a.k_off[b], k1 = a.k_off[b + 1];
-    const int q0 = a.q_off[b], q1 = a.q_off[b + 1];
+    // no query offsets: one query row per sequence (decode proxies)
+    const int q0 = a.q_off ? a.q_off[b] : b, q1 = a.q_off ? a.q_off[b + 1] : b + 1;
     const int nb = (int)(k1 - k0);
     u.row0 = q0;
     u.nq = q1 - q0;
@@ -119,11 +121,28 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     // group refine: members of group g against the group's gathered bank
     const int unit = a.n_units - 1 - v;
     const int g = unit / a.mblocks, mbk = unit % a.mblocks;
-    const int r_end = min(a.T, (g + 1) * a.group);
-    u.row0 = g * a.group + mbk * kQB;
-    u.nq = max(0, min(kQB, r_end - u.row0));
-    const int64_t L = a.pos_base + r_end - 1;
-    const int nbk = (int)min((int64_t)a.bank, L + 1);
+    int nbk;
+    if (a.k_off != nullptr) {
+      // decode groups: group g is sequence g, its queries at N_g - m_g + j,
+      // its bank indices local to the sequence
+      const int q0 = a.q_off[g], q1 = a.q_off[g + 1];
+      const int nb = (int)(a.k_off[g + 1] - a.k_off[g]);
+      u.row0 = q0 + mbk * kQB;
+      u.nq = max(0, min(kQB, q1 - u.row0));
+      u.pos0 = nb - (q1 - q0) + (u.row0 - q0);
+      nbk = min(a.bank, nb);
+      if (q1 - q0 < 1 || q1 - q0 > kQB * a.mblocks || q1 - q0 > nb) {  // 1 <= m_b <= min(4, N_b) is required
+        if (threadIdx.x == 0) report_error(a.status, DSA_ERR_INTERNAL, 4);
+        u.nq = 0;
+      }
+    } else {
+      const int r_end = min(a.T, (g + 1) * a.group);
+      u.row0 = g * a.group + mbk * kQB;
+      u.nq = max(0, min(kQB, r_end - u.row0));
+      u.pos0 = (int)(a.pos_base + u.row0);
+      const int64_t L = a.pos_base + r_end - 1;
+      nbk = (int)min((int64_t)a.bank, L + 1);
+    }
     u.key_row0 = g * a.bank;
     u.tile0 = 0;
     u.ntiles = u.nq > 0 ? (nbk + kTileKeys - 1) / kTileKeys : 0;
@@ -139,7 +158,7 @@ template <int kKind>
 __device__ __forceinline__ int64_t slot_pos(const TcArgs& a, const UnitInfo& u, int slot) {
   if constexpr (kKind == 0) return prefill_pos(a, u.row0 + slot);
   if constexpr (kKind == 1) return (int64_t)u.nkeys - u.nq + slot;
-  return a.pos_base + u.row0 + slot;
+  return (int64_t)u.pos0 + slot;
 }
 
 __device__ __forceinline__ bool group_and(int bar, int nthr, bool ok) {
@@ -363,7 +382,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
-      const float* kscale = a.k_scale;  // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0
+      // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0; decode
+      // groups index the scales of their own sequence
+      const float* kscale =
+          (kKind == 2 && a.k_scale != nullptr && a.k_off != nullptr) ? a.k_scale + a.k_off[u.seq_split] : a.k_scale;
       const int u_key_row0 = u.key_row0;
       if (active) {
         if (ttid == 0) tb_retire(st);
