@@ -49,6 +49,20 @@ def _f64(t):
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
+GROUP_OVERRIDE = None   # --group: group size of the group workloads
+BANK_OVERRIDE = None    # --bank: candidate bank of the group workloads
+
+
+def _row_recall(got_idx, ref_idx):
+    """Per row |got ∩ ref| / |ref| (ignoring -1 padding), on the host."""
+    g, r = got_idx.cpu().numpy(), ref_idx.cpu().numpy()
+    out = np.empty(r.shape[0])
+    for t in range(r.shape[0]):
+        ref = r[t][r[t] >= 0]
+        out[t] = np.intersect1d(g[t][g[t] >= 0], ref).size / max(1, ref.size)
+    return out
+
+
 class Workload:
     """One step = one full call of the indexer on resident inputs.
 
@@ -162,6 +176,8 @@ class Group(Workload):
             self.cfg["T"] = self.cfg["N"] = int(size)
         self.inp = make_dense_inputs(name, device=device, T=self.cfg["T"], N=self.cfg["N"])
         c = self.cfg
+        c["G"] = GROUP_OVERRIDE or c["G"]
+        c["bank"] = BANK_OVERRIDE or c["bank"]
         self.T, self.N, self.k, self.G, self.B = c["T"], c["N"], c["k"], c["G"], c["bank"]
         q0 = self.inp.q_pos0
         self.pairs = self.T * q0 + self.T * (self.T + 1) // 2      # dense-equivalent
@@ -205,6 +221,22 @@ class Group(Workload):
         import sparse_attention_token_index_b200 as dsa
         dsa.dsa_index_group(q, w, k, self.k, self.G, self.B, mode=self.mode, q_pos0=self.inp.q_pos0, K_scale=ks,
                             out=self.out, workspace=self.ws)
+
+    def recall(self, blocks=4, rows=512):
+        """Mean recall of the exact dense top-k (this library's dense kernel)
+        by the group output, over `blocks` row blocks spread over the
+        workload, outside the timed region."""
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        got = []
+        for t0 in np.linspace(0, self.T - rows, blocks).astype(int):
+            t0 = int(t0) // self.G * self.G
+            di, _ = dsa.dsa_index_dense(i.q[t0:t0 + rows], i.w[t0:t0 + rows], i.k, self.k,
+                                        q_pos0=i.q_pos0 + t0, K_scale=i.k_scale)
+            got.append(_row_recall(self.out[0][t0:t0 + rows], di))
+        r = np.concatenate(got)
+        return {"mean": float(r.mean()), "min": float(r.min()), "rows": int(r.size),
+                "note": f"|group top-k ∩ dense top-k| / |dense top-k| over {blocks} blocks of {rows} rows"}
 
     def oracle_sample(self, budget_s=15.0, seed=0):
         from oracle import dsa_oracle as O
@@ -341,6 +373,16 @@ class DecodeGroup(Decode):
         dsa.dsa_index_decode_group(q, w, k, self.k, self.ko, self.qo, self.bank, mode=self.mode,
                                    max_keys=self.cfg["Nb"], total_keys=self.total_keys, out=self.out,
                                    workspace=self.ws)
+
+    def recall(self):
+        """Mean recall of the decode indexer's exact top-k by the group output."""
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        di, _ = dsa.dsa_index_decode(i.q, i.w, i.k, self.k, self.ko, self.qo, max_keys=self.cfg["Nb"],
+                                     total_keys=self.total_keys)
+        r = _row_recall(self.out[0], di)
+        return {"mean": float(r.mean()), "min": float(r.min()), "rows": int(r.size),
+                "note": "|group top-k ∩ decode top-k| / |decode top-k| over every query row"}
 
     def oracle_sample(self, budget_s=15.0, seed=0):
         from oracle import dsa_oracle as O
@@ -532,10 +574,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--T", type=int, default=None,
                     help="other T = N (prefill) or cache length (decode), e.g. for profiling captures")
+    ap.add_argument("--group", type=int, default=None, help="group size G of the group workloads")
+    ap.add_argument("--bank", type=int, default=None, help="candidate bank B of the group workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    global GROUP_OVERRIDE, BANK_OVERRIDE
+    GROUP_OVERRIDE, BANK_OVERRIDE = args.group, args.bank
+    if args.bank:
+        DecodeGroup.bank = args.bank
     if args.impl == "reference":
         run_reference(args)
         return
@@ -625,6 +673,7 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "note": "pinned host inputs copied in, indexer run, idx/val copied out, every step"}
 
+    recall = wl.recall() if hasattr(wl, "recall") else None   # after timing; the last step's output
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         p, r, el = wl.oracle_sample(budget_s=15.0)
@@ -640,6 +689,8 @@ def main():
                 "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
                 "launch_ms": {"min": min(per), "median": statistics.median(per), "max": max(per)}}
         line["config"]["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+        if hasattr(wl, "recall"):
+            line["recall_vs_dense"] = recall
         print(json.dumps(line))
     if dist is not None:
         dist.destroy_process_group()
