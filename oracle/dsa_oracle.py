@@ -47,6 +47,7 @@ __all__ = [
 
 REFINE = 0
 REUSE = 1
+REFINE_LOCAL = 2  # Refine with query-specific additions (see ``group``)
 
 
 # ----------------------------------------------------------------------------
@@ -200,6 +201,12 @@ def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=Non
       3. Refine: member t scores bank keys <= p_t with its own q, w and keeps
          its top-k; Reuse: member t keeps the first k bank entries (in the
          proxy's order) with key <= p_t, valued by the proxy score.
+         REFINE_LOCAL: Refine over the bank plus the query-specific keys the
+         ADIndex page asks refinement to add (section Inference: tokens
+         unique to one query are recovered).  The page does not say which;
+         the reading taken here is the member's own stretch of the group,
+         keys at positions p_first .. p_t (p_first = the group's first
+         member), recent keys that the shared proxy may rank low.
 
     ``qbar``/``wbar`` default to ``proxy(q, w, G)``; a caller may pass the
     proxy exactly as another implementation rounded it.  ``groups`` restricts
@@ -242,10 +249,13 @@ def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=Non
         for r in rows:
             p = q_pos0 + r
             keep = b_idx <= p
-            if mode == REFINE:
+            if mode in (REFINE, REFINE_LOCAL):
                 ms = score_rows(q[r:r + 1], w[r:r + 1], Kd[:_n_visible(p)])[0]
                 res["member_scores"][r] = ms
-                si, sv = select_topk(ms[b_idx[keep]], k, idx=b_idx[keep])
+                cand = b_idx[keep]
+                if mode == REFINE_LOCAL:
+                    cand = np.union1d(cand, np.arange(q_pos0 + r0, p + 1))
+                si, sv = select_topk(ms[cand], k, idx=cand)
             elif mode == REUSE:
                 si, sv = b_idx[keep][:k], b_val[keep][:k]
             else:

@@ -309,11 +309,47 @@ def pin_decode_group_invariants(O):
             assert np.allclose(ru["val"][last], dec["val"][last], rtol=1e-12), b
 
 
+def pin_group_local_hand(O):
+    g = _load("group_local_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["K"], float)
+    for mode, key in ((O.REFINE, "refine"), (O.REFINE_LOCAL, "refine_local"), (O.REUSE, "reuse")):
+        r = O.group(q, w, K, g["k"], g["G"], g["bank"], mode, q_pos0=g["q_pos0"])
+        assert np.array_equal(r["bank_idx"][0], g["bank_idx"]), (key, r["bank_idx"][0])
+        for t in range(2):
+            assert np.array_equal(r["idx"][t], g[key + "_idx"][t]), (key, t, r["idx"][t])
+            assert np.array_equal(r["val"][t], g[key + "_val"][t]), (key, t, r["val"][t])
+
+
+def pin_group_local_invariants(O):
+    q, w, K, _ = _rand_case(12, T=14, N=24, H=3, d=4, q_pos0=10)
+    k, G = 4, 5
+    dn = O.dense(q, w, K, k, q_pos0=10)
+    full = O.group(q, w, K, k, G, 24, O.REFINE_LOCAL, q_pos0=10)
+    rf = O.group(q, w, K, k, G, 6, O.REFINE, q_pos0=10)
+    rl = O.group(q, w, K, k, G, 6, O.REFINE_LOCAL, q_pos0=10)
+    for t in range(14):
+        p = 10 + t
+        # a bank covering the prefix: the dense indexer
+        assert np.array_equal(full["idx"][t], dn["idx"][t]), t
+        n = rl["count"][t]
+        sel = rl["idx"][t][:n]
+        # causal, and never worse than plain Refine: its candidates are a superset
+        assert np.all(sel <= p), t
+        S = rl["member_scores"][t]
+        assert S[sel].min() >= S[rf["idx"][t][:rf["count"][t]]].min() - 1e-15, t
+        # the member's own key is always a candidate
+        cand = np.union1d(rl["bank_idx"][t // G][rl["bank_idx"][t // G] <= p], np.arange(10 + (t // G) * G, p + 1))
+        assert p in cand
+        oi, _ = O.select_topk(S[cand], k, idx=cand)
+        assert np.array_equal(sel, oi), t
+
+
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
         pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
-        pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants]
+        pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants,
+        pin_group_local_hand, pin_group_local_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -457,11 +493,45 @@ def _m_decode_group_scan_first_member(mp):
     mp.setattr(O, "decode_group", dg)
 
 
+def _m_local_window_before_self(mp):
+    # the query-specific keys stop before the member's own position
+    real_union = np.union1d
+
+    def bad(a, b):
+        b = np.asarray(b)
+        return real_union(a, b[:-1]) if b.size and b.dtype.kind == "i" else real_union(a, b)
+    mp.setattr(O.np, "union1d", bad)
+
+
+def _m_local_window_whole_group(mp):
+    # every member adds the whole group's keys, its later members' included
+    real = O.group
+
+    def bad(q, w, K, k, G, bank, mode, q_pos0=0, **kw):
+        if mode != O.REFINE_LOCAL:
+            return real(q, w, K, k, G, bank, mode, q_pos0=q_pos0, **kw)
+        res = real(q, w, K, k, G, bank, O.REFINE, q_pos0=q_pos0, **kw)
+        Kd = O.key_values(K, kw.get("k_scale"))
+        T = q.shape[0]
+        for t in res["idx"]:
+            g = t // G
+            p = q_pos0 + t
+            last = q_pos0 + min(T, (g + 1) * G) - 1
+            b = res["bank_idx"][g]
+            cand = np.union1d(b[b <= p], np.arange(q_pos0 + g * G, last + 1))
+            S = O.score_rows(q[t:t + 1], w[t:t + 1], Kd[:last + 1])[0]
+            si, sv = O.select_topk(S[cand], k, idx=cand)
+            res["idx"][t], res["val"][t] = O._pad(si, sv, k)
+            res["count"][t] = si.shape[0]
+        return res
+    mp.setattr(O, "group", bad)
+
+
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
            _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
-           _m_decode_group_scan_first_member]
+           _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
