@@ -184,22 +184,24 @@ class Group(Workload):
         ng = (self.T + self.G - 1) // self.G
         scan = sum(min(self.T, (g + 1) * self.G) + q0 for g in range(ng))
         refine = 0
-        if mode == 0:
+        if mode in (0, 2):
             for g in range(ng):
                 nb = min(self.B, q0 + min(self.T, (g + 1) * self.G))
-                refine += nb * (min(self.T, (g + 1) * self.G) - g * self.G)
+                nm = min(self.T, (g + 1) * self.G) - g * self.G
+                # Refine with local additions streams G more key slots per group
+                refine += (nb + (self.G if mode == 2 else 0)) * nm
         self.alg_pairs = scan + refine
         self.alg_flops = self.alg_pairs * 2 * c["H"] * c["d"]
         self.rows = self.T
         i = self.inp
         self.host_src = [i.q, i.w, i.k] + ([i.k_scale] if i.k_scale is not None else [])
-        # proxy mean, proxy scan, then Refine: bank gather + re-scoring; Reuse: bank ranking
-        self.launches_per_step = (4 if mode == 0 else 3) + (1 if c["k_dtype"] == "fp8" else 0)
-        self.kernel_launches_per_step = 2 if mode == 0 else 1
+        # proxy mean, proxy scan, then Refine: (local key map +) bank gather + re-scoring; Reuse: bank ranking
+        self.launches_per_step = {0: 4, 1: 3, 2: 5}[mode] + (1 if c["k_dtype"] == "fp8" else 0)
+        self.kernel_launches_per_step = 1 if mode == 1 else 2
 
     def describe(self):
         c = self.cfg
-        m = "Refine" if self.mode == 0 else "Reuse"
+        m = {0: "Refine", 1: "Reuse", 2: "Refine with local additions"}[self.mode]
         kd = "fp8 e4m3 k + scale" if c["k_dtype"] == "fp8" else "bf16 k"
         return {"workload": f"{self.name}: group-shared prefill ({m}) T=N={c['T']} causal, H={c['H']}, d={c['d']}, "
                             f"G={c['G']}, bank={c['bank']}, k={c['k']}, bf16 q, {kd}, fp32 w, seed {c['seed']}",
@@ -409,6 +411,7 @@ WORKLOADS = {
     "decode_bf16_32x128k_group_reuse": lambda dev, size: DecodeGroup(dev, size, 1),
     "group_bf16_128k_refine": lambda dev, size: Group(dev, size, "group_bf16_128k", 0),
     "group_bf16_128k_reuse": lambda dev, size: Group(dev, size, "group_bf16_128k", 1),
+    "group_bf16_128k_refine_local": lambda dev, size: Group(dev, size, "group_bf16_128k", 2),
     "dense_bf16_128k": lambda dev, size: Dense(dev, size or 131072, name="group_bf16_128k"),
     "fp8_256k_dense": lambda dev, size: Dense(dev, size, name="fp8_256k"),
     "fp8_256k_group_refine": lambda dev, size: Group(dev, size, "fp8_256k", 0),

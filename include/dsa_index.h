@@ -64,9 +64,11 @@ extern "C" {
 #define DSA_ERR_DEVICE (-6)      /* current device is not sm_100 */
 #define DSA_ERR_INTERNAL (-7)    /* a device-side consistency check failed */
 
-/* group modes (PIVOT abstract: the Refine and Reuse variants) */
+/* group modes (PIVOT abstract: the Refine and Reuse variants; ADIndex —
+ * Inference: refinement that also adds query-specific tokens) */
 #define DSA_GROUP_REFINE 0
 #define DSA_GROUP_REUSE 1
+#define DSA_GROUP_REFINE_LOCAL 2
 
 /* Human-readable text for a status code (static storage). */
 const char* dsa_status_string(int status);
@@ -111,6 +113,11 @@ int dsa_index_dense(const void* Q, const float* w, const void* K,
  *          its own q, w and keeps its top-k.
  *          DSA_GROUP_REUSE: member t keeps the first k bank keys <= p_t in
  *          the proxy's ranking, valued by the proxy score.
+ *          DSA_GROUP_REFINE_LOCAL: Refine whose candidates also hold the
+ *          member's own stretch of the group, positions p_first .. p_t
+ *          (p_first = the group's first member): the query-specific tokens
+ *          the ADIndex page keeps in refinement, read as the recent keys a
+ *          shared proxy may rank low.  Needs G <= 4096.
  *   Proxy: qbar[g] = mean of the members' q (fp32 mean, rounded to q_dtype),
  *          wbar[g] = mean of the members' w (fp32).  The proxy scans keys
  *          0..L_g, L_g = position of the group's last member.
@@ -175,7 +182,9 @@ int dsa_index_decode(const void* Q, const float* w, const void* K,
  *   mode    DSA_GROUP_REFINE: query j (position N_b - m_b + j) re-scores the
  *           bank keys <= its position with its own q, w and keeps its top-k;
  *           DSA_GROUP_REUSE: it keeps the first k bank keys <= its position
- *           in the proxy's ranking, valued by the proxy score.
+ *           in the proxy's ranking, valued by the proxy score;
+ *           DSA_GROUP_REFINE_LOCAL: Refine whose candidates also hold the
+ *           sequence's new keys N_b - m_b .. its own position.
  *   Arguments as for dsa_index_decode (1 <= m_b <= min(4, N_b), device
  *   offsets, local output indices), plus bank (k <= bank <= 16384), mode and
  *   the optional outputs bank_idx/bank_val [B, bank] (ranked, -1 / -inf

@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     DSA_DTYPE_FP8_E4M3,
     DSA_GROUP_REFINE,
     DSA_GROUP_REUSE,
+    DSA_GROUP_REFINE_LOCAL,
     DsaError,
     lib,
     lib_path,

@@ -12,6 +12,7 @@ DSA_DTYPE_FP32 = 1
 DSA_DTYPE_FP8_E4M3 = 2
 DSA_GROUP_REFINE = 0
 DSA_GROUP_REUSE = 1
+DSA_GROUP_REFINE_LOCAL = 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # DSA_LIB overrides the in-tree library (to compare builds)

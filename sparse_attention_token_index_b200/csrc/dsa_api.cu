@@ -340,7 +340,8 @@ namespace {
 struct GroupPlan {
   size_t widen_off;
   int ng;
-  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off;
+  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off, map_off;
+  int slots;            // refine key slots per group: bank + G (query-specific additions)
   DensePlan scan;       // proxy scan
   int64_t ref_cap;      // refine candidate capacity
   size_t ref_cand_off;
@@ -359,11 +360,14 @@ int plan_group(const DeviceInfo& di, int T, int N, int H, int d, int k, int G, i
   gp.bval_off = L.take((size_t)gp.ng * B * sizeof(float));
   gp.scan = plan_dense(di, gp.ng, N, H, d, q_dtype, k_dtype, L);
   gp.kg_off = 0;
+  gp.map_off = 0;
   gp.ref_cand_off = 0;
-  gp.ref_cap = ((int64_t)B + 511) / 512 * 512;
+  gp.slots = B + G;
+  gp.ref_cap = ((int64_t)gp.slots + 511) / 512 * 512;
   gp.ref_grid = 0;
   if (use_tc(H, d, q_dtype, k_dtype)) {
-    gp.kg_off = L.take((size_t)gp.ng * B * d * 2);  // gathered bank keys, bf16
+    gp.kg_off = L.take((size_t)gp.ng * gp.slots * d * 2);  // gathered bank keys, bf16
+    gp.map_off = L.take((size_t)gp.ng * gp.slots * sizeof(int32_t));
     const int mblocks = (G + 3) / 4;
     const int64_t units = (int64_t)gp.ng * mblocks;
     gp.ref_grid = units < di.sms ? (int)units : di.sms;
@@ -399,9 +403,11 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!idx || !val || !workspace || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
-  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE) return DSA_ERR_INVALID_ARG;
+  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE && mode != DSA_GROUP_REFINE_LOCAL)
+    return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
   if ((proxy_q && !aligned16(proxy_q)) || (proxy_w && !aligned16(proxy_w))) return DSA_ERR_INVALID_ARG;
+  if (mode == DSA_GROUP_REFINE_LOCAL && group > 4096) return DSA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   GroupPlan gp;
@@ -434,12 +440,22 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
       return r;
   }
   if (mode == DSA_GROUP_REUSE) return DSA_OK;
-  // 4. Refine: members re-score their group's bank on tensor cores
+  // 4. Refine: members re-score their group's bank on tensor cores; with
+  // query-specific additions each group's keys also follow its bank
+  const bool local = mode == DSA_GROUP_REFINE_LOCAL;
+  const int S = local ? bank + group : bank;
+  const int32_t* kmap = bi;
+  if (local) {
+    int32_t* map = reinterpret_cast<int32_t*>(ws + gp.map_off);
+    if ((r = launch_local_extend(bi, gp.ng, bank, group, T, q_pos0, nullptr, nullptr, S, map, st)) != DSA_OK)
+      return r;
+    kmap = map;
+  }
   void* Kg = ws + gp.kg_off;
-  if ((r = launch_bank_gather(K, k_dtype, d, bi, gp.ng, bank, Kg, st)) != DSA_OK) return r;
+  if ((r = launch_bank_gather(K, k_dtype, d, kmap, gp.ng, S, Kg, st)) != DSA_OK) return r;
   CUtensorMap tmQ, tmK;
   if ((r = make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
-  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)gp.ng * bank, (uint64_t)d, 128)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)gp.ng * S, (uint64_t)d, 128)) != DSA_OK) return r;
   TcArgs a;
   memset(&a, 0, sizeof(a));
   a.kind = 2;
@@ -456,8 +472,9 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   a.cand = reinterpret_cast<uint2*>(ws + gp.ref_cand_off);
   a.cand_cap = gp.ref_cap;
   a.status = reinterpret_cast<int*>(ws);
-  a.key_map = bi;
-  a.bank = bank;
+  a.key_map = kmap;
+  a.bank = S;
+  a.key_slots = local ? S : 0;
   a.group = group;
   a.T = T;
   return launch_tc_index(tmQ, tmK, a, gp.ref_grid, st);
@@ -653,7 +670,8 @@ namespace {
 
 struct DecodeGroupPlan {
   DecodePlan scan;  // the proxies' cache scan: one row per sequence, k = bank
-  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off, ref_cand_off, total;
+  size_t qbar_off, wbar_off, bidx_off, bval_off, kg_off, map_off, ref_cand_off, total;
+  int slots;  // refine key slots per sequence: bank + 4 (query-specific additions)
   int ref_grid;
   int64_t ref_cap;
 };
@@ -667,10 +685,12 @@ void plan_decode_group(const DeviceInfo& di, int B, int64_t total_keys, int max_
   gp.wbar_off = L.take((size_t)B * H * sizeof(float));
   gp.bidx_off = L.take((size_t)B * bank * sizeof(int32_t));
   gp.bval_off = L.take((size_t)B * bank * sizeof(float));
-  gp.kg_off = L.take((size_t)B * bank * d * 2);
+  gp.slots = bank + 4;
+  gp.kg_off = L.take((size_t)B * gp.slots * d * 2);
+  gp.map_off = L.take((size_t)B * gp.slots * sizeof(int32_t));
   // refine: one unit per sequence (m_b <= 4 queries), candidate lists as for
   // the prefill refine (whole groups of 4 key tiles)
-  gp.ref_cap = ((int64_t)bank + 511) / 512 * 512;
+  gp.ref_cap = ((int64_t)gp.slots + 511) / 512 * 512;
   gp.ref_grid = B < di.sms ? B : di.sms;
   gp.ref_cand_off = L.take((size_t)gp.ref_grid * 4 * gp.ref_cap * sizeof(uint2));
   gp.total = L.off;
@@ -705,7 +725,8 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
   if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1 || max_keys > total_keys) return DSA_ERR_INVALID_ARG;
   if (bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
-  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE) return DSA_ERR_INVALID_ARG;
+  if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE && mode != DSA_GROUP_REFINE_LOCAL)
+    return DSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
   if ((proxy_q && !aligned16(proxy_q)) || (proxy_w && !aligned16(proxy_w))) return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
@@ -744,12 +765,21 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
       return r;
   }
   if (mode == DSA_GROUP_REUSE) return DSA_OK;
-  // 4. Refine: each sequence's queries re-score its bank on tensor cores
+  // 4. Refine: each sequence's queries re-score its bank on tensor cores;
+  // with query-specific additions the sequence's new keys follow its bank
+  const bool local = mode == DSA_GROUP_REFINE_LOCAL;
+  const int S = local ? gp.slots : bank;
+  const int32_t* kmap = bi;
+  if (local) {
+    int32_t* map = reinterpret_cast<int32_t*>(ws + gp.map_off);
+    if ((r = launch_local_extend(bi, B, bank, 4, total_q, 0, q_offsets, k_offsets, S, map, st)) != DSA_OK) return r;
+    kmap = map;
+  }
   void* Kg = ws + gp.kg_off;
-  if ((r = launch_bank_gather(K, DSA_DTYPE_BF16, d, bi, B, bank, Kg, st, k_offsets)) != DSA_OK) return r;
+  if ((r = launch_bank_gather(K, DSA_DTYPE_BF16, d, kmap, B, S, Kg, st, k_offsets)) != DSA_OK) return r;
   CUtensorMap tmQ, tmK;
   if ((r = make_map_bf16(&tmQ, Q, (uint64_t)total_q * H, (uint64_t)d, 64)) != DSA_OK) return r;
-  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)B * bank, (uint64_t)d, 128)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, Kg, (uint64_t)B * S, (uint64_t)d, 128)) != DSA_OK) return r;
   TcArgs a;
   memset(&a, 0, sizeof(a));
   a.kind = 2;
@@ -765,8 +795,9 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   a.cand = reinterpret_cast<uint2*>(ws + gp.ref_cand_off);
   a.cand_cap = gp.ref_cap;
   a.status = reinterpret_cast<int*>(ws);
-  a.key_map = bi;
-  a.bank = bank;
+  a.key_map = kmap;
+  a.bank = S;
+  a.key_slots = local ? S : 0;
   a.T = total_q;
   a.k_off = k_offsets;
   a.q_off = q_offsets;

@@ -110,6 +110,52 @@ int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, i
 }
 
 // ---------------------------------------------------------------------------
+// Refine with query-specific additions: map[g] = the group's bank (B slots),
+// then S - B slots for its own stretch of positions p_first .. p_first + m - 1
+// (m members; -1 beyond), each -1 when the bank holds that key already, so
+// that no key is a candidate twice.  Decode groups (q_off / k_off): sequence
+// g, p_first = N_g - m_g, local indices.
+// ---------------------------------------------------------------------------
+__global__ void local_extend_kernel(const int32_t* __restrict__ bank, int B, int G, int T, int64_t q_pos0,
+                                    const int32_t* __restrict__ q_off, const int64_t* __restrict__ k_off, int S,
+                                    int32_t* __restrict__ map) {
+  extern __shared__ int in_bank[];  // [S - B]
+  const int g = blockIdx.x, tid = threadIdx.x;
+  const int W = S - B;
+  int r0, r1;
+  int64_t p_first;
+  if (q_off) {
+    r0 = q_off[g];
+    r1 = q_off[g + 1];
+    p_first = (k_off[g + 1] - k_off[g]) - (r1 - r0);
+  } else {
+    r0 = g * G;
+    r1 = min(T, r0 + G);
+    p_first = q_pos0 + r0;
+  }
+  const int m = r1 - r0;
+  for (int i = tid; i < W; i += blockDim.x) in_bank[i] = 0;
+  __syncthreads();
+  for (int j = tid; j < B; j += blockDim.x) {
+    const int32_t key = bank[(int64_t)g * B + j];
+    map[(int64_t)g * S + j] = key;
+    const int64_t o = (int64_t)key - p_first;
+    if (key >= 0 && o >= 0 && o < m) in_bank[o] = 1;
+  }
+  __syncthreads();
+  for (int i = tid; i < W; i += blockDim.x)
+    map[(int64_t)g * S + B + i] = (i < m && !in_bank[i]) ? (int32_t)(p_first + i) : -1;
+}
+
+int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
+                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream) {
+  if (S - B < 1 || S - B > 4096) return DSA_ERR_INVALID_ARG;
+  local_extend_kernel<<<ng, 256, (size_t)(S - B) * sizeof(int), stream>>>(bank, B, G, T, q_pos0, q_off, k_off, S,
+                                                                          map);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // bank ranking + Reuse.  One CTA per group; the bank (at most 16384 entries)
 // is held in shared memory as 64-bit keys (order-preserving score bits,
 // inverted key index: larger key = higher rank, unique per entry).

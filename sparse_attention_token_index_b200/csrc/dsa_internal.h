@@ -44,10 +44,11 @@ struct TcArgs {
   int tiles_per_split;
   // refine
   const int32_t* key_map;   // [ng, bank] bank key positions (-1 = empty)
-  int bank;
+  int bank;        // key slots per group in the gathered bank (its row stride)
   int group;
   int mblocks;
   int T;
+  int key_slots;   // nonzero: every slot is streamed, key_map alone marks the valid ones
 };
 
 // Event pair for timing one scoring-kernel launch (dsa_timer.cu); both null
@@ -101,6 +102,9 @@ int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, i
                        void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr);
 // rank_all: sort and write back the whole bank; otherwise only the top
 // k + G - 1 entries are ranked (enough for Reuse) and the bank is not written.
+// Refine with query-specific additions: map [ng, S] = bank (B) + own stretch (S - B).
+int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
+                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream);
 // q_off / k_off (decode): group g is sequence g with members q_off[g] ..
 // q_off[g+1]-1 at positions N_g - m_g + j (local key indices).
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,

@@ -143,6 +143,7 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
       const int64_t L = a.pos_base + r_end - 1;
       nbk = (int)min((int64_t)a.bank, L + 1);
     }
+    if (a.key_slots) nbk = a.key_slots;  // query-specific additions follow the bank
     u.key_row0 = g * a.bank;
     u.tile0 = 0;
     u.ntiles = u.nq > 0 ? (nbk + kTileKeys - 1) / kTileKeys : 0;

@@ -59,15 +59,17 @@ def _check(inp, k, bank, mode, what, seqs=None):
         for j in range(mb):
             r, p = r0 + j, nb - mb + j
             cand = bank_keys[bank_keys <= p]
-            if mode == dsa.DSA_GROUP_REFINE:
+            if mode in (dsa.DSA_GROUP_REFINE, dsa.DSA_GROUP_REFINE_LOCAL):
                 S = O.score_rows(q[r:r + 1], w[r:r + 1], Kd[k0:k0 + p + 1])[0]
-                check_row(gi[r], gv[r], S[cand], k, what=f"{what} refine b={b} j={j}", idx_map=cand)
+                if mode == dsa.DSA_GROUP_REFINE_LOCAL:
+                    cand = np.union1d(cand, np.arange(nb - mb, p + 1))   # the sequence's new keys up to p
+                check_row(gi[r], gv[r], S[cand], k, what=f"{what} refine(mode {mode}) b={b} j={j}", idx_map=cand)
             else:
                 check_row(gi[r], gv[r], ps[cand], k, what=f"{what} reuse b={b} j={j}", idx_map=cand)
     return idx, val
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["refine", "reuse", "refine_local"])
 def test_decode_group_mixed(mode):
     # mixed cache lengths (ragged tiles, one shorter than the bank) and 1..4 queries per sequence
     inp = make_decode_inputs("decode_bf16_32x128k", device=DEV, lengths=[300, 700, 1500, 129, 2050, 90],
@@ -75,7 +77,7 @@ def test_decode_group_mixed(mode):
     _check(inp, 32, 128, mode, "mixed")
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["refine", "reuse", "refine_local"])
 def test_decode_group_fp8(mode):
     inp = make_decode_inputs("decode_bf16_32x128k", device=DEV, lengths=[640, 1100, 257], m=[2, 3, 1], seed=32,
                              k_dtype="fp8")

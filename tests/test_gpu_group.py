@@ -56,9 +56,12 @@ def _check_group(inp, k, G, B, mode, what):
         for t in range(g * G, min(T, (g + 1) * G)):
             p = inp.q_pos0 + t
             cand = bank[bank <= p]
-            if mode == dsa.DSA_GROUP_REFINE:
+            if mode in (dsa.DSA_GROUP_REFINE, dsa.DSA_GROUP_REFINE_LOCAL):
                 S = O.score_rows(q[t:t + 1], w[t:t + 1], K[:p + 1])[0]
-                check_row(gi[t], gv[t], S[cand], k, what=f"{what} refine t={t}", idx_map=cand)
+                if mode == dsa.DSA_GROUP_REFINE_LOCAL:
+                    # plus the member's own stretch of the group
+                    cand = np.union1d(cand, np.arange(inp.q_pos0 + g * G, p + 1))
+                check_row(gi[t], gv[t], S[cand], k, what=f"{what} refine(mode {mode}) t={t}", idx_map=cand)
             else:
                 # Reuse: the first k bank keys it may see, in the proxy's ranking,
                 # valued by the proxy score
@@ -66,13 +69,13 @@ def _check_group(inp, k, G, B, mode, what):
     return idx, val
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["refine", "reuse", "refine_local"])
 def test_group_small(mode):
     inp = make_dense_inputs("group_bf16_128k", device=DEV, T=640, N=640, seed=21)
     _check_group(inp, 64, 64, 256, mode, "G64 B256")
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["refine", "reuse", "refine_local"])
 def test_group_ragged(mode):
     # group size not a multiple of the 4-query unit, partial last group, offset queries
     inp = make_dense_inputs("group_bf16_128k", device=DEV, T=100, N=700, seed=22)
@@ -109,7 +112,7 @@ def _same_rows(a_idx, a_val, b_idx, b_val):
     assert torch.equal(torch.gather(a_val, 1, ap), torch.gather(b_val, 1, bp))
 
 
-@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+@pytest.mark.parametrize("mode", [0, 1, 2], ids=["refine", "reuse", "refine_local"])
 @pytest.mark.parametrize("shape", [(640, 640, 64, 256, 64), (100, 700, 6, 48, 16), (300, 300, 64, 2048, 100)],
                          ids=["G64", "G6", "bank-ge-prefix"])
 def test_group_without_bank_output(mode, shape):
@@ -175,3 +178,23 @@ def test_group_fp8_keys(mode):
             cand = bank[bank <= p]
             S = (O.score_rows(q[t:t + 1], w[t:t + 1], Kd[:p + 1])[0] if mode == 0 else ps)
             check_row(gi[t], gv[t], S[cand], 32, what=f"fp8 member t={t}", idx_map=cand)
+
+
+def test_refine_local_full_size_sampled():
+    # the 128K group workload with query-specific additions, sampled groups
+    inp = make_dense_inputs("group_bf16_128k", device=DEV)
+    G, B, k = 64, 8192, 2048
+    T = inp.q.shape[0]
+    idx, val, bidx, bval = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=dsa.DSA_GROUP_REFINE_LOCAL,
+                                               q_pos0=inp.q_pos0, return_bank=True, check=True)
+    K = _f64(inp.k)
+    bi, gi, gv = bidx.cpu().numpy(), idx.cpu().numpy(), val.cpu().numpy()
+    for g in [0, 777, T // G - 1]:
+        bank = bi[g][bi[g] >= 0].astype(np.int64)
+        for t in (g * G, g * G + 40, min(T, (g + 1) * G) - 1):
+            p = inp.q_pos0 + t
+            cand = np.union1d(bank[bank <= p], np.arange(inp.q_pos0 + g * G, p + 1))
+            q = inp.q[t:t + 1].double().cpu().numpy()
+            w = inp.w[t:t + 1].double().cpu().numpy()
+            S = O.score_rows(q, w, K[:p + 1])[0]
+            check_row(gi[t], gv[t], S[cand], k, what=f"refine_local t={t}", idx_map=cand)
