@@ -490,7 +490,7 @@ struct DecodePlan {
   int grid;
   int64_t cand_cap;
   int splits, tiles_per_split;
-  size_t cand_off, pidx_off, pval_off, pcnt_off, mscr_off, total;
+  size_t cand_off, ppair_off, pcnt_off, total;
 };
 
 void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, int max_keys, int H, int d, int k,
@@ -535,10 +535,8 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
     p.cand_off = L.take((size_t)p.grid * 2 * p.cand_cap * sizeof(uint2));
   }
   const size_t parts = (size_t)total_q * p.splits;
-  p.pidx_off = L.take(parts * k * sizeof(int32_t));
-  p.pval_off = L.take(parts * k * sizeof(float));
+  p.ppair_off = L.take(parts * k * sizeof(uint2));
   p.pcnt_off = L.take(parts * sizeof(int));
-  p.mscr_off = L.take(parts * k * sizeof(uint2));
   p.total = L.off;
 }
 
@@ -549,8 +547,7 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
                   const int64_t* k_offsets, const int32_t* q_offsets, int B, int rows, int64_t total_keys, int H,
                   int d, int k, int32_t* idx, float* val, uint8_t* ws, cudaStream_t st) {
   int r;
-  int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
-  float* pval = reinterpret_cast<float*>(ws + p.pval_off);
+  uint2* ppair = reinterpret_cast<uint2*>(ws + p.ppair_off);
   int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
   int* status = reinterpret_cast<int*>(ws);
   CUtensorMap tmQ, tmK;
@@ -566,8 +563,7 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
   a.n_units = B * p.splits;
   a.k = k;
   a.w = w;
-  a.out_idx = pidx;
-  a.out_val = pval;
+  a.out_pair = ppair;
   a.out_ld = k;
   a.out_cnt = pcnt;
   a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
@@ -578,8 +574,7 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
   a.splits = p.splits;
   a.tiles_per_split = p.tiles_per_split;
   if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
-  return launch_decode_merge(pidx, pval, pcnt, rows, p.splits, k, idx, val,
-                             reinterpret_cast<uint2*>(ws + p.mscr_off), status, st);
+  return launch_decode_merge(ppair, pcnt, rows, p.splits, k, idx, val, status, st);
 }
 
 }  // namespace
@@ -626,8 +621,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
   if (p.tc)
     return run_decode_tc(p, Q, w, K, K_scale, k_offsets, q_offsets, B, total_q, total_keys, H, d, k, idx, val, ws, st);
   int* status = reinterpret_cast<int*>(ws);
-  int32_t* pidx = reinterpret_cast<int32_t*>(ws + p.pidx_off);
-  float* pval = reinterpret_cast<float*>(ws + p.pval_off);
+  uint2* ppair = reinterpret_cast<uint2*>(ws + p.ppair_off);
   int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
   {
     SimtArgs a;
@@ -643,8 +637,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
     a.w = w;
     a.K = K;
     a.K_scale = K_scale;
-    a.out_idx = pidx;
-    a.out_val = pval;
+    a.out_pair = ppair;
     a.out_ld = k;
     a.out_cnt = pcnt;
     a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
@@ -657,8 +650,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
     a.keys_per_split = p.tiles_per_split * 128;
     if ((r = launch_simt_index(a, p.grid, st)) != DSA_OK) return r;
   }
-  return launch_decode_merge(pidx, pval, pcnt, total_q, p.splits, k, idx, val,
-                             reinterpret_cast<uint2*>(ws + p.mscr_off), status, st);
+  return launch_decode_merge(ppair, pcnt, total_q, p.splits, k, idx, val, status, st);
 }
 
 }  // extern "C"

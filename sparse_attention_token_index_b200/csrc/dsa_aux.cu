@@ -351,59 +351,37 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
 }
 
 // ---------------------------------------------------------------------------
-// decode merge: per query row, its splits' top-k lists are compacted into one
-// contiguous list while their histogram is built (one pass, batched loads),
-// the exact threshold bin is read off the histogram, and the row is selected.
+// decode merge: per query row, its splits' top-k lists (packed pairs) are one
+// segmented candidate list.  One pass builds their histogram, the exact
+// threshold bin is read off it, and the row is selected straight from the
+// lists (no copy).
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 256;
-constexpr int kMergeStage = 2048;
+constexpr int kMergeThreads = 512;
+constexpr int kMergeStage = 4096;  // <= 8 entries per thread for the stage resolve
 
 struct MergeSmem {
   RowState st;
   uint2 stage[kMergeStage];
-  int base[257];  // prefix sums of the splits' counts
 };
 
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32_t* __restrict__ part_idx,
-                                                                     const float* __restrict__ part_val,
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const uint2* __restrict__ parts,
                                                                      const int* __restrict__ part_cnt, int splits,
                                                                      int k, int32_t* __restrict__ out_idx,
-                                                                     float* __restrict__ out_val,
-                                                                     uint2* __restrict__ scratch, int* status) {
+                                                                     float* __restrict__ out_val, int* status) {
   __shared__ MergeSmem M;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   RowState& st = M.st;
   row_reset(st, tid, kMergeThreads);
-  if (tid == 0) {
-    int acc = 0;
-    for (int s = 0; s < splits; ++s) {
-      M.base[s] = acc;
-      acc += part_cnt[(int64_t)row * splits + s];
-    }
-    M.base[splits] = acc;
-  }
+  CandList cl;
+  cl.base = parts + (int64_t)row * splits * k;
+  cl.stride = k;
+  cl.nseg = splits;
+  cl.cnt = part_cnt + (int64_t)row * splits;
+  cl.l2 = true;  // written by the scoring kernel's other CTAs
   __syncthreads();
-  uint2* cand = scratch + (int64_t)row * splits * k;
-  for (int s = 0; s < splits; ++s) {
-    const int64_t o = ((int64_t)row * splits + s) * k;
-    const int c = M.base[s + 1] - M.base[s], b0 = M.base[s];
-    for (int i0 = 0; i0 < c; i0 += kMergeThreads * 4) {
-      uint2 e[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = i0 + j * kMergeThreads + tid;
-        e[j] = (i < c) ? make_uint2(__float_as_uint(part_val[o + i]), (uint32_t)part_idx[o + i]) : make_uint2(0, 0);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int i = i0 + j * kMergeThreads + tid;
-        if (i < c) {
-          cand[b0 + i] = e[j];
-          atomicAdd(&st.hist[score_bin(__uint_as_float(e[j].x))], 1u);
-        }
-      }
-    }
-  }
+  for_each_cand(cl, tid, kMergeThreads, [&](uint2 e, bool v) {
+    if (v) atomicAdd(&st.hist[score_bin(__uint_as_float(e.x))], 1u);
+  });
   __syncthreads();
   if (tid < 32) {
     const int2 r = hist_scan(st, 0, kBins - 1, k, lane);
@@ -413,16 +391,14 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const int32
     }
   }
   __syncthreads();
-  row_select(st, single_list(cand, &M.base[splits]), k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k),
-             M.stage, kMergeStage, tid, kMergeThreads, 1, status);
+  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k), M.stage, kMergeStage, tid,
+             kMergeThreads, 1, status);
 }
 
-int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
-                        int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
-                        cudaStream_t stream) {
+int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
+                        float* out_val, int* status, cudaStream_t stream) {
   if (splits > 256) return DSA_ERR_UNSUPPORTED;
-  decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(part_idx, part_val, part_cnt, splits, k, out_idx,
-                                                              out_val, scratch, status);
+  decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(parts, part_cnt, splits, k, out_idx, out_val, status);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

@@ -30,6 +30,7 @@ struct TcArgs {
   const float* w;
   int32_t* out_idx;
   float* out_val;
+  uint2* out_pair;   // decode: partial lists as {score bits, index} pairs
   int64_t out_ld;
   int* out_cnt;
   uint2* cand;
@@ -76,6 +77,7 @@ struct SimtArgs {
   int64_t q_pos0;
   int32_t* out_idx;
   float* out_val;
+  uint2* out_pair;   // decode: partial lists as {score bits, index} pairs
   int64_t out_ld;
   int* out_cnt;
   uint2* cand;
@@ -110,9 +112,9 @@ int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,
                            int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all,
                            cudaStream_t stream, const int32_t* q_off = nullptr, const int64_t* k_off = nullptr);
-int launch_decode_merge(const int32_t* part_idx, const float* part_val, const int* part_cnt, int total_q,
-                        int splits, int k, int32_t* out_idx, float* out_val, uint2* scratch, int* status,
-                        cudaStream_t stream);
+// parts [total_q, splits, k] {score bits, index} pairs, part_cnt [total_q, splits]
+int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
+                        float* out_val, int* status, cudaStream_t stream);
 int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
 // Exact e4m3 -> bf16 copy of n bytes (n a multiple of 16, both 16-byte aligned).
 int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream);

@@ -100,8 +100,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_index_kernel(const SimtArgs
       if (lw == 0) row_update(G.st, a.k, lane);
       named_bar(bar, 128);
     }
-    const int cnt = row_select(G.st, single_list(cand, &G.st.cnt), a.k, row_out(a.out_idx + out_row * a.out_ld, a.out_val + out_row * a.out_ld),
-                               G.stage, kSimtStageCap, tid, 128, bar, a.status);
+    const RowOut out = a.kind == 1 ? RowOut{nullptr, nullptr, a.out_pair + out_row * a.out_ld}
+                                   : row_out(a.out_idx + out_row * a.out_ld, a.out_val + out_row * a.out_ld);
+    const int cnt =
+        row_select(G.st, single_list(cand, &G.st.cnt), a.k, out, G.stage, kSimtStageCap, tid, 128, bar, a.status);
     if (a.kind == 1 && tid == 0) a.out_cnt[out_row] = cnt;
     named_bar(bar, 128);
   }

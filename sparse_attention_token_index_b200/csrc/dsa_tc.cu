@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if constexpr (kKind == 1) {
         // decode: this split's local top-k, combined later by decode_merge
         const int64_t o = row * a.splits + u.seq_split;
-        const int cnt = row_select(st, cl, a.k, row_out(a.out_idx + o * a.out_ld, a.out_val + o * a.out_ld),
+        const int cnt = row_select(st, cl, a.k, RowOut{nullptr, nullptr, a.out_pair + o * a.out_ld},
                                    S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
         if (ttid == 0) a.out_cnt[o] = cnt;
       } else {
