@@ -352,3 +352,48 @@ def decode_group(q, w, K, k_offsets, q_offsets, k, bank, mode, k_scale=None, qba
             out_i[r0 + j], out_v[r0 + j], cnt[r0 + j] = r["idx"][j], r["val"][j], r["count"][j]
     res.update(idx=out_i, val=out_v, count=cnt)
     return res
+
+
+def block_reps(K, block=128, k_scale=None):
+    """Mean key of each contiguous block of `block` keys (the last block may
+    be shorter): the block representatives of two-stage selection over
+    contiguous blocks (AttentionIndex page, Why Positional Blocks Lose
+    Recall: blocks ranked by mean-pooled representatives)."""
+    Kd = key_values(K, k_scale)
+    N = Kd.shape[0]
+    nb = (N + block - 1) // block
+    return np.stack([Kd[b * block:min(N, (b + 1) * block)].mean(axis=0) for b in range(nb)])
+
+
+def block_routed(q, w, K, k, n_blocks, q_pos0=0, k_scale=None, block=128, reps=None, rows=None):
+    """Two-stage selection over contiguous blocks, then the native score.
+
+    Query row t at position p: (1) route: score the representatives of the
+    complete blocks before it (blocks 0 .. (p+1)//block - 1, so routing sees
+    no key beyond p) with the indexer formula and keep the best `n_blocks`
+    (ties to the lower block); (2) refine: the candidates are the keys of
+    those blocks plus the query's own partial block (keys (p+1)//block*block
+    .. p), scored with the query's own q, w; keep the top-k.  ``reps`` may
+    replace the float64 means (another implementation's rounding).  Returns
+    idx/val/count per row plus the selected blocks.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Kd = key_values(K, k_scale)
+    R = block_reps(K, block, k_scale) if reps is None else np.asarray(reps, dtype=np.float64)
+    T = q.shape[0]
+    rows = range(T) if rows is None else rows
+    res = {"idx": {}, "val": {}, "count": {}, "blocks": {}}
+    for t in rows:
+        p = q_pos0 + t
+        c = (p + 1) // block
+        bs = score_rows(q[t:t + 1], w[t:t + 1], R[:c])[0] if c > 0 else np.zeros(0)
+        sel, _ = select_topk(bs, n_blocks)
+        cand = np.concatenate([np.arange(b * block, (b + 1) * block) for b in np.sort(sel)] +
+                              [np.arange(c * block, p + 1)]).astype(np.int64)
+        S = score_rows(q[t:t + 1], w[t:t + 1], Kd[cand])[0]
+        si, sv = select_topk(S, k, idx=cand)
+        res["idx"][t], res["val"][t] = _pad(si, sv, k)
+        res["count"][t] = si.shape[0]
+        res["blocks"][t] = sel
+    return res

@@ -344,12 +344,42 @@ def pin_group_local_invariants(O):
         assert np.array_equal(sel, oi), t
 
 
+def pin_block_routed_hand(O):
+    g = _load("block_routed_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["K"], float)
+    r = O.block_routed(q, w, K, g["k"], g["n_blocks"], q_pos0=g["q_pos0"], block=g["block"])
+    assert np.array_equal(r["blocks"][0], g["blocks"]), r["blocks"][0]
+    assert np.array_equal(r["idx"][0], g["idx"]) and np.array_equal(r["val"][0], g["val"]), (r["idx"][0], r["val"][0])
+    d = O.dense(q, w, K, g["k"], q_pos0=g["q_pos0"])
+    assert np.array_equal(d["idx"][0], g["dense_idx"]) and np.array_equal(d["val"][0], g["dense_val"])
+
+
+def pin_block_routed_invariants(O):
+    q, w, K, _ = _rand_case(13, T=10, N=40, H=3, d=4, q_pos0=30)
+    k = 5
+    dn = O.dense(q, w, K, k, q_pos0=30)
+    # every complete block routed: the candidates are the whole prefix
+    allb = O.block_routed(q, w, K, k, 100, q_pos0=30, block=4)
+    # blocks of one key: routing by the native score itself, so the k routed
+    # keys are the dense top-k (the own partial block is then empty)
+    one = O.block_routed(q, w, K, k, k, q_pos0=30, block=1)
+    for t in range(10):
+        assert np.array_equal(allb["idx"][t], dn["idx"][t]), t
+        assert np.array_equal(one["idx"][t], dn["idx"][t]), t
+    # the representative of a block is its mean key
+    R = O.block_reps(K, 4)
+    assert np.allclose(R[3], K[12:16].mean(axis=0)) and R.shape[0] == 10
+    # routing sees complete blocks only: a query at p = 33 routes among blocks 0..7
+    r = O.block_routed(q[3:4], w[3:4], K, k, 2, q_pos0=33, block=4)
+    assert np.all(r["blocks"][0] < 8)
+
+
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
         pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
         pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants,
-        pin_group_local_hand, pin_group_local_invariants]
+        pin_group_local_hand, pin_group_local_invariants, pin_block_routed_hand, pin_block_routed_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -527,11 +557,45 @@ def _m_local_window_whole_group(mp):
     mp.setattr(O, "group", bad)
 
 
+def _m_block_own_block_dropped(mp):
+    # the query's own partial block left out of the candidates
+    real = O.block_routed
+
+    def bad(q, w, K, k, n_blocks, q_pos0=0, k_scale=None, block=128, reps=None, rows=None):
+        Kd = O.key_values(K, k_scale)
+        R = O.block_reps(K, block, k_scale) if reps is None else reps
+        res = {"idx": {}, "val": {}, "count": {}, "blocks": {}}
+        for t in (range(q.shape[0]) if rows is None else rows):
+            p = q_pos0 + t
+            c = (p + 1) // block
+            bs = O.score_rows(q[t:t + 1], w[t:t + 1], R[:c])[0]
+            sel, _ = O.select_topk(bs, n_blocks)
+            cand = np.concatenate([np.arange(b * block, (b + 1) * block) for b in np.sort(sel)]).astype(np.int64)
+            S = O.score_rows(q[t:t + 1], w[t:t + 1], Kd[cand])[0]
+            si, sv = O.select_topk(S, k, idx=cand)
+            res["idx"][t], res["val"][t] = O._pad(si, sv, k)
+            res["count"][t] = si.shape[0]
+            res["blocks"][t] = sel
+        return res
+    mp.setattr(O, "block_routed", bad)
+
+
+def _m_block_partial_blocks_routed(mp):
+    # routing also ranks the block holding the query (its mean includes later keys)
+    real = O.block_routed
+
+    def bad(q, w, K, k, n_blocks, q_pos0=0, k_scale=None, block=128, reps=None, rows=None):
+        return real(q, w, K, k, n_blocks, q_pos0=q_pos0 + block - 1, k_scale=k_scale, block=block, reps=reps,
+                    rows=rows)
+    mp.setattr(O, "block_routed", bad)
+
+
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
            _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
-           _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group]
+           _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group,
+           _m_block_own_block_dropped, _m_block_partial_blocks_routed]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
