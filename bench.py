@@ -166,6 +166,79 @@ class Dense(Workload):
         return self._oracle_loop(budget_s, one)
 
 
+class BlockRouted(Dense):
+    """Two-stage selection over 128-key blocks (comparator): route each query
+    to its best n_blocks complete blocks by their mean key, refine on them."""
+    n_blocks = 64   # an 8K-key candidate budget
+
+    def __init__(self, device, size=None, name="fp8_256k"):
+        super().__init__(device, size, name=name)
+        T, q0, nb = self.T, self.inp.q_pos0, self.n_blocks
+        H, d = self.cfg["H"], self.cfg["d"]
+        # routing scores each complete block before the query; the refine
+        # scores the routed blocks plus the own partial block
+        route = sum((q0 + t + 1) // 128 for t in range(0, T, 64)) * 64
+        refine = sum(min(nb, (q0 + t + 1) // 128) * 128 + (q0 + t + 1) % 128 for t in range(0, T, 64)) * 64
+        self.alg_pairs = route + refine
+        self.alg_flops = self.alg_pairs * 2 * H * d
+        kd = self.cfg["k_dtype"] == "fp8"
+        # (fp8 widening,) block means, routing, refine; routing and refine
+        # both run the scoring kernel
+        self.launches_per_step = 4 if kd else 3
+        self.kernel_launches_per_step = 2
+
+    def describe(self):
+        d = super().describe()
+        d["workload"] = d["workload"].replace("dense prefill", f"block-routed prefill ({self.n_blocks} blocks of 128 "
+                                                               f"keys routed by their mean, then refined)")
+        d["n_blocks"] = self.n_blocks
+        d["metric_pairs"] = "dense-equivalent causal pairs (alg_pairs = routing + refine)"
+        return d
+
+    def setup(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        T, H, d = i.q.shape
+        kd = 2 if self.cfg["k_dtype"] == "fp8" else 0
+        self.ws = torch.zeros(dsa.block_routed_workspace_bytes(T, self.N, H, d, self.k, self.n_blocks, 0, kd),
+                              dtype=torch.uint8, device=i.q.device)
+        self.out = (torch.empty((T, self.k), dtype=torch.int32, device=i.q.device),
+                    torch.empty((T, self.k), dtype=torch.float32, device=i.q.device))
+
+    def call(self, q, w, k, ks=None):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_block_routed(q, w, k, self.k, self.n_blocks, q_pos0=self.inp.q_pos0, K_scale=ks, out=self.out,
+                                   workspace=self.ws)
+
+    def recall(self, blocks=4, rows=512):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        got = []
+        for t0 in np.linspace(0, self.T - rows, blocks).astype(int):
+            t0 = int(t0)
+            di, _ = dsa.dsa_index_dense(i.q[t0:t0 + rows], i.w[t0:t0 + rows], i.k, self.k,
+                                        q_pos0=i.q_pos0 + t0, K_scale=i.k_scale)
+            got.append(_row_recall(self.out[0][t0:t0 + rows], di))
+        r = np.concatenate(got)
+        return {"mean": float(r.mean()), "min": float(r.min()), "rows": int(r.size),
+                "note": f"|routed top-k ∩ dense top-k| / |dense top-k| over {blocks} blocks of {rows} rows"}
+
+    def oracle_sample(self, budget_s=15.0, seed=0):
+        from oracle import dsa_oracle as O
+        i = self.inp
+        K = i.k.cpu().numpy() if self.cfg["k_dtype"] == "fp8" else _f64(i.k)
+        ks = i.k_scale.cpu().numpy() if i.k_scale is not None else None
+        R = O.block_reps(K, 128, ks)
+        rng = np.random.default_rng(seed)
+
+        def one(_):
+            t = int(rng.integers(0, self.T))
+            O.block_routed(_f64(i.q[t:t + 1]), _f64(i.w[t:t + 1]), K, self.k, self.n_blocks, q_pos0=i.q_pos0 + t,
+                           k_scale=ks, reps=R)
+            return i.q_pos0 + t + 1
+        return self._oracle_loop(budget_s, one)
+
+
 class Group(Workload):
     def __init__(self, device, size=None, name="group_bf16_128k", mode=0):
         from synthetic import CONFIGS, make_dense_inputs
@@ -414,6 +487,8 @@ WORKLOADS = {
     "group_bf16_128k_refine_local": lambda dev, size: Group(dev, size, "group_bf16_128k", 2),
     "dense_bf16_128k": lambda dev, size: Dense(dev, size or 131072, name="group_bf16_128k"),
     "fp8_256k_dense": lambda dev, size: Dense(dev, size, name="fp8_256k"),
+    "fp8_256k_block_routed": lambda dev, size: BlockRouted(dev, size, name="fp8_256k"),
+    "group_bf16_128k_block_routed": lambda dev, size: BlockRouted(dev, size, name="group_bf16_128k"),
     "fp8_256k_group_refine": lambda dev, size: Group(dev, size, "fp8_256k", 0),
     "fp8_256k_group_reuse": lambda dev, size: Group(dev, size, "fp8_256k", 1),
 }

@@ -207,6 +207,34 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K,
                            size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Two-stage selection over contiguous key blocks (block routing; the
+ * AttentionIndex page, Why Positional Blocks Lose Recall): a comparator for
+ * the dense and group-shared forms.  Keys form blocks of 128 (the last one
+ * may be shorter); a block's representative is its mean key (fp32 mean of
+ * the keys times their scale, rounded to bf16).  Query t at p_t:
+ *   route   score the representatives of the complete blocks before it
+ *           (blocks 0 .. (p_t+1)/128 - 1: no key beyond p_t reaches routing)
+ *           with the indexer formula and keep the best n_blocks (ties to the
+ *           lower block);
+ *   refine  the candidates are those blocks' keys plus its own partial block
+ *           (keys (p_t+1)/128*128 .. p_t); keep the top-k by the native
+ *           score.
+ *   Arguments as for dsa_index_dense, plus n_blocks (1 .. 65536) and the
+ *   optional outputs block_idx [T, n_blocks] int32 (routed blocks, -1
+ *   padded, in no particular order) and reps [ceil(N/128), d] bf16.
+ *   Tensor-core shape only (bf16 q, bf16 or fp8 k, H = 64, d = 128).
+ * ---------------------------------------------------------------------- */
+int dsa_index_block_routed_workspace_size(int T, int N, int H, int d, int k,
+                                          int n_blocks, int q_dtype,
+                                          int k_dtype, size_t* bytes);
+int dsa_index_block_routed(const void* Q, const float* w, const void* K,
+                           const float* K_scale, int T, int N, int H, int d,
+                           int64_t q_pos0, int k, int n_blocks, int q_dtype,
+                           int k_dtype, int32_t* idx, float* val,
+                           int32_t* block_idx, void* reps, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dense indexer that allocates nothing (the pages have no counterpart: this
  * is an integration aid).  For callers that cannot hand the library a
  * workspace — code running inside a host application that reserved all

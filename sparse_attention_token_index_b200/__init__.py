@@ -23,6 +23,7 @@ from ._binding import (  # noqa: F401
     dsa_index_group,
     dsa_index_decode,
     dsa_index_decode_group,
+    dsa_index_block_routed,
     dsa_debug_scores,
     dsa_index_dense_static,
     dsa_kernel_timer_start,
@@ -32,5 +33,6 @@ from ._binding import (  # noqa: F401
     group_workspace_bytes,
     decode_workspace_bytes,
     decode_group_workspace_bytes,
+    block_routed_workspace_bytes,
     EXPORTED_SYMBOLS,
 )

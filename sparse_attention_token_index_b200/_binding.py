@@ -26,6 +26,7 @@ EXPORTED_SYMBOLS = (
     "dsa_debug_scores", "dsa_index_dense_static",
     "dsa_kernel_timer_start", "dsa_kernel_timer_stop",
     "dsa_index_decode_group_workspace_size", "dsa_index_decode_group",
+    "dsa_index_block_routed_workspace_size", "dsa_index_block_routed",
 )
 
 
@@ -58,6 +59,9 @@ _SIGS = {
                                         _vp]),
     "dsa_kernel_timer_start": (_c_int, [_c_int]),
     "dsa_index_decode_group_workspace_size": (_c_int, [_c_int] * 9 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_block_routed_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_block_routed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                        _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_sz, _vp]),
     "dsa_index_decode_group": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
                                         _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _c_sz, _vp]),
@@ -308,6 +312,44 @@ def dsa_index_decode_group(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: 
         res += [bi, bv]
     if return_proxy:
         res += [pq, pw]
+    return tuple(res)
+
+
+def block_routed_workspace_bytes(T, N, H, d, k, n_blocks, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_block_routed_workspace_size(T, N, H, d, k, n_blocks, q_dtype, k_dtype, ctypes.byref(n)),
+           "dsa_index_block_routed_workspace_size")
+    return int(n.value)
+
+
+def dsa_index_block_routed(Q, w, K, k: int, n_blocks: int, q_pos0: Optional[int] = None, K_scale=None, out=None,
+                           return_blocks: bool = False, return_reps: bool = False, workspace=None, stream=None,
+                           check: bool = False):
+    """Two-stage selection over 128-key blocks (block routing), then the native score.
+
+    Returns (idx, val) and, on request, the routed blocks [T, n_blocks] and
+    the block representatives [ceil(N/128), d] (bf16).
+    """
+    _need_cuda(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    nb = block_routed_workspace_bytes(T, N, H, d, k, n_blocks, qd, kd)
+    ws = _workspace(nb, Q.device, workspace)
+    idx, val = _outputs(T, k, Q.device, out)
+    bi = torch.empty((T, n_blocks), dtype=torch.int32, device=Q.device) if return_blocks else None
+    rp = torch.empty(((N + 127) // 128, d), dtype=torch.bfloat16, device=Q.device) if return_reps else None
+    _check(lib().dsa_index_block_routed(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, k, n_blocks,
+                                        qd, kd, _ptr(idx), _ptr(val), _ptr(bi), _ptr(rp), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "dsa_index_block_routed")
+    if check:
+        dsa_check_status(ws, stream)
+    res = [idx, val]
+    if return_blocks:
+        res.append(bi)
+    if return_reps:
+        res.append(rp)
     return tuple(res)
 
 

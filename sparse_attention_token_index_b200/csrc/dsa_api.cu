@@ -158,7 +158,7 @@ DensePlan plan_dense(const DeviceInfo& di, int T, int N, int H, int d, int q_dty
 int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, const float* w, const void* K,
                    const float* K_scale, int n_rows, int N, int H, int d, int64_t pos_base, int64_t pos_mul,
                    int64_t pos_add, int64_t pos_clamp, int k, int q_dtype, int k_dtype, int32_t* idx, float* val,
-                   uint8_t* ws, float* dbg, int64_t dbg_ld, cudaStream_t st) {
+                   uint8_t* ws, float* dbg, int64_t dbg_ld, cudaStream_t st, int64_t pos_div = 0) {
   int* status = reinterpret_cast<int*>(ws);
   uint2* cand = reinterpret_cast<uint2*>(ws + p.cand_off);
   if (p.tc) {
@@ -178,6 +178,7 @@ int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, cons
     a.pos_mul = pos_mul;
     a.pos_add = pos_add;
     a.pos_clamp = pos_clamp;
+    a.pos_div = pos_div;
     a.w = w;
     a.out_idx = idx;
     a.out_val = val;
@@ -794,6 +795,110 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   a.k_off = k_offsets;
   a.q_off = q_offsets;
   return launch_tc_index(tmQ, tmK, a, gp.ref_grid, st);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Two-stage selection over contiguous blocks (block routing) with the native
+// score on the routed keys.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct RoutedPlan {
+  size_t widen_off, reps_off, bidx_off, bval_off, ref_cand_off, total;
+  int64_t nblocks;
+  DensePlan route;  // the queries against the block representatives
+  int ref_grid;
+  int64_t ref_cap;
+};
+
+void plan_routed(const DeviceInfo& di, int T, int N, int H, int d, int n_blocks, int q_dtype, int k_dtype,
+                 RoutedPlan& p) {
+  Layout L;
+  p.widen_off = take_widen(L, N, H, d, q_dtype, k_dtype);
+  p.nblocks = ((int64_t)N + 127) / 128;
+  p.reps_off = L.take((size_t)p.nblocks * d * 2);
+  p.bidx_off = L.take((size_t)T * n_blocks * sizeof(int32_t));
+  p.bval_off = L.take((size_t)T * n_blocks * sizeof(float));
+  p.route = plan_dense(di, T, (int)p.nblocks, H, d, q_dtype, DSA_DTYPE_BF16, L);
+  // refine: one query per unit over at most n_blocks + 1 tiles (whole groups of 4)
+  p.ref_cap = ((int64_t)n_blocks + 1 + 3) / 4 * 4 * 128;
+  p.ref_grid = T < di.sms ? T : di.sms;
+  p.ref_cand_off = L.take((size_t)p.ref_grid * 4 * p.ref_cap * sizeof(uint2));
+  p.total = L.off;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_index_block_routed_workspace_size(int T, int N, int H, int d, int k, int n_blocks, int q_dtype,
+                                          int k_dtype, size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (T < 1 || N < 1 || n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  RoutedPlan p;
+  plan_routed(di, T, N, H, d, n_blocks, q_dtype, k_dtype, p);
+  *bytes = p.total;
+  return DSA_OK;
+}
+
+int dsa_index_block_routed(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H,
+                           int d, int64_t q_pos0, int k, int n_blocks, int q_dtype, int k_dtype, int32_t* idx,
+                           float* val, int32_t* block_idx, void* reps, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!idx || !val || !workspace || n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (reps && !aligned16(reps)) return DSA_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  RoutedPlan p;
+  plan_routed(di, T, N, H, d, n_blocks, q_dtype, k_dtype, p);
+  if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, N, d, ws, p.widen_off, st)) != DSA_OK) return r;
+    K = ws + p.widen_off;
+  }
+  // 1. block representatives (fp8 keys: the mean of the scaled keys)
+  void* R = reps ? reps : ws + p.reps_off;
+  if ((r = launch_block_mean(K, K_scale, N, d, R, st)) != DSA_OK) return r;
+  // 2. routing: each query's best n_blocks complete blocks before it
+  int32_t* bi = block_idx ? block_idx : reinterpret_cast<int32_t*>(ws + p.bidx_off);
+  float* bv = reinterpret_cast<float*>(ws + p.bval_off);
+  if ((r = run_dense_rows(di, p.route, Q, w, R, nullptr, T, (int)p.nblocks, H, d, q_pos0, 1, 0, (int64_t)T, n_blocks,
+                          q_dtype, DSA_DTYPE_BF16, bi, bv, ws, nullptr, 0, st, 128)) != DSA_OK)
+    return r;
+  // 3. refine: the native score over the routed blocks and the own partial block
+  CUtensorMap tmQ, tmK;
+  if ((r = make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, K, (uint64_t)N, (uint64_t)d, 128)) != DSA_OK) return r;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 3;
+  a.k_scale = K_scale;
+  a.n_rows = T;
+  a.n_units = T;
+  a.k = k;
+  a.pos_base = q_pos0;
+  a.w = w;
+  a.out_idx = idx;
+  a.out_val = val;
+  a.out_ld = k;
+  a.cand = reinterpret_cast<uint2*>(ws + p.ref_cand_off);
+  a.cand_cap = p.ref_cap;
+  a.status = reinterpret_cast<int*>(ws);
+  a.route_blocks = bi;
+  a.route_n = n_blocks;
+  return launch_tc_index(tmQ, tmK, a, p.ref_grid, st);
 }
 
 }  // extern "C"

@@ -82,6 +82,32 @@ int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G,
 }
 
 // ---------------------------------------------------------------------------
+// block representatives: R[b] = mean of keys b*128 .. min(N, b*128+128) - 1
+// (keys times their per-key scale when given), fp32 sums in key order,
+// rounded to bf16.  One CTA per block, thread j owns element j.
+// ---------------------------------------------------------------------------
+__global__ void block_mean_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ K_scale, int64_t N,
+                                  int d, __nv_bfloat16* __restrict__ R) {
+  const int64_t b = blockIdx.x;
+  const int64_t r0 = b * 128, r1 = min(N, r0 + 128);
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float s = 0.f;
+    for (int64_t r = r0; r < r1; ++r) {
+      const float x = __bfloat162float(K[r * d + j]);
+      s += K_scale ? x * K_scale[r] : x;
+    }
+    R[b * d + j] = __float2bfloat16_rn(s / (float)(r1 - r0));
+  }
+}
+
+int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, void* R, cudaStream_t stream) {
+  const int64_t nb = (N + 127) / 128;
+  block_mean_kernel<<<(unsigned)nb, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(K), K_scale, N, d,
+                                                      static_cast<__nv_bfloat16*>(R));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // bank gather: Kg[g*B + j, :] = K[base_g + bank[g*B + j], :] (zero rows for
 // -1), base_g = row_off[g] when the bank holds indices local to a sequence
 // (decode), else 0.  Rows are copied 16 bytes per thread.

@@ -14,6 +14,7 @@ namespace dsa {
 //           pos_add G-1 so the proxy scans its group's last member's prefix).
 //   kind 1: decode segments; unit v = (sequence v / splits, split v % splits);
 //           each leaves a partial top-k list that decode_merge combines.
+//   kind 3: routed refine; unit v = query row v over its routed key blocks.
 //   kind 2: group refine; unit v = (group v / mblocks, member block v % mblocks);
 //           keys are the group's gathered bank rows, key_map gives their
 //           positions.  With k_off / q_off set, group g is decode sequence g
@@ -50,6 +51,14 @@ struct TcArgs {
   int mblocks;
   int T;
   int key_slots;   // nonzero: every slot is streamed, key_map alone marks the valid ones
+  // kind 0 rows see (pos_base + r + 1) / pos_div - 1 when pos_div > 0 (the
+  // complete 128-key blocks before a query, for block routing)
+  int64_t pos_div;
+  // kind 3 (routed refine): one query row per unit; it streams the blocks
+  // route_blocks[row, 0 .. min(route_n, complete blocks)) then its own
+  // partial block, keys <= its position
+  const int32_t* route_blocks;
+  int route_n;
 };
 
 // Event pair for timing one scoring-kernel launch (dsa_timer.cu); both null
@@ -116,6 +125,8 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
                         float* out_val, int* status, cudaStream_t stream);
 int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
+// Block representatives of bf16 keys (fp8 keys widened; K_scale applied when given).
+int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, void* R, cudaStream_t stream);
 // Exact e4m3 -> bf16 copy of n bytes (n a multiple of 16, both 16-byte aligned).
 int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream);
 

@@ -69,10 +69,18 @@ struct UnitInfo {
   int nkeys;         // keys in the range (local index < nkeys is valid)
   int seq_split;     // decode: split; refine: group index
   int partial;       // decode: leaves a partial list
-  int pos0;          // refine: causal position of the unit's first query
+  int pos0;          // refine / routed: causal position of the unit's first query
+  int rsel;          // routed: routed blocks streamed first
+  int rown;          // routed: the query's own partial block, streamed last
 };
 
+// Key block of iteration j of a routed unit: its routed blocks, then its own.
+__device__ __forceinline__ int routed_block(const TcArgs& a, const UnitInfo& u, int j) {
+  return j < u.rsel ? a.route_blocks[(int64_t)u.row0 * a.route_n + j] : u.rown;
+}
+
 __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
+  if (a.pos_div > 0) return (a.pos_base + r + 1) / a.pos_div - 1;
   int64_t v = (int64_t)r * a.pos_mul + a.pos_add;
   if (v > a.pos_clamp) v = a.pos_clamp;
   return a.pos_base + v;
@@ -91,10 +99,26 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     const int64_t maxpos = prefill_pos(a, u.row0 + u.nq - 1);
     u.key_row0 = 0;
     u.tile0 = 0;
-    u.ntiles = (int)(maxpos / kTileKeys) + 1;
+    u.ntiles = maxpos >= 0 ? (int)(maxpos / kTileKeys) + 1 : 0;
     u.nkeys = (int)(maxpos + 1);
     u.seq_split = -1;
     u.partial = 0;
+  } else if constexpr (kKind == 3) {
+    // routed refine: one query row over its routed blocks (longest first)
+    const int t = a.n_units - 1 - v;
+    const int64_t p = a.pos_base + t;
+    const int own = (int)((p + 1) / kTileKeys);  // complete blocks before the query
+    u.row0 = t;
+    u.nq = 1;
+    u.rsel = min(a.route_n, own);
+    u.rown = own;
+    u.key_row0 = 0;
+    u.tile0 = 0;
+    u.ntiles = u.rsel + (((int64_t)own * kTileKeys <= p) ? 1 : 0);  // own block non-empty
+    u.nkeys = (int)(p + 1);
+    u.seq_split = -1;
+    u.partial = 0;
+    u.pos0 = (int)p;
   } else if constexpr (kKind == 1) {
     const int b = v / a.splits, sp = v % a.splits;
     const int64_t k0 = a.k_off[b], k1 = a.k_off[b + 1];
@@ -159,7 +183,7 @@ template <int kKind>
 __device__ __forceinline__ int64_t slot_pos(const TcArgs& a, const UnitInfo& u, int slot) {
   if constexpr (kKind == 0) return prefill_pos(a, u.row0 + slot);
   if constexpr (kKind == 1) return (int64_t)u.nkeys - u.nq + slot;
-  return (int64_t)u.pos0 + slot;
+  return (int64_t)u.pos0 + slot;  // kinds 2 and 3
 }
 
 __device__ __forceinline__ bool group_and(int bar, int nthr, bool ok) {
@@ -275,7 +299,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = 0; j < u.ntiles; ++j) {
           if (!(ok = mbar_wait(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11))) break;
           mbar_arrive_expect_tx(&S.k_full[s], (uint32_t)kKStageBytes);
-          const int row = u.key_row0 + (u.tile0 + j) * kTileKeys;
+          const int row = (kKind == 3) ? routed_block(a, u, j) * kTileKeys : u.key_row0 + (u.tile0 + j) * kTileKeys;
           for (int c = 0; c < 2; ++c)
             tma_load_2d(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row);
           armed |= 1u << s;
@@ -379,7 +403,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[q]);
       // per-unit scalars (kept in registers through the tile loop)
       const int64_t row = (int64_t)u.row0 + q;
-      const int pos = active ? (int)slot_pos<kKind>(a, u, q) : -1;  // key positions fit in int (N <= INT_MAX)
+      // keys 0 .. pos are visible (pos = -1: none); positions fit in int (N <= INT_MAX)
+      const int pos = active ? (int)slot_pos<kKind>(a, u, q) : -1;
+      const unsigned n_vis = (unsigned)(pos + 1);
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
       const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
@@ -425,7 +451,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         eph ^= 1u << buf;
         buf ^= 1;
         if (mine) {
-          const int key = key0 + jt * kTileKeys;  // local key index
+          const int key = key0 + (kKind == 3 ? routed_block(a, u, jt) : jt) * kTileKeys;  // local key index
           const bool in_range = key < nkeys;
           int kpos = key;
           if (kmap != nullptr) kpos = in_range ? kmap[key] : -1;
@@ -433,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
           if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
-          const bool valid = in_range && (unsigned)kpos <= (unsigned)pos;
+          const bool valid = in_range && (unsigned)kpos < n_vis;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
           row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
         }
@@ -491,7 +517,7 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream) {
-  if (a.kind < 0 || a.kind > 2 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
+  if (a.kind < 0 || a.kind > 3 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
   const TimerSlot ts = timer_acquire();
   if (ts.start) cudaEventRecord(ts.start, stream);
   int r;
@@ -501,8 +527,10 @@ int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs
     r = launch_tc<false, 0>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 1)
     r = launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
-  else
+  else if (a.kind == 2)
     r = launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
+  else
+    r = launch_tc<false, 3>(tmQ, tmK, a, grid, stream);
   if (ts.end) cudaEventRecord(ts.end, stream);
   return r;
 }
