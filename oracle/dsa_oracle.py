@@ -397,3 +397,53 @@ def block_routed(q, w, K, k, n_blocks, q_pos0=0, k_scale=None, block=128, reps=N
         res["count"][t] = si.shape[0]
         res["blocks"][t] = sel
     return res
+
+
+def kmeans(K, C, iters, k_scale=None):
+    """Plain Lloyd's k-means over the keys (Euclidean), the index build of
+    inverted-file routing (AttentionIndex page: keys grouped by similarity
+    rather than position; its learned encoder and causal index versions are
+    not part of this plain form).  Centroid i starts at key floor(i N / C);
+    each iteration assigns every key to its nearest centroid (ties to the
+    lower centroid), then moves each centroid to the mean of its members (a
+    centroid without members stays).  Returns (assign [N] int64, centroids
+    [C, d] float64)."""
+    Kd = key_values(K, k_scale)
+    N = Kd.shape[0]
+    cen = Kd[(np.arange(C) * N) // C].copy()
+    assign = np.zeros(N, dtype=np.int64)
+    for _ in range(iters):
+        d2 = (Kd * Kd).sum(1)[:, None] - 2.0 * Kd @ cen.T + (cen * cen).sum(1)[None, :]
+        assign = np.argmin(d2, axis=1)  # first minimum = lower centroid on ties
+        for c in range(C):
+            m = assign == c
+            if m.any():
+                cen[c] = Kd[m].mean(axis=0)
+    return assign, cen
+
+
+def ivf_routed(q, w, K, k, n_probe, assign, centroids, q_pos0=0, k_scale=None, rows=None):
+    """Inverted-file routing, then the native score (AttentionIndex page:
+    route each query over the clusters, refine the candidates with the
+    native indexer score).  Query row t at position p: score the centroids
+    with the indexer formula, keep the best n_probe clusters (ties to the
+    lower cluster); the candidates are their members with key <= p (the
+    clusters span the whole key set: causality by masking, not versions);
+    keep the top-k by the native score."""
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    Kd = key_values(K, k_scale)
+    assign = np.asarray(assign, dtype=np.int64)
+    cen = np.asarray(centroids, dtype=np.float64)
+    res = {"idx": {}, "val": {}, "count": {}, "clusters": {}}
+    for t in (range(q.shape[0]) if rows is None else rows):
+        p = q_pos0 + t
+        cs = score_rows(q[t:t + 1], w[t:t + 1], cen)[0]
+        sel, _ = select_topk(cs, n_probe)
+        cand = np.nonzero(np.isin(assign[:p + 1], sel))[0].astype(np.int64)
+        S = score_rows(q[t:t + 1], w[t:t + 1], Kd[cand])[0]
+        si, sv = select_topk(S, k, idx=cand)
+        res["idx"][t], res["val"][t] = _pad(si, sv, k)
+        res["count"][t] = si.shape[0]
+        res["clusters"][t] = sel
+    return res

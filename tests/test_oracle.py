@@ -374,12 +374,49 @@ def pin_block_routed_invariants(O):
     assert np.all(r["blocks"][0] < 8)
 
 
+def pin_ivf_hand(O):
+    g = _load("ivf_hand.json")
+    K = np.array(g["K"], float)
+    a, c = O.kmeans(K, g["C"], g["iters"])
+    assert np.array_equal(a, g["assign"]), a
+    assert np.allclose(c, g["centroids"]), c
+    q, w = np.array(g["q"], float), np.array(g["w"], float)
+    for pos, key in ((5, "at5"), (3, "at3")):
+        r = O.ivf_routed(q, w, K, g["k"], g["n_probe"], a, c, q_pos0=pos)
+        assert np.array_equal(r["idx"][0], g[key + "_idx"]), (pos, r["idx"][0])
+        assert np.allclose(r["val"][0], g[key + "_val"]), (pos, r["val"][0])
+
+
+def pin_ivf_invariants(O):
+    rng = np.random.default_rng(14)
+    K = np.concatenate([rng.standard_normal((15, 4)) * 0.1 + m for m in (rng.standard_normal((3, 4)) * 3)])
+    K = K[rng.permutation(45)]
+    a, c = O.kmeans(K, 3, 5)
+    # a fixed point: every key sits with a nearest centroid, every centroid is its members' mean
+    d2 = ((K[:, None, :] - c[None, :, :]) ** 2).sum(-1)
+    assert np.all(d2[np.arange(45), a] <= d2.min(1) + 1e-12)
+    for j in range(3):
+        assert np.allclose(c[j], K[a == j].mean(0))
+    q, w, _, _ = _rand_case(15, T=5, N=45, H=2, d=4, q_pos0=40)
+    dn = O.dense(q, w, K, 4, q_pos0=40)
+    # probing every cluster: the dense indexer
+    r = O.ivf_routed(q, w, K, 4, 3, a, c, q_pos0=40)
+    for t in range(5):
+        assert np.array_equal(r["idx"][t], dn["idx"][t]), t
+    # candidates stay causal and inside the routed clusters
+    r1 = O.ivf_routed(q, w, K, 4, 1, a, c, q_pos0=40)
+    for t in range(5):
+        sel = r1["idx"][t][:r1["count"][t]]
+        assert np.all(sel <= 40 + t) and np.all(np.isin(a[sel], r1["clusters"][t]))
+
+
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
         pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
         pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants,
-        pin_group_local_hand, pin_group_local_invariants, pin_block_routed_hand, pin_block_routed_invariants]
+        pin_group_local_hand, pin_group_local_invariants, pin_block_routed_hand, pin_block_routed_invariants,
+        pin_ivf_hand, pin_ivf_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -590,12 +627,32 @@ def _m_block_partial_blocks_routed(mp):
     mp.setattr(O, "block_routed", bad)
 
 
+def _m_kmeans_one_iteration_short(mp):
+    # the build stops one Lloyd iteration early
+    real = O.kmeans
+
+    def bad(K, C, iters, k_scale=None):
+        return real(K, C, max(0, iters - 1), k_scale)
+    mp.setattr(O, "kmeans", bad)
+
+
+def _m_ivf_no_causal_mask(mp):
+    # candidates taken from the whole cluster, later keys included
+    real = O.ivf_routed
+
+    def bad(q, w, K, k, n_probe, assign, centroids, q_pos0=0, k_scale=None, rows=None):
+        return real(q, w, K, k, n_probe, assign, centroids, q_pos0=len(assign) - q.shape[0], k_scale=k_scale,
+                    rows=rows)
+    mp.setattr(O, "ivf_routed", bad)
+
+
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
            _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
            _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group,
-           _m_block_own_block_dropped, _m_block_partial_blocks_routed]
+           _m_block_own_block_dropped, _m_block_partial_blocks_routed, _m_kmeans_one_iteration_short,
+           _m_ivf_no_causal_mask]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
