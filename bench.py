@@ -239,6 +239,78 @@ class BlockRouted(Dense):
         return self._oracle_loop(budget_s, one)
 
 
+class IvfRouted(BlockRouted):
+    """Inverted-file routing (comparator): a plain k-means index of the keys,
+    each query probing its best n_probe clusters, refined on their members."""
+    iters = 10
+    # the oracle routes on this library's index: no CPU-only reference arm
+    reference_unavailable = ("the plain k-means index of 256K keys takes minutes of CPU time; the oracle times "
+                             "routing + refine as the cpu_baseline of the GPU arm, on the GPU-built index")
+
+    def __init__(self, device, size=None, name="fp8_256k"):
+        super().__init__(device, size, name=name)
+        self.C = max(1, self.N // 128)          # about 128 keys per cluster
+        self.n_probe = self.n_blocks            # the same 8K-key budget as block routing
+        T, q0 = self.T, self.inp.q_pos0
+        # routing scores every centroid; the refine about n_probe * 128 keys
+        self.alg_pairs = T * self.C + T * self.n_probe * 128
+        self.alg_flops = self.alg_pairs * 2 * self.cfg["H"] * self.cfg["d"]
+        self.launches_per_step = 3              # routing, tiles per query, refine
+        self.kernel_launches_per_step = 2
+        self.build_ms = None
+        i = self.inp
+        # the keys enter through the index, built once outside the timed steps
+        self.host_src = [i.q, i.w] + ([i.k_scale] if i.k_scale is not None else [])
+
+    def describe(self):
+        d = Dense.describe(self)
+        d["workload"] = d["workload"].replace("dense prefill", f"IVF-routed prefill (k-means index of {self.C} "
+                                                               f"clusters, {self.iters} iterations, {self.n_probe} "
+                                                               f"probed per query, then refined)")
+        d.update(clusters=self.C, n_probe=self.n_probe, build_ms=self.build_ms,
+                 metric_pairs="dense-equivalent causal pairs (alg_pairs = centroid routing + refine)")
+        return d
+
+    def setup(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        self.index = dsa.dsa_ivf_build(i.k, self.C, iters=self.iters, K_scale=i.k_scale)
+        e1.record()
+        torch.cuda.synchronize()
+        self.build_ms = e0.elapsed_time(e1)
+        self.max_tiles = self.index.probe_tile_bound(self.n_probe)
+        T, H, d = i.q.shape
+        self.out = (torch.empty((T, self.k), dtype=torch.int32, device=i.q.device),
+                    torch.empty((T, self.k), dtype=torch.float32, device=i.q.device))
+        kd = 2 if self.cfg["k_dtype"] == "fp8" else 0
+        self.ws = torch.zeros(dsa.ivf_routed_workspace_bytes(T, self.N, H, d, self.k, self.C, self.n_probe,
+                                                             self.max_tiles, 0, kd),
+                              dtype=torch.uint8, device=i.q.device)
+
+    def call(self, q, w, ks=None):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_ivf_routed(q, w, self.index, self.k, self.n_probe, q_pos0=self.inp.q_pos0, K_scale=ks,
+                                 max_tiles=self.max_tiles, out=self.out, workspace=self.ws)
+
+    def oracle_sample(self, budget_s=15.0, seed=0):
+        from oracle import dsa_oracle as O
+        i = self.inp
+        K = i.k.cpu().numpy() if self.cfg["k_dtype"] == "fp8" else _f64(i.k)
+        ks = i.k_scale.cpu().numpy() if i.k_scale is not None else None
+        a = self.index.part("assign").cpu().numpy().astype(np.int64)
+        cen = self.index.part("centroids_bf16").cpu().double().numpy()
+        rng = np.random.default_rng(seed)
+
+        def one(_):
+            t = int(rng.integers(0, self.T))
+            O.ivf_routed(_f64(i.q[t:t + 1]), _f64(i.w[t:t + 1]), K, self.k, self.n_probe, a, cen,
+                         q_pos0=i.q_pos0 + t, k_scale=ks)
+            return i.q_pos0 + t + 1
+        return self._oracle_loop(budget_s, one)
+
+
 class Group(Workload):
     def __init__(self, device, size=None, name="group_bf16_128k", mode=0):
         from synthetic import CONFIGS, make_dense_inputs
@@ -489,6 +561,8 @@ WORKLOADS = {
     "fp8_256k_dense": lambda dev, size: Dense(dev, size, name="fp8_256k"),
     "fp8_256k_block_routed": lambda dev, size: BlockRouted(dev, size, name="fp8_256k"),
     "group_bf16_128k_block_routed": lambda dev, size: BlockRouted(dev, size, name="group_bf16_128k"),
+    "fp8_256k_ivf_routed": lambda dev, size: IvfRouted(dev, size, name="fp8_256k"),
+    "group_bf16_128k_ivf_routed": lambda dev, size: IvfRouted(dev, size, name="group_bf16_128k"),
     "fp8_256k_group_refine": lambda dev, size: Group(dev, size, "fp8_256k", 0),
     "fp8_256k_group_reuse": lambda dev, size: Group(dev, size, "fp8_256k", 1),
 }
@@ -618,6 +692,9 @@ def run_reference(args):
         return
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     wl = WORKLOADS[args.config](dev, args.T)
+    if getattr(wl, "reference_unavailable", None):
+        print(json.dumps({"impl": "reference", "unavailable": wl.reference_unavailable}))
+        return
     cores = torch.get_num_threads()
     per_step = max(1.0, 20.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):

@@ -235,6 +235,51 @@ int dsa_index_block_routed(const void* Q, const float* w, const void* K,
                            size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Inverted-file routing (AttentionIndex page: keys grouped by similarity
+ * rather than position, each query routed over the cluster centres, the
+ * candidates refined with the native indexer score), a comparator in its
+ * plain form: no learned encoder, no causal index versions (causality by
+ * masking: a query's candidates are cluster members with key <= p_t).
+ *
+ * dsa_ivf_build: Lloyd k-means over the keys (Euclidean; centroid i starts
+ *   at key floor(i N / C); nearest centroid, ties to the lower one; means;
+ *   an empty cluster keeps its centroid), `iters` >= 1 iterations, then the
+ *   keys are laid out cluster after cluster in `index` (size from
+ *   dsa_ivf_index_size; the caller owns it).  fp8 keys are clustered by
+ *   their scaled values.  Centroid sums use atomics, so the low bits of the
+ *   centroids (and, at near-ties, assignments) may differ between runs.
+ *   Layout of `index` (256-byte aligned parts): off [C+1] int32, perm [N]
+ *   int32 (clustered row -> key), assign [N] int32, keys [N, d] bf16,
+ *   centroids [C, d] bf16, centroids [C, d] fp32.
+ * dsa_index_ivf_routed: query t scores the bf16 centroids with the indexer
+ *   formula, keeps the best n_probe clusters (ties to the lower cluster),
+ *   and keeps the top-k of the native score over their members with key
+ *   <= p_t.  max_tiles bounds the 128-row tiles of one query's probed
+ *   clusters (sum of ceil(size/128)); a query above it is cut there and
+ *   DSA_ERR_INTERNAL is recorded.  cluster_idx [T, n_probe]: optional
+ *   output.  Tensor-core shape only (bf16 q, bf16 or fp8 k, H = 64,
+ *   d = 128).
+ * ---------------------------------------------------------------------- */
+int dsa_ivf_index_size(int N, int d, int C, size_t* bytes);
+int dsa_ivf_build_workspace_size(int N, int H, int d, int C, int q_dtype,
+                                 int k_dtype, size_t* bytes);
+int dsa_ivf_build(const void* K, const float* K_scale, int N, int H, int d,
+                  int C, int iters, int q_dtype, int k_dtype, void* index,
+                  size_t index_bytes, void* workspace, size_t workspace_bytes,
+                  void* stream);
+int dsa_index_ivf_routed_workspace_size(int T, int N, int H, int d, int k,
+                                        int C, int n_probe, int max_tiles,
+                                        int q_dtype, int k_dtype,
+                                        size_t* bytes);
+int dsa_index_ivf_routed(const void* Q, const float* w, const void* index,
+                         const float* K_scale, int T, int N, int H, int d,
+                         int64_t q_pos0, int k, int C, int n_probe,
+                         int max_tiles, int q_dtype, int k_dtype,
+                         int32_t* idx, float* val, int32_t* cluster_idx,
+                         void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------
  * Dense indexer that allocates nothing (the pages have no counterpart: this
  * is an integration aid).  For callers that cannot hand the library a
  * workspace — code running inside a host application that reserved all

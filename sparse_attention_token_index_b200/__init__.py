@@ -24,6 +24,9 @@ from ._binding import (  # noqa: F401
     dsa_index_decode,
     dsa_index_decode_group,
     dsa_index_block_routed,
+    dsa_ivf_build,
+    dsa_index_ivf_routed,
+    IvfIndex,
     dsa_debug_scores,
     dsa_index_dense_static,
     dsa_kernel_timer_start,
@@ -34,5 +37,6 @@ from ._binding import (  # noqa: F401
     decode_workspace_bytes,
     decode_group_workspace_bytes,
     block_routed_workspace_bytes,
+    ivf_routed_workspace_bytes,
     EXPORTED_SYMBOLS,
 )

@@ -5,6 +5,7 @@ import ctypes
 import os
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 DSA_DTYPE_BF16 = 0
@@ -27,6 +28,8 @@ EXPORTED_SYMBOLS = (
     "dsa_kernel_timer_start", "dsa_kernel_timer_stop",
     "dsa_index_decode_group_workspace_size", "dsa_index_decode_group",
     "dsa_index_block_routed_workspace_size", "dsa_index_block_routed",
+    "dsa_ivf_index_size", "dsa_ivf_build_workspace_size", "dsa_ivf_build",
+    "dsa_index_ivf_routed_workspace_size", "dsa_index_ivf_routed",
 )
 
 
@@ -60,6 +63,13 @@ _SIGS = {
     "dsa_kernel_timer_start": (_c_int, [_c_int]),
     "dsa_index_decode_group_workspace_size": (_c_int, [_c_int] * 9 + [ctypes.POINTER(_c_sz)]),
     "dsa_index_block_routed_workspace_size": (_c_int, [_c_int] * 8 + [ctypes.POINTER(_c_sz)]),
+    "dsa_ivf_index_size": (_c_int, [_c_int] * 3 + [ctypes.POINTER(_c_sz)]),
+    "dsa_ivf_build_workspace_size": (_c_int, [_c_int] * 6 + [ctypes.POINTER(_c_sz)]),
+    "dsa_ivf_build": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _c_sz, _vp,
+                               _c_sz, _vp]),
+    "dsa_index_ivf_routed_workspace_size": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_ivf_routed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                      _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _c_sz, _vp]),
     "dsa_index_block_routed": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
                                         _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _c_sz, _vp]),
     "dsa_index_decode_group": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
@@ -351,6 +361,90 @@ def dsa_index_block_routed(Q, w, K, k: int, n_blocks: int, q_pos0: Optional[int]
     if return_reps:
         res.append(rp)
     return tuple(res)
+
+
+class IvfIndex:
+    """A plain k-means inverted-file index of the keys (device buffer owned by torch).
+
+    Parts (views into ``buffer``): off [C+1], perm [N] (clustered row -> key),
+    assign [N], keys [N, d] bf16 (clustered), centroids_bf16 [C, d],
+    centroids [C, d] fp32.
+    """
+
+    def __init__(self, buffer: torch.Tensor, N: int, d: int, C: int):
+        self.buffer, self.N, self.d, self.C = buffer, N, d, C
+        o = 0
+        parts = {}
+        for name, nbytes in (("off", (C + 1) * 4), ("perm", N * 4), ("assign", N * 4), ("keys", N * d * 2),
+                             ("centroids_bf16", C * d * 2), ("centroids", C * d * 4)):
+            parts[name] = (o, nbytes)
+            o += (nbytes + 255) // 256 * 256
+        self._parts = parts
+        self.max_cluster_tiles = None
+
+    def part(self, name):
+        o, n = self._parts[name]
+        raw = self.buffer[o:o + n]
+        if name in ("off", "perm", "assign"):
+            return raw.view(torch.int32)
+        if name in ("keys", "centroids_bf16"):
+            return raw.view(torch.bfloat16).view(-1, self.d)
+        return raw.view(torch.float32).view(-1, self.d)
+
+    def probe_tile_bound(self, n_probe: int) -> int:
+        """Tiles of the n_probe largest clusters (a bound for any query's probe)."""
+        if self.max_cluster_tiles is None:
+            off = self.part("off").cpu().numpy().astype(np.int64)
+            self.max_cluster_tiles = np.sort(-(-(off[1:] - off[:-1]) // 128))[::-1]
+        return max(1, int(self.max_cluster_tiles[:n_probe].sum()))
+
+
+def dsa_ivf_build(K, C: int, iters: int = 10, K_scale=None, stream=None, check: bool = False) -> IvfIndex:
+    """Plain k-means index of the keys (Lloyd, `iters` iterations) for inverted-file routing."""
+    _need_cuda(K, K_scale)
+    N, d = K.shape
+    kd = _dtype_code(K, allow_fp8=True)
+    nb = ctypes.c_size_t(0)
+    _check(lib().dsa_ivf_index_size(N, d, C, ctypes.byref(nb)), "dsa_ivf_index_size")
+    buf = torch.zeros(int(nb.value), dtype=torch.uint8, device=K.device)
+    wb = ctypes.c_size_t(0)
+    _check(lib().dsa_ivf_build_workspace_size(N, 64, d, C, DSA_DTYPE_BF16, kd, ctypes.byref(wb)),
+           "dsa_ivf_build_workspace_size")
+    ws = torch.zeros(max(int(wb.value), 256), dtype=torch.uint8, device=K.device)
+    _check(lib().dsa_ivf_build(_ptr(K), _ptr(K_scale), N, 64, d, C, iters, DSA_DTYPE_BF16, kd, _ptr(buf), buf.numel(),
+                               _ptr(ws), ws.numel(), _stream(stream)), "dsa_ivf_build")
+    if check:
+        dsa_check_status(ws, stream)
+    return IvfIndex(buf, N, d, C)
+
+
+def ivf_routed_workspace_bytes(T, N, H, d, k, C, n_probe, max_tiles, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_ivf_routed_workspace_size(T, N, H, d, k, C, n_probe, max_tiles, q_dtype, k_dtype,
+                                                     ctypes.byref(n)), "dsa_index_ivf_routed_workspace_size")
+    return int(n.value)
+
+
+def dsa_index_ivf_routed(Q, w, index: IvfIndex, k: int, n_probe: int, q_pos0: Optional[int] = None, K_scale=None,
+                         max_tiles: Optional[int] = None, out=None, return_clusters: bool = False, workspace=None,
+                         stream=None, check: bool = False):
+    """Inverted-file routing over `index`, then the native score on the probed clusters' keys."""
+    _need_cuda(Q, w, K_scale)
+    T, H, d = Q.shape
+    N, C = index.N, index.C
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd = _dtype_code(Q)
+    kd = DSA_DTYPE_FP8_E4M3 if K_scale is not None else DSA_DTYPE_BF16
+    mt = index.probe_tile_bound(n_probe) if max_tiles is None else int(max_tiles)
+    ws = _workspace(ivf_routed_workspace_bytes(T, N, H, d, k, C, n_probe, mt, qd, kd), Q.device, workspace)
+    idx, val = _outputs(T, k, Q.device, out)
+    ci = torch.empty((T, n_probe), dtype=torch.int32, device=Q.device) if return_clusters else None
+    _check(lib().dsa_index_ivf_routed(_ptr(Q), _ptr(w), _ptr(index.buffer), _ptr(K_scale), T, N, H, d, q_pos0, k, C,
+                                      n_probe, mt, qd, kd, _ptr(idx), _ptr(val), _ptr(ci), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "dsa_index_ivf_routed")
+    if check:
+        dsa_check_status(ws, stream)
+    return (idx, val, ci) if return_clusters else (idx, val)
 
 
 def dsa_debug_scores(Q, w, K, q_pos0: Optional[int] = None, K_scale=None, workspace=None, stream=None,

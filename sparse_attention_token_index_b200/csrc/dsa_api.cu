@@ -902,3 +902,159 @@ int dsa_index_block_routed(const void* Q, const float* w, const void* K, const f
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Inverted-file routing: plain k-means index, then the native score on the
+// probed clusters' keys.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct IvfPlan {
+  size_t widen_off, scratch_off, cidx_off, cval_off, tiles_off, ref_cand_off, total;
+  DensePlan route;  // the queries against the centroids
+  int ref_grid;
+  int64_t ref_cap;
+};
+
+// Build workspace: the widened keys (fp8) and the k-means sums.
+size_t ivf_build_workspace(int64_t N, int H, int d, int C, int q_dtype, int k_dtype) {
+  Layout L;
+  take_widen(L, N, H, d, q_dtype, k_dtype);
+  L.take(ivf_build_scratch_bytes(d, C));
+  return L.off;
+}
+
+void plan_ivf(const DeviceInfo& di, int T, int N, int H, int d, int C, int n_probe, int64_t max_tiles, int q_dtype,
+              IvfPlan& p) {
+  Layout L;
+  p.widen_off = 0;
+  p.scratch_off = 0;
+  p.cidx_off = L.take((size_t)T * n_probe * sizeof(int32_t));
+  p.cval_off = L.take((size_t)T * n_probe * sizeof(float));
+  p.tiles_off = L.take((size_t)T * sizeof(int32_t));
+  p.route = plan_dense(di, T, C, H, d, q_dtype, DSA_DTYPE_BF16, L);
+  // refine: one query per unit over at most max_tiles tiles (whole groups of 4)
+  p.ref_cap = (max_tiles + 3) / 4 * 4 * 128;
+  p.ref_grid = T < di.sms ? T : di.sms;
+  p.ref_cand_off = L.take((size_t)p.ref_grid * 4 * p.ref_cap * sizeof(uint2));
+  p.total = L.off;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_ivf_index_size(int N, int d, int C, size_t* bytes) {
+  if (!bytes || N < 1 || d < 32 || d > 256 || d % 32 || C < 1 || C > N || C > 65536) return DSA_ERR_INVALID_ARG;
+  *bytes = ivf_index_view(nullptr, N, d, C).bytes;
+  return DSA_OK;
+}
+
+int dsa_ivf_build_workspace_size(int N, int H, int d, int C, int q_dtype, int k_dtype, size_t* bytes) {
+  if (!bytes || N < 1 || C < 1 || C > N || C > 65536) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, 1, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  *bytes = ivf_build_workspace(N, H, d, C, q_dtype, k_dtype);
+  return DSA_OK;
+}
+
+int dsa_ivf_build(const void* K, const float* K_scale, int N, int H, int d, int C, int iters, int q_dtype,
+                  int k_dtype, void* index, size_t index_bytes, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int r = check_common(H, d, 1, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!K || !index || !workspace || N < 1 || C < 1 || C > N || C > 65536 || iters < 1 || iters > 1000)
+    return DSA_ERR_INVALID_ARG;
+  if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(index)) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  const IvfIndex x = ivf_index_view(index, N, d, C);
+  if (index_bytes < x.bytes) return DSA_ERR_WORKSPACE;
+  if (workspace_bytes < ivf_build_workspace(N, H, d, C, q_dtype, k_dtype)) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Layout L;
+  const size_t widen_off = take_widen(L, N, H, d, q_dtype, k_dtype);
+  const size_t scratch_off = L.take(ivf_build_scratch_bytes(d, C));
+  if (needs_widen(H, d, q_dtype, k_dtype)) {
+    if ((r = widen_keys(K, N, d, ws, widen_off, st)) != DSA_OK) return r;
+    K = ws + widen_off;
+  }
+  return ivf_build(K, K_scale, N, d, C, iters, x, ws + scratch_off, st);
+}
+
+int dsa_index_ivf_routed_workspace_size(int T, int N, int H, int d, int k, int C, int n_probe, int max_tiles,
+                                        int q_dtype, int k_dtype, size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (T < 1 || N < 1 || C < 1 || n_probe < 1 || n_probe > C || max_tiles < 1) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  IvfPlan p;
+  plan_ivf(di, T, N, H, d, C, n_probe, max_tiles, q_dtype, p);
+  *bytes = p.total;
+  return DSA_OK;
+}
+
+int dsa_index_ivf_routed(const void* Q, const float* w, const void* index, const float* K_scale, int T, int N,
+                         int H, int d, int64_t q_pos0, int k, int C, int n_probe, int max_tiles, int q_dtype,
+                         int k_dtype, int32_t* idx, float* val, int32_t* cluster_idx, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  if (!Q || !w || !index || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
+  if (T < 1 || N < 1 || q_pos0 < 0 || q_pos0 + (int64_t)T > (int64_t)N) return DSA_ERR_INVALID_ARG;
+  if (C < 1 || C > N || n_probe < 1 || n_probe > C || max_tiles < 1) return DSA_ERR_INVALID_ARG;
+  if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(w) || !aligned16(index)) return DSA_ERR_INVALID_ARG;
+  if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((r = device_info(di)) != DSA_OK) return r;
+  IvfPlan p;
+  plan_ivf(di, T, N, H, d, C, n_probe, max_tiles, q_dtype, p);
+  if (workspace_bytes < p.total) return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const IvfIndex x = ivf_index_view(const_cast<void*>(index), N, d, C);
+  // 1. routing: every centroid is visible to every query (pos = C - 1)
+  int32_t* ci = cluster_idx ? cluster_idx : reinterpret_cast<int32_t*>(ws + p.cidx_off);
+  float* cv = reinterpret_cast<float*>(ws + p.cval_off);
+  if ((r = run_dense_rows(di, p.route, Q, w, x.cen_bf16, nullptr, T, C, H, d, C - 1, 0, 0, 0, n_probe, q_dtype,
+                          DSA_DTYPE_BF16, ci, cv, ws, nullptr, 0, st)) != DSA_OK)
+    return r;
+  // 2. the tiles each query streams, then the refine over its clusters' keys
+  int32_t* tiles = reinterpret_cast<int32_t*>(ws + p.tiles_off);
+  if ((r = launch_ivf_tiles(ci, n_probe, T, x.off, tiles, st)) != DSA_OK) return r;
+  CUtensorMap tmQ, tmK;
+  if ((r = make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  if ((r = make_map_bf16(&tmK, x.keys, (uint64_t)N, (uint64_t)d, 128)) != DSA_OK) return r;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kind = 4;
+  a.k_scale = K_scale;
+  a.n_rows = T;
+  a.n_units = T;
+  a.k = k;
+  a.pos_base = q_pos0;
+  a.w = w;
+  a.out_idx = idx;
+  a.out_val = val;
+  a.out_ld = k;
+  a.cand = reinterpret_cast<uint2*>(ws + p.ref_cand_off);
+  a.cand_cap = p.ref_cap;
+  a.status = reinterpret_cast<int*>(ws);
+  a.key_map = x.perm;
+  a.route_blocks = ci;
+  a.route_n = n_probe;
+  a.ivf_off = x.off;
+  a.ivf_tiles = tiles;
+  a.ivf_max_tiles = max_tiles;
+  return launch_tc_index(tmQ, tmK, a, p.ref_grid, st);
+}
+
+}  // extern "C"

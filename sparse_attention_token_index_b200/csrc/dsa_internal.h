@@ -59,6 +59,13 @@ struct TcArgs {
   // partial block, keys <= its position
   const int32_t* route_blocks;
   int route_n;
+  // kind 4 (inverted-file refine): one query row per unit over its probed
+  // clusters (route_blocks / route_n: cluster lists), whose keys sit at
+  // sorted rows ivf_off[c] .. ivf_off[c+1]-1 (key_map: sorted row -> key);
+  // ivf_tiles[row]: the tiles it streams
+  const int32_t* ivf_off;
+  const int32_t* ivf_tiles;
+  int ivf_max_tiles;  // candidate lists hold this many tiles per query
 };
 
 // Event pair for timing one scoring-kernel launch (dsa_timer.cu); both null
@@ -129,5 +136,21 @@ int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
 int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, void* R, cudaStream_t stream);
 // Exact e4m3 -> bf16 copy of n bytes (n a multiple of 16, both 16-byte aligned).
 int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream);
+
+// Inverted-file index (dsa_ivf.cu): views into the caller's index buffer.
+struct IvfIndex {
+  int32_t* off;     // [C+1] first sorted row of each cluster
+  int32_t* perm;    // [N] sorted row -> key index
+  int32_t* assign;  // [N] cluster of each key
+  void* keys;       // [N, d] bf16, cluster after cluster
+  void* cen_bf16;   // [C, d] bf16 centroids (routing)
+  float* cen;       // [C, d] fp32 centroids
+  size_t bytes;
+};
+IvfIndex ivf_index_view(void* base, int64_t N, int d, int C);
+size_t ivf_build_scratch_bytes(int d, int C);
+int ivf_build(const void* K, const float* K_scale, int64_t N, int d, int C, int iters, const IvfIndex& x,
+              uint8_t* scratch, cudaStream_t st);
+int launch_ivf_tiles(const int32_t* list, int n_probe, int T, const int32_t* off, int32_t* tiles, cudaStream_t st);
 
 }  // namespace dsa

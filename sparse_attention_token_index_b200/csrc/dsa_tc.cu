@@ -74,6 +74,37 @@ struct UnitInfo {
   int rown;          // routed: the query's own partial block, streamed last
 };
 
+// Sorted-key rows an inverted-file unit streams: its probed clusters one after
+// the other, 128 rows a tile (a cluster's last tile is cut at the cluster's
+// end).  The producer and the epilogue each step one through every tile.
+struct ClusterWalk {
+  const int32_t* list;
+  int n, ci, row, end;
+  __device__ __forceinline__ void seek(const TcArgs& a) {  // first non-empty cluster from ci on
+    while (ci < n) {
+      const int c = list[ci];
+      row = c >= 0 ? a.ivf_off[c] : 0;
+      end = c >= 0 ? a.ivf_off[c + 1] : 0;
+      if (row < end) return;
+      ++ci;
+    }
+    row = end = 0;
+  }
+  __device__ __forceinline__ void start(const TcArgs& a, int t) {
+    list = a.route_blocks + (int64_t)t * a.route_n;
+    n = a.route_n;
+    ci = 0;
+    seek(a);
+  }
+  __device__ __forceinline__ void next(const TcArgs& a) {
+    row += 128;
+    if (row >= end) {
+      ++ci;
+      seek(a);
+    }
+  }
+};
+
 // Key block of iteration j of a routed unit: its routed blocks, then its own.
 __device__ __forceinline__ int routed_block(const TcArgs& a, const UnitInfo& u, int j) {
   return j < u.rsel ? a.route_blocks[(int64_t)u.row0 * a.route_n + j] : u.rown;
@@ -103,6 +134,22 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     u.nkeys = (int)(maxpos + 1);
     u.seq_split = -1;
     u.partial = 0;
+  } else if constexpr (kKind == 4) {
+    // inverted-file refine: one query row over its probed clusters (longest first)
+    const int t = a.n_units - 1 - v;
+    u.row0 = t;
+    u.nq = 1;
+    u.key_row0 = 0;
+    u.tile0 = 0;
+    u.ntiles = a.ivf_tiles[t];
+    if (u.ntiles > a.ivf_max_tiles) {  // more tiles than the candidate lists hold: report, stay in bounds
+      if (threadIdx.x == 0) report_error(a.status, DSA_ERR_INTERNAL, 5);
+      u.ntiles = a.ivf_max_tiles;
+    }
+    u.nkeys = 0;  // rows are checked against their cluster's end
+    u.seq_split = -1;
+    u.partial = 0;
+    u.pos0 = (int)(a.pos_base + t);
   } else if constexpr (kKind == 3) {
     // routed refine: one query row over its routed blocks (longest first)
     const int t = a.n_units - 1 - v;
@@ -296,10 +343,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(S.q + c * kQChunkBytes + q * kQHeadBlockBytes, &tmQ, &S.q_full, c * 64,
                         (u.row0 + q) * kHeads);
         ++qi;
+        ClusterWalk walk;
+        if constexpr (kKind == 4) walk.start(a, u.row0);
         for (int j = 0; j < u.ntiles; ++j) {
           if (!(ok = mbar_wait(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11))) break;
           mbar_arrive_expect_tx(&S.k_full[s], (uint32_t)kKStageBytes);
-          const int row = (kKind == 3) ? routed_block(a, u, j) * kTileKeys : u.key_row0 + (u.tile0 + j) * kTileKeys;
+          int row;
+          if constexpr (kKind == 4) {
+            row = walk.row;
+            walk.next(a);
+          } else {
+            row = (kKind == 3) ? routed_block(a, u, j) * kTileKeys : u.key_row0 + (u.tile0 + j) * kTileKeys;
+          }
           for (int c = 0; c < 2; ++c)
             tma_load_2d(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row);
           armed |= 1u << s;
@@ -408,7 +463,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const unsigned n_vis = (unsigned)(pos + 1);
       const int ntiles = u.ntiles, nkeys = u.nkeys;
       const int key0 = u.tile0 * kTileKeys + lq * 32 + lane;
-      const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : nullptr;
+      const int32_t* kmap = (kKind == 2) ? a.key_map + (int64_t)u.seq_split * a.bank : (kKind == 4 ? a.key_map : nullptr);
       // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0; decode
       // groups index the scales of their own sequence
       const float* kscale =
@@ -423,6 +478,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (ttid == 0) tb_open(st);
       }
       int count = 0;  // my segment's fill
+      ClusterWalk walk;
+      if constexpr (kKind == 4) walk.start(a, u.row0);
       for (int jt = 0; jt < ntiles; ++jt) {
         if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30)) {
           ok = false;
@@ -451,8 +508,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         eph ^= 1u << buf;
         buf ^= 1;
         if (mine) {
-          const int key = key0 + (kKind == 3 ? routed_block(a, u, jt) : jt) * kTileKeys;  // local key index
-          const bool in_range = key < nkeys;
+          int key;  // local key index (inverted file: sorted key row)
+          bool in_range;
+          if constexpr (kKind == 4) {
+            key = walk.row + lq * 32 + lane;
+            in_range = key < walk.end;
+          } else {
+            key = key0 + (kKind == 3 ? routed_block(a, u, jt) : jt) * kTileKeys;
+            in_range = key < nkeys;
+          }
           int kpos = key;
           if (kmap != nullptr) kpos = in_range ? kmap[key] : -1;
           const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
@@ -463,6 +527,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
           row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
         }
+        if constexpr (kKind == 4) walk.next(a);
       }
       if (!active) {
         ok = group_and(1 + slot, 128, ok);
@@ -517,7 +582,7 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream) {
-  if (a.kind < 0 || a.kind > 3 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
+  if (a.kind < 0 || a.kind > 4 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
   const TimerSlot ts = timer_acquire();
   if (ts.start) cudaEventRecord(ts.start, stream);
   int r;
@@ -529,8 +594,10 @@ int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs
     r = launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 2)
     r = launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
-  else
+  else if (a.kind == 3)
     r = launch_tc<false, 3>(tmQ, tmK, a, grid, stream);
+  else
+    r = launch_tc<false, 4>(tmQ, tmK, a, grid, stream);
   if (ts.end) cudaEventRecord(ts.end, stream);
   return r;
 }
