@@ -158,7 +158,7 @@ DensePlan plan_dense(const DeviceInfo& di, int T, int N, int H, int d, int q_dty
 int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, const float* w, const void* K,
                    const float* K_scale, int n_rows, int N, int H, int d, int64_t pos_base, int64_t pos_mul,
                    int64_t pos_add, int64_t pos_clamp, int k, int q_dtype, int k_dtype, int32_t* idx, float* val,
-                   uint8_t* ws, float* dbg, int64_t dbg_ld, cudaStream_t st, int64_t pos_div = 0) {
+                   uint8_t* ws, float* dbg, int64_t dbg_ld, cudaStream_t st, int pos_shift = 0) {
   int* status = reinterpret_cast<int*>(ws);
   uint2* cand = reinterpret_cast<uint2*>(ws + p.cand_off);
   if (p.tc) {
@@ -178,7 +178,7 @@ int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, cons
     a.pos_mul = pos_mul;
     a.pos_add = pos_add;
     a.pos_clamp = pos_clamp;
-    a.pos_div = pos_div;
+    a.pos_shift = pos_shift;
     a.w = w;
     a.out_idx = idx;
     a.out_val = val;
@@ -875,7 +875,7 @@ int dsa_index_block_routed(const void* Q, const float* w, const void* K, const f
   int32_t* bi = block_idx ? block_idx : reinterpret_cast<int32_t*>(ws + p.bidx_off);
   float* bv = reinterpret_cast<float*>(ws + p.bval_off);
   if ((r = run_dense_rows(di, p.route, Q, w, R, nullptr, T, (int)p.nblocks, H, d, q_pos0, 1, 0, (int64_t)T, n_blocks,
-                          q_dtype, DSA_DTYPE_BF16, bi, bv, ws, nullptr, 0, st, 128)) != DSA_OK)
+                          q_dtype, DSA_DTYPE_BF16, bi, bv, ws, nullptr, 0, st, 7)) != DSA_OK)  // 128-key blocks
     return r;
   // 3. refine: the native score over the routed blocks and the own partial block
   CUtensorMap tmQ, tmK;

@@ -51,9 +51,9 @@ struct TcArgs {
   int mblocks;
   int T;
   int key_slots;   // nonzero: every slot is streamed, key_map alone marks the valid ones
-  // kind 0 rows see (pos_base + r + 1) / pos_div - 1 when pos_div > 0 (the
-  // complete 128-key blocks before a query, for block routing)
-  int64_t pos_div;
+  // kind 0 rows see ((pos_base + r + 1) >> pos_shift) - 1 when pos_shift > 0
+  // (the complete 128-key blocks before a query, for block routing)
+  int pos_shift;
   // kind 3 (routed refine): one query row per unit; it streams the blocks
   // route_blocks[row, 0 .. min(route_n, complete blocks)) then its own
   // partial block, keys <= its position

@@ -111,7 +111,7 @@ __device__ __forceinline__ int routed_block(const TcArgs& a, const UnitInfo& u, 
 }
 
 __device__ __forceinline__ int64_t prefill_pos(const TcArgs& a, int r) {
-  if (a.pos_div > 0) return (a.pos_base + r + 1) / a.pos_div - 1;
+  if (a.pos_shift > 0) return ((a.pos_base + r + 1) >> a.pos_shift) - 1;
   int64_t v = (int64_t)r * a.pos_mul + a.pos_add;
   if (v > a.pos_clamp) v = a.pos_clamp;
   return a.pos_base + v;
