@@ -645,11 +645,17 @@ def _barrier(dist):
 
 
 def _kernel_source_hash():
+    """sha256 (16 hex digits) of the scoring kernel's sources with comments
+    and whitespace removed: only a change of code makes a capture stale."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in ("dsa_tc.cu", "dsa_topk.cuh", "dsa_common.cuh"):
-        with open(os.path.join(ROOT, "sparse_attention_token_index_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "sparse_attention_token_index_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
 
 

@@ -5,7 +5,9 @@
 //   * bank_rank_reuse: ranks each group's bank by (proxy score desc, key
 //     asc) with a shared-memory bitonic sort and, for Reuse, hands each
 //     member the first k ranked keys it may see;
-//   * decode_merge: combines the per-split top-k lists of a decode query.
+//   * decode_merge: combines the per-split top-k lists of a decode query;
+//   * local_extend: bank + a group's own stretch (Refine with local additions);
+//   * block_mean: block representatives for block routing.
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
 #include "dsa_internal.h"

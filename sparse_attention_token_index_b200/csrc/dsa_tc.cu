@@ -17,11 +17,14 @@
 //     packed fp32x2 FMAs, and the causal cut and the streaming top-k filter
 //     follow at once.
 //
-// Work units come in three kinds: prefill rows (dense queries or group
-// proxies, each row with its own causal position), decode segments (the m
-// new queries of one sequence against one slice of that sequence's key
-// cache; a merge kernel combines the slices), and group-refine blocks (up to
-// 4 members of a group against the group's gathered candidate bank).
+// Work units come in five kinds (a template parameter): prefill rows (dense
+// queries, group proxies or block-routing rows, each row with its own causal
+// position), decode segments (the m new queries of one sequence against one
+// slice of that sequence's key cache; a merge kernel combines the slices),
+// group-refine blocks (up to 4 members of a group against the group's
+// gathered candidate bank), and the refine stages of the two routing
+// comparators (one query against its routed key blocks, or against its
+// probed clusters in the clustered keys).
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
 #include "dsa_internal.h"

@@ -93,3 +93,29 @@ def test_decode_host_checks(L):
     assert f(ok, ok, ok, None, ok, ok, 1, 2, 100, 101, 64, 128, 16, 0, 0, ok, ok, ok, 1 << 20, None) == -1
     # more keys than 32-bit TMA row coordinates reach (tensor-core shape)
     assert f(ok, ok, ok, None, ok, ok, 1, 2, 1 << 31, 1 << 20, 64, 128, 16, 0, 0, ok, ok, ok, 1 << 20, None) == -2
+
+
+def test_comparator_and_group_host_checks(L):
+    ok = ctypes.c_void_p(4096)
+    n = ctypes.c_size_t(0)
+    # block routing: null Q, zero blocks
+    f = L.dsa_index_block_routed
+    assert f(None, ok, ok, None, 8, 256, 64, 128, 248, 4, 2, 0, 0, ok, ok, None, None, ok, 1 << 20, None) == -1
+    assert f(ok, ok, ok, None, 8, 256, 64, 128, 248, 4, 0, 0, 0, ok, ok, None, None, ok, 1 << 20, None) == -1
+    # inverted file: more clusters than keys, d not a multiple of 32
+    assert L.dsa_ivf_index_size(100, 128, 200, ctypes.byref(n)) == -1
+    assert L.dsa_ivf_index_size(100, 100, 10, ctypes.byref(n)) == -1
+    assert L.dsa_ivf_index_size(100, 128, 10, ctypes.byref(n)) == 0 and n.value > 100 * 128 * 2
+    # routed query: more probes than clusters
+    g = L.dsa_index_ivf_routed
+    assert g(ok, ok, ok, None, 8, 256, 64, 128, 248, 4, 10, 11, 4, 0, 0, ok, ok, None, ok, 1 << 20, None) == -1
+    # decode group: bank smaller than k, unknown mode
+    h = L.dsa_index_decode_group
+    assert h(ok, ok, ok, None, ok, ok, 1, 2, 100, 100, 64, 128, 16, 8, 0, 0, 0, ok, ok, None, None, None, None, ok,
+             1 << 20, None) == -1
+    assert h(ok, ok, ok, None, ok, ok, 1, 2, 100, 100, 64, 128, 16, 32, 7, 0, 0, ok, ok, None, None, None, None, ok,
+             1 << 20, None) == -1
+    # group: unknown mode
+    gg = L.dsa_index_group
+    assert gg(ok, ok, ok, None, 8, 8, 64, 128, 0, 4, 2, 8, 7, 0, 0, ok, ok, None, None, None, None, ok, 1 << 20,
+              None) == -1
