@@ -175,3 +175,20 @@ def test_fp8_debug_scores_tensor_core():
     pos = inp.q_pos0 + np.arange(200)
     ref = np.where(np.arange(300)[None, :] <= pos[:, None], ref, -np.inf)
     check_scores(S.cpu().numpy(), ref, what="fp8 tc")
+
+
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_maximum_k(path):
+    # k at its maximum (65536) over a prefix a little longer: the threshold bin
+    # holds thousands of entries, so the select's sub-bin and radix paths run
+    N, T, k = 70000, 6, 65536
+    if path == "tc":
+        inp = make_dense_inputs("dense_bf16_32k", device=DEV, T=T, N=N, seed=71)
+    else:
+        inp = make_dense_inputs("tiny_fp32_2k", device=DEV, T=T, N=N, seed=71)
+    idx, val = dsa.dsa_index_dense(inp.q, inp.w, inp.k, k, q_pos0=inp.q_pos0, check=True)
+    q, w, K = _f64(inp.q), _f64(inp.w), _f64(inp.k)
+    S = O.score_rows(q, w, K)
+    rows = list(range(T))
+    check_rows(idx.cpu().numpy(), val.cpu().numpy(), [S[t, :inp.q_pos0 + t + 1] for t in rows], k,
+               what=f"max k {path}")

@@ -198,3 +198,10 @@ def test_refine_local_full_size_sampled():
             w = inp.w[t:t + 1].double().cpu().numpy()
             S = O.score_rows(q, w, K[:p + 1])[0]
             check_row(gi[t], gv[t], S[cand], k, what=f"refine_local t={t}", idx_map=cand)
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+def test_group_maximum_bank(mode):
+    # the largest bank the ABI takes (16384) with k = 4096
+    inp = make_dense_inputs("group_bf16_128k", device=DEV, T=192, N=20000, seed=72)
+    _check_group(inp, 4096, 64, 16384, mode, "bank 16384")
