@@ -644,19 +644,30 @@ def _barrier(dist):
         dist.barrier()
 
 
-def _kernel_source_hash():
-    """sha256 (16 hex digits) of the scoring kernel's sources with comments
-    and whitespace removed: only a change of code makes a capture stale."""
+def kernel_source_hash(read):
+    """sha256 (16 hex digits) of the scoring kernel's device code: dsa_tc.cu
+    up to its host launchers, dsa_topk.cuh and dsa_common.cuh, without
+    comments, #include lines and whitespace.  `read(name)` returns a file's
+    text.  Only a change of device code makes a traffic capture stale."""
     import hashlib
     import re
     h = hashlib.sha256()
     for f in ("dsa_tc.cu", "dsa_topk.cuh", "dsa_common.cuh"):
-        with open(os.path.join(ROOT, "sparse_attention_token_index_b200", "csrc", f)) as fh:
-            src = fh.read()
+        src = read(f)
+        if f == "dsa_tc.cu":
+            src = src[:src.index("static int launch_tc(")]
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
+        src = re.sub(r"#include[^\n]*", "", src)
         h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
+
+
+def _kernel_source_hash():
+    def read(name):
+        with open(os.path.join(ROOT, "sparse_attention_token_index_b200", "csrc", name)) as fh:
+            return fh.read()
+    return kernel_source_hash(read)
 
 
 def _traffic(config):

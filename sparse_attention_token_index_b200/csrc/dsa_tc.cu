@@ -25,6 +25,8 @@
 // gathered candidate bank), and the refine stages of the two routing
 // comparators (one query against its routed key blocks, or against its
 // probed clusters in the clustered keys).
+#include <atomic>
+
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
 #include "dsa_internal.h"
@@ -572,12 +574,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 template <bool kDebug, int kKind>
 static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
+  // the shared-memory opt-in is a per-device function attribute: set it once
+  // on each device the kernel runs on
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
     if (cudaFuncSetAttribute(tc_index_kernel<kDebug, kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kTcSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
-    configured = true;
+    configured.fetch_or(bit, std::memory_order_release);
   }
   tc_index_kernel<kDebug, kKind><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
