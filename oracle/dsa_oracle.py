@@ -175,6 +175,21 @@ def dense(q, w, K, k, q_pos0=0, k_scale=None, rows=None, return_scores=False):
     return res
 
 
+def round_bf16(x):
+    """Round float64 values to the nearest bfloat16 (8 significant bits),
+    ties to even.  The group form stores its proxy query in the query's own
+    dtype, and block routing its representatives in bf16; this is that
+    rounding, applied to the float64 means.  Zero stays zero; values are
+    assumed in the normal bf16 range."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    e = np.floor(np.log2(np.abs(x[nz])))
+    ulp = np.exp2(e - 7)
+    out[nz] = np.round(x[nz] / ulp) * ulp   # np.round: half to even
+    return out
+
+
 def proxy(q, w, G):
     """PIVOT proxy per group of G consecutive rows: the members' mean q and mean w.
 

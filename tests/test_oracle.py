@@ -410,13 +410,28 @@ def pin_ivf_invariants(O):
         assert np.all(sel <= 40 + t) and np.all(np.isin(a[sel], r1["clusters"][t]))
 
 
+def pin_round_bf16_library(O):
+    # against torch's float32 -> bfloat16 conversion (round to nearest even)
+    # on values exactly representable in float32, where both see the same number
+    import torch
+    rng = np.random.default_rng(16)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+                        [1.0, -1.0, 1.00390625, 1.01171875, 3.0, 255.5, -0.0078125]])
+    x32 = x.astype(np.float32).astype(np.float64)
+    ref = torch.tensor(x32, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.round_bf16(x32), ref)
+    # ties: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 and goes to the even 1
+    assert O.round_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0
+    assert O.round_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+
+
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
         pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
         pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants,
         pin_group_local_hand, pin_group_local_invariants, pin_block_routed_hand, pin_block_routed_invariants,
-        pin_ivf_hand, pin_ivf_invariants]
+        pin_ivf_hand, pin_ivf_invariants, pin_round_bf16_library]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -646,13 +661,25 @@ def _m_ivf_no_causal_mask(mp):
     mp.setattr(O, "ivf_routed", bad)
 
 
+def _m_round_bf16_truncate(mp):
+    # bf16 rounding that truncates the mantissa instead of rounding to nearest
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        out = np.zeros_like(x)
+        nz = x != 0
+        ulp = np.exp2(np.floor(np.log2(np.abs(x[nz]))) - 7)
+        out[nz] = np.trunc(x[nz] / ulp) * ulp
+        return out
+    mp.setattr(O, "round_bf16", bad)
+
+
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
            _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
            _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group,
            _m_block_own_block_dropped, _m_block_partial_blocks_routed, _m_kmeans_one_iteration_short,
-           _m_ivf_no_causal_mask]
+           _m_ivf_no_causal_mask, _m_round_bf16_truncate]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS, ids=[m.__name__ for m in MUTANTS])
