@@ -93,6 +93,19 @@ class Workload:
         host_out[0].copy_(self.out[0], non_blocking=True)
         host_out[1].copy_(self.out[1], non_blocking=True)
 
+    e2e_note = ("pinned host inputs copied in (torch copies on the stream), the device entry point, idx/val "
+                "copied out, every step")
+
+    def _host_e2e_buffers(self, staging_bytes):
+        """Buffers of the host-buffer entry point: a device staging buffer
+        and page-locked outputs; the byte counts are the step's copies."""
+        self.staging = torch.empty(staging_bytes, dtype=torch.uint8, device=self.out[0].device)
+        hout = [torch.empty(self.out[0].shape, dtype=torch.int32).pin_memory(),
+                torch.empty(self.out[1].shape, dtype=torch.float32).pin_memory()]
+        h2d = sum(t.numel() * t.element_size() for t in self.host_src)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        return None, hout, h2d, d2h
+
     def step(self):
         self.call(*self.host_src)
 
@@ -166,10 +179,29 @@ class Dense(Workload):
         return self._oracle_loop(budget_s, one)
 
 
+    e2e_note = ("dsa_index_dense_host: page-locked host inputs and outputs, copy-in / indexer / copy-out "
+                "pipelined in row chunks by the library, every step")
+
+    def e2e_buffers(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        T, H, d = i.q.shape
+        kd = dsa.DSA_DTYPE_FP8_E4M3 if i.k_scale is not None else dsa.DSA_DTYPE_BF16
+        return self._host_e2e_buffers(dsa.dense_host_staging_bytes(T, self.N, H, d, self.k, dsa.DSA_DTYPE_BF16, kd))
+
+    def e2e_step(self, host, dev_bufs, host_out):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_dense_host(host[0], host[1], host[2], self.k, q_pos0=self.inp.q_pos0,
+                                 K_scale=host[3] if len(host) > 3 else None, out=host_out, staging=self.staging)
+
+
 class BlockRouted(Dense):
     """Two-stage selection over 128-key blocks (comparator): route each query
     to its best n_blocks complete blocks by their mean key, refine on them."""
     n_blocks = 64   # an 8K-key candidate budget
+    e2e_buffers = Workload.e2e_buffers
+    e2e_step = Workload.e2e_step
+    e2e_note = Workload.e2e_note
 
     def __init__(self, device, size=None, name="fp8_256k"):
         super().__init__(device, size, name=name)
@@ -369,6 +401,23 @@ class Group(Workload):
         dsa.dsa_index_group(q, w, k, self.k, self.G, self.B, mode=self.mode, q_pos0=self.inp.q_pos0, K_scale=ks,
                             out=self.out, workspace=self.ws)
 
+    e2e_note = ("dsa_index_group_host: page-locked host inputs and outputs, copy-in / indexer / copy-out "
+                "pipelined in chunks of whole groups by the library, every step")
+
+    def e2e_buffers(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        T, H, d = i.q.shape
+        kd = dsa.DSA_DTYPE_FP8_E4M3 if i.k_scale is not None else dsa.DSA_DTYPE_BF16
+        return self._host_e2e_buffers(dsa.group_host_staging_bytes(T, self.N, H, d, self.k, self.G, self.B,
+                                                                   dsa.DSA_DTYPE_BF16, kd))
+
+    def e2e_step(self, host, dev_bufs, host_out):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_group_host(host[0], host[1], host[2], self.k, self.G, self.B, mode=self.mode,
+                                 q_pos0=self.inp.q_pos0, K_scale=host[3] if len(host) > 3 else None, out=host_out,
+                                 staging=self.staging)
+
     def recall(self, blocks=4, rows=512):
         """Mean recall of the exact dense top-k (this library's dense kernel)
         by the group output, over `blocks` row blocks spread over the
@@ -453,6 +502,23 @@ class Decode(Workload):
         dsa.dsa_index_decode(q, w, k, self.k, self.ko, self.qo, max_keys=self.cfg["Nb"], total_keys=self.total_keys,
                              out=self.out, workspace=self.ws)
 
+    e2e_note = ("dsa_index_decode_host: page-locked host caches, queries and outputs, one copy-in / indexer / "
+                "copy-out per step")
+
+    def e2e_buffers(self):
+        import sparse_attention_token_index_b200 as dsa
+        i = self.inp
+        c = self.cfg
+        self.ko_h, self.qo_h = i.k_offsets.cpu().to(torch.int64), i.q_offsets.cpu().to(torch.int32)
+        return self._host_e2e_buffers(dsa.decode_host_staging_bytes(c["B"], i.q.shape[0], self.total_keys, c["Nb"],
+                                                                    c["H"], c["d"], self.k, dsa.DSA_DTYPE_BF16,
+                                                                    dsa.DSA_DTYPE_BF16))
+
+    def e2e_step(self, host, dev_bufs, host_out):
+        import sparse_attention_token_index_b200 as dsa
+        dsa.dsa_index_decode_host(host[0], host[1], host[2], self.k, self.ko_h, self.qo_h, max_keys=self.cfg["Nb"],
+                                  out=host_out, staging=self.staging)
+
     def oracle_sample(self, budget_s=15.0, seed=0):
         from oracle import dsa_oracle as O
         i = self.inp
@@ -476,6 +542,9 @@ class Decode(Workload):
 class DecodeGroup(Decode):
     """PIVOT in decode: each sequence's new queries form one group (bank 8192)."""
     bank = 8192
+    e2e_buffers = Workload.e2e_buffers
+    e2e_step = Workload.e2e_step
+    e2e_note = Workload.e2e_note
     alg_bytes_note = "cached keys once + proxies (+ Refine: gathered bank keys, queries, weights)"
 
     def __init__(self, device, size=None, mode=0):
@@ -843,7 +912,7 @@ def main():
         e2e_ms = _max_over_ranks(dist, e0.elapsed_time(e1))
         e2e = {"value": whole_job_rate(wl.pairs, world, n_e2e, e2e_ms) / 1e9, "unit": "Gpairs/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "note": "pinned host inputs copied in, indexer run, idx/val copied out, every step"}
+               "note": wl.e2e_note}
 
     recall = wl.recall() if hasattr(wl, "recall") else None   # after timing; the last step's output
     cpu = None

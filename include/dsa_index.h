@@ -23,7 +23,8 @@
  * index -1 and score -inf.
  *
  * Conventions for every call below
- *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device
+ *     (except the *_host calls, whose tensors are in host memory),
  *     row-major and contiguous, 16-byte aligned.  Offsets arrays of the decode
  *     call are device pointers too.
  *   - The caller owns every buffer, including `workspace`; the library never
@@ -32,6 +33,8 @@
  *   - Size the workspace with the matching *_workspace_size call; its first
  *     bytes hold a device status word that kernels set on a device-side
  *     failure (a bounded wait that gave up); read it with dsa_check_status.
+ *     Zero the workspace's first 8 bytes before its first use;
+ *     dsa_check_status clears the word again after reading it.
  *   - Return value: DSA_OK or a negative DSA_ERR_* code; on an error nothing
  *     has been launched.
  *   - Supported shapes: bf16 Q/K with H = 64, d = 128 run on the tcgen05
@@ -304,6 +307,64 @@ int dsa_index_ivf_routed(const void* Q, const float* w, const void* index,
 int dsa_index_dense_static(const void* Q, const float* w, const void* K, int T,
                            int N, int H, int d, int64_t q_pos0, int k,
                            int32_t* idx, float* val, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Host-buffer entry points (an integration aid; the pages have none): the
+ * dense, group and decode indexers above with every tensor argument in HOST
+ * memory — inputs, outputs and, for decode, the offsets arrays.  Same
+ * operation, argument meaning, layouts and results as the device calls.
+ *   staging: a DEVICE buffer of at least *_host_staging_size bytes, 16-byte
+ *          aligned, owned by the caller; the call stages the inputs, the
+ *          outputs and the indexer's workspace in it (no zeroing needed).
+ *   chunk_rows (dense, group): rows per pipeline chunk, 0 for the library's
+ *          choice (about 16 chunks of at least 1024 rows, at most 64
+ *          chunks), rounded up to a multiple of 4 (dense) or of `group`, so
+ *          that every group lies inside one chunk and the results equal one
+ *          call over all rows.  The keys are copied first; then, chunk by
+ *          chunk, the copy in of chunk c+1, the indexer on chunk c and the
+ *          copy out of chunk c-1 overlap: the copies run on two streams the
+ *          call creates and destroys, the indexer on `stream`, ordered by
+ *          events.  The group staging size depends on chunk_rows: pass the
+ *          same value to both calls.
+ *   Decode is one chunk (the cache copy dwarfs the scan); its copies and
+ *          the indexer run on `stream`.
+ *   Synchronous: returns once the outputs are in host memory (or an error
+ *   has stopped the call and every copy it queued has drained), with
+ *   DSA_OK, a DSA_ERR_* of the arguments or of a CUDA call, or the device
+ *   status of the call (DSA_ERR_TIMEOUT, DSA_ERR_INTERNAL).
+ *   Host buffers should be page-locked (cudaHostAlloc, cudaHostRegister):
+ *   then the copies overlap the indexer; pageable memory gives the same
+ *   results with the copies serialised by the driver.
+ * ---------------------------------------------------------------------- */
+int dsa_index_dense_host_staging_size(int T, int N, int H, int d, int k,
+                                      int q_dtype, int k_dtype,
+                                      size_t* bytes);
+int dsa_index_dense_host(const void* Q, const float* w, const void* K,
+                         const float* K_scale, int T, int N, int H, int d,
+                         int64_t q_pos0, int k, int q_dtype, int k_dtype,
+                         int chunk_rows, int32_t* idx, float* val,
+                         void* staging, size_t staging_bytes, void* stream);
+int dsa_index_group_host_staging_size(int T, int N, int H, int d, int k,
+                                      int group, int bank, int q_dtype,
+                                      int k_dtype, int chunk_rows,
+                                      size_t* bytes);
+int dsa_index_group_host(const void* Q, const float* w, const void* K,
+                         const float* K_scale, int T, int N, int H, int d,
+                         int64_t q_pos0, int k, int group, int bank, int mode,
+                         int q_dtype, int k_dtype, int chunk_rows,
+                         int32_t* idx, float* val, void* staging,
+                         size_t staging_bytes, void* stream);
+int dsa_index_decode_host_staging_size(int B, int total_q,
+                                       int64_t total_keys, int max_keys,
+                                       int H, int d, int k, int q_dtype,
+                                       int k_dtype, size_t* bytes);
+int dsa_index_decode_host(const void* Q, const float* w, const void* K,
+                          const float* K_scale, const int64_t* k_offsets,
+                          const int32_t* q_offsets, int B, int total_q,
+                          int64_t total_keys, int max_keys, int H, int d,
+                          int k, int q_dtype, int k_dtype, int32_t* idx,
+                          float* val, void* staging, size_t staging_bytes,
+                          void* stream);
 
 /* ------------------------------------------------------------------------
  * Test aid: the full score matrix S [T, N] fp32 of the dense call (the same

@@ -29,6 +29,12 @@ from ._binding import (  # noqa: F401
     IvfIndex,
     dsa_debug_scores,
     dsa_index_dense_static,
+    dsa_index_dense_host,
+    dsa_index_group_host,
+    dsa_index_decode_host,
+    dense_host_staging_bytes,
+    group_host_staging_bytes,
+    decode_host_staging_bytes,
     dsa_kernel_timer_start,
     dsa_kernel_timer_stop,
     dsa_check_status,

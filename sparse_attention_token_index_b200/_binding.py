@@ -76,6 +76,16 @@ _SIGS = {
                                         _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _c_sz, _vp]),
     "dsa_kernel_timer_stop": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int)]),
+    "dsa_index_dense_host_staging_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_dense_host": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                      _c_int, _c_int, _vp, _vp, _vp, _c_sz, _vp]),
+    "dsa_index_group_host_staging_size": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_group_host": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                      _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_sz, _vp]),
+    "dsa_index_decode_host_staging_size": (_c_int, [_c_int, _c_int, _c_i64] + [_c_int] * 6
+                                           + [ctypes.POINTER(_c_sz)]),
+    "dsa_index_decode_host": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _c_int,
+                                       _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_sz, _vp]),
 }
 
 
@@ -496,3 +506,122 @@ def dsa_kernel_timer_stop() -> Tuple[float, int]:
     ms, n = ctypes.c_float(0.0), _c_int(0)
     _check(lib().dsa_kernel_timer_stop(ctypes.byref(ms), ctypes.byref(n)), "dsa_kernel_timer_stop")
     return float(ms.value), int(n.value)
+
+
+# ---------------------------------------------------------------------------
+# host-buffer entry points: inputs and outputs in host memory (page-locked for
+# overlap), staged through a device buffer; synchronous
+# ---------------------------------------------------------------------------
+def _need_host(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if t.is_cuda:
+            raise ValueError("host-buffer call: tensors must be in host memory")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _host_outputs(rows: int, k: int, out):
+    if out is not None:
+        _need_host(*out)
+        return out
+    return (torch.empty((rows, k), dtype=torch.int32).pin_memory(),
+            torch.empty((rows, k), dtype=torch.float32).pin_memory())
+
+
+def _staging(nbytes: int, device, staging):
+    if staging is not None:
+        if not staging.is_cuda or staging.numel() * staging.element_size() < nbytes:
+            raise ValueError(f"staging must be a device buffer of at least {nbytes} bytes")
+        return staging
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+
+
+def dense_host_staging_bytes(T, N, H, d, k, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_dense_host_staging_size(T, N, H, d, k, q_dtype, k_dtype, ctypes.byref(n)),
+           "dsa_index_dense_host_staging_size")
+    return int(n.value)
+
+
+def group_host_staging_bytes(T, N, H, d, k, group, bank, q_dtype, k_dtype, chunk_rows=0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_group_host_staging_size(T, N, H, d, k, group, bank, q_dtype, k_dtype, chunk_rows,
+                                                   ctypes.byref(n)), "dsa_index_group_host_staging_size")
+    return int(n.value)
+
+
+def decode_host_staging_bytes(B, total_q, total_keys, max_keys, H, d, k, q_dtype, k_dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dsa_index_decode_host_staging_size(B, total_q, total_keys, max_keys, H, d, k, q_dtype, k_dtype,
+                                                    ctypes.byref(n)), "dsa_index_decode_host_staging_size")
+    return int(n.value)
+
+
+def dsa_index_dense_host(Q, w, K, k: int, q_pos0: Optional[int] = None, K_scale=None, out=None,
+                         chunk_rows: int = 0, staging=None, device=None, stream=None):
+    """Dense indexer on host tensors; returns host (idx [T,k], val [T,k]).
+
+    The inputs are copied in and the outputs out in row chunks that overlap
+    the indexer; ``staging`` is an optional device uint8 buffer of at least
+    ``dense_host_staging_bytes`` bytes.  Returns once the outputs are filled.
+    """
+    _need_host(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    st = _staging(dense_host_staging_bytes(T, N, H, d, k, qd, kd), device, staging)
+    idx, val = _host_outputs(T, k, out)
+    with torch.cuda.device(st.device):
+        _check(lib().dsa_index_dense_host(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, k, qd, kd,
+                                          int(chunk_rows), _ptr(idx), _ptr(val), _ptr(st), st.numel(),
+                                          _stream(stream)), "dsa_index_dense_host")
+    return idx, val
+
+
+def dsa_index_group_host(Q, w, K, k: int, group: int, bank: int, mode: int = DSA_GROUP_REFINE,
+                         q_pos0: Optional[int] = None, K_scale=None, out=None, chunk_rows: int = 0, staging=None,
+                         device=None, stream=None):
+    """Group-shared (PIVOT) indexer on host tensors; returns host (idx, val).
+
+    Chunks hold whole groups, so the results equal one call over all rows.
+    """
+    _need_host(Q, w, K, K_scale)
+    T, H, d = Q.shape
+    N = K.shape[0]
+    q_pos0 = N - T if q_pos0 is None else int(q_pos0)
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    st = _staging(group_host_staging_bytes(T, N, H, d, k, group, bank, qd, kd, int(chunk_rows)), device, staging)
+    idx, val = _host_outputs(T, k, out)
+    with torch.cuda.device(st.device):
+        _check(lib().dsa_index_group_host(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), T, N, H, d, q_pos0, k, group,
+                                          bank, mode, qd, kd, int(chunk_rows), _ptr(idx), _ptr(val), _ptr(st),
+                                          st.numel(), _stream(stream)), "dsa_index_group_host")
+    return idx, val
+
+
+def dsa_index_decode_host(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.Tensor,
+                          max_keys: Optional[int] = None, K_scale=None, out=None, staging=None, device=None,
+                          stream=None):
+    """Decode indexer on host tensors and host offsets ([B+1] int64 / int32);
+    returns host (idx [sum m_b, k], val) with key indices local to each
+    sequence."""
+    _need_host(Q, w, K, K_scale, k_offsets, q_offsets)
+    total_q, H, d = Q.shape
+    B = k_offsets.numel() - 1
+    ko = k_offsets.to(torch.int64).contiguous()
+    qo = q_offsets.to(torch.int32).contiguous()
+    total_keys = int(ko[-1])
+    if max_keys is None:
+        max_keys = int((ko[1:] - ko[:-1]).max())
+    qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
+    st = _staging(decode_host_staging_bytes(B, total_q, total_keys, max_keys, H, d, k, qd, kd), device, staging)
+    idx, val = _host_outputs(total_q, k, out)
+    with torch.cuda.device(st.device):
+        _check(lib().dsa_index_decode_host(_ptr(Q), _ptr(w), _ptr(K), _ptr(K_scale), _ptr(ko), _ptr(qo), B,
+                                           total_q, total_keys, int(max_keys), H, d, k, qd, kd, _ptr(idx), _ptr(val),
+                                           _ptr(st), st.numel(), _stream(stream)), "dsa_index_decode_host")
+    return idx, val
