@@ -37,6 +37,10 @@
  *     dsa_check_status clears the word again after reading it.
  *   - Return value: DSA_OK or a negative DSA_ERR_* code; on an error nothing
  *     has been launched.
+ *   - Empty calls are valid: no query rows (prefill T = 0; decode B = 0,
+ *     then total_q = total_keys = 0).  They check the shape arguments,
+ *     launch nothing, may pass NULL tensor pointers and return DSA_OK; their
+ *     workspace (or staging) size is 256 bytes.
  *   - Supported shapes: bf16 Q/K with H = 64, d = 128 run on the tcgen05
  *     tensor-core kernel; fp32 Q/K (any H <= 128, d <= 256, H*d <= 8192) and
  *     other bf16 / fp8-key shapes run on an exact fp32 CUDA-core kernel.

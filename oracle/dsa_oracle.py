@@ -193,13 +193,16 @@ def round_bf16(x):
 def proxy(q, w, G):
     """PIVOT proxy per group of G consecutive rows: the members' mean q and mean w.
 
-    A last group with fewer than G rows averages over its actual members.
-    Returns (qbar [ng, H, d], wbar [ng, H]) in float64.
+    A last group with fewer than G rows averages over its actual members;
+    no rows form no groups.  Returns (qbar [ng, H, d], wbar [ng, H]) in
+    float64.
     """
     q = np.asarray(q, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
     T = q.shape[0]
     ng = (T + G - 1) // G
+    if ng == 0:
+        return np.zeros((0,) + q.shape[1:]), np.zeros((0,) + w.shape[1:])
     qb = np.stack([q[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
     wb = np.stack([w[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
     return qb, wb

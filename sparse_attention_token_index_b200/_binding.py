@@ -30,6 +30,9 @@ EXPORTED_SYMBOLS = (
     "dsa_index_block_routed_workspace_size", "dsa_index_block_routed",
     "dsa_ivf_index_size", "dsa_ivf_build_workspace_size", "dsa_ivf_build",
     "dsa_index_ivf_routed_workspace_size", "dsa_index_ivf_routed",
+    "dsa_index_dense_host_staging_size", "dsa_index_dense_host",
+    "dsa_index_group_host_staging_size", "dsa_index_group_host",
+    "dsa_index_decode_host_staging_size", "dsa_index_decode_host",
 )
 
 
@@ -286,7 +289,7 @@ def _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys):
     if max_keys is None or total_keys is None:
         ko_host = k_offsets.to("cpu", torch.int64)
         if max_keys is None:
-            max_keys = int((ko_host[1:] - ko_host[:-1]).max())
+            max_keys = int((ko_host[1:] - ko_host[:-1]).max()) if ko_host.numel() > 1 else 0
         if total_keys is None:
             total_keys = int(ko_host[-1])
     ko = k_offsets if (k_offsets.is_cuda and k_offsets.dtype == torch.int64) else \
@@ -616,7 +619,7 @@ def dsa_index_decode_host(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: t
     qo = q_offsets.to(torch.int32).contiguous()
     total_keys = int(ko[-1])
     if max_keys is None:
-        max_keys = int((ko[1:] - ko[:-1]).max())
+        max_keys = int((ko[1:] - ko[:-1]).max()) if ko.numel() > 1 else 0
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     st = _staging(decode_host_staging_bytes(B, total_q, total_keys, max_keys, H, d, k, qd, kd), device, staging)
     idx, val = _host_outputs(total_q, k, out)

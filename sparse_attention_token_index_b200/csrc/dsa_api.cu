@@ -218,6 +218,33 @@ int run_dense_rows(const DeviceInfo& di, const DensePlan& p, const void* Q, cons
   return launch_simt_index(a, grid, st);
 }
 
+// Empty calls: no query rows (prefill T = 0, decode B = 0).  Nothing is
+// computed and nothing is launched; the shape arguments are still checked
+// and the workspace needs only its status word.
+constexpr size_t kEmptyWorkspaceBytes = 256;
+
+int empty_workspace(size_t* bytes) {
+  *bytes = kEmptyWorkspaceBytes;
+  return DSA_OK;
+}
+
+int empty_prefill(int N, int H, int d, int k, int q_dtype, int k_dtype, int64_t q_pos0) {
+  const int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  return (N < 0 || q_pos0 < 0 || q_pos0 > (int64_t)N) ? DSA_ERR_INVALID_ARG : DSA_OK;
+}
+
+int empty_decode(int total_q, int64_t total_keys, int H, int d, int k, int q_dtype, int k_dtype) {
+  const int r = check_common(H, d, k, q_dtype, k_dtype);
+  if (r != DSA_OK) return r;
+  return (total_q != 0 || total_keys != 0) ? DSA_ERR_INVALID_ARG : DSA_OK;
+}
+
+bool group_args_ok(int k, int group, int bank, int mode) {
+  return group >= 1 && bank >= k && bank <= 16384 &&
+         (mode == DSA_GROUP_REFINE || mode == DSA_GROUP_REUSE || mode == DSA_GROUP_REFINE_LOCAL);
+}
+
 int validate_dense(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
                    int64_t q_pos0, int k, int q_dtype, int k_dtype) {
   int r = check_common(H, d, k, q_dtype, k_dtype);
@@ -268,7 +295,9 @@ int dsa_index_dense_workspace_size(int T, int N, int H, int d, int k, int q_dtyp
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (T < 1 || N < 1) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || N < 0) return DSA_ERR_INVALID_ARG;
+  if (T == 0) return empty_workspace(bytes);
+  if (N < 1) return DSA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   Layout L;
@@ -280,6 +309,7 @@ int dsa_index_dense_workspace_size(int T, int N, int H, int d, int k, int q_dtyp
 int dsa_index_dense(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H, int d,
                     int64_t q_pos0, int k, int q_dtype, int k_dtype, int32_t* idx, float* val, void* workspace,
                     size_t workspace_bytes, void* stream) {
+  if (T == 0) return empty_prefill(N, H, d, k, q_dtype, k_dtype, q_pos0);
   int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
@@ -387,8 +417,10 @@ int dsa_index_group_workspace_size(int T, int N, int H, int d, int k, int group,
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (T < 1 || N < 1 || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || N < 0 || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return empty_workspace(bytes);
+  if (N < 1) return DSA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   GroupPlan gp;
@@ -401,6 +433,10 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
                     int64_t q_pos0, int k, int group, int bank, int mode, int q_dtype, int k_dtype, int32_t* idx,
                     float* val, int32_t* bank_idx, float* bank_val, void* proxy_q, float* proxy_w, void* workspace,
                     size_t workspace_bytes, void* stream) {
+  if (T == 0) {
+    if (!group_args_ok(k, group, bank, mode)) return DSA_ERR_INVALID_ARG;
+    return use_tc(H, d, q_dtype, k_dtype) ? empty_prefill(N, H, d, k, q_dtype, k_dtype, q_pos0) : DSA_ERR_UNSUPPORTED;
+  }
   int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!idx || !val || !workspace || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
@@ -587,7 +623,9 @@ int dsa_index_decode_workspace_size(int B, int total_q, int max_keys, int H, int
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (B < 1 || total_q < 1 || max_keys < 1) return DSA_ERR_INVALID_ARG;
+  if (B < 0 || total_q < 0 || max_keys < 0) return DSA_ERR_INVALID_ARG;
+  if (B == 0) return total_q == 0 ? empty_workspace(bytes) : DSA_ERR_INVALID_ARG;
+  if (total_q < 1 || max_keys < 1) return DSA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   DecodePlan p;
@@ -600,6 +638,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
                      const int32_t* q_offsets, int B, int total_q, int64_t total_keys, int max_keys, int H, int d,
                      int k, int q_dtype, int k_dtype, int32_t* idx, float* val, void* workspace,
                      size_t workspace_bytes, void* stream) {
+  if (B == 0) return empty_decode(total_q, total_keys, H, d, k, q_dtype, k_dtype);
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
@@ -698,8 +737,10 @@ int dsa_index_decode_group_workspace_size(int B, int total_q, int max_keys, int 
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (B < 1 || total_q < 1 || max_keys < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (B < 0 || total_q < 0 || max_keys < 0 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (B == 0) return total_q == 0 ? empty_workspace(bytes) : DSA_ERR_INVALID_ARG;
+  if (total_q < 1 || max_keys < 1) return DSA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   DecodeGroupPlan gp;
@@ -713,6 +754,11 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
                            int max_keys, int H, int d, int k, int bank, int mode, int q_dtype, int k_dtype,
                            int32_t* idx, float* val, int32_t* bank_idx, float* bank_val, void* proxy_q,
                            float* proxy_w, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B == 0) {
+    if (!group_args_ok(k, 1, bank, mode)) return DSA_ERR_INVALID_ARG;
+    if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+    return empty_decode(total_q, total_keys, H, d, k, q_dtype, k_dtype);
+  }
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
@@ -838,8 +884,10 @@ int dsa_index_block_routed_workspace_size(int T, int N, int H, int d, int k, int
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (T < 1 || N < 1 || n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || N < 0 || n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return empty_workspace(bytes);
+  if (N < 1) return DSA_ERR_INVALID_ARG;
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   RoutedPlan p;
@@ -852,6 +900,10 @@ int dsa_index_block_routed(const void* Q, const float* w, const void* K, const f
                            int d, int64_t q_pos0, int k, int n_blocks, int q_dtype, int k_dtype, int32_t* idx,
                            float* val, int32_t* block_idx, void* reps, void* workspace, size_t workspace_bytes,
                            void* stream) {
+  if (T == 0) {
+    if (n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
+    return use_tc(H, d, q_dtype, k_dtype) ? empty_prefill(N, H, d, k, q_dtype, k_dtype, q_pos0) : DSA_ERR_UNSUPPORTED;
+  }
   int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!idx || !val || !workspace || n_blocks < 1 || n_blocks > 65536) return DSA_ERR_INVALID_ARG;
@@ -991,8 +1043,9 @@ int dsa_index_ivf_routed_workspace_size(int T, int N, int H, int d, int k, int C
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (T < 1 || N < 1 || C < 1 || n_probe < 1 || n_probe > C || max_tiles < 1) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || N < 1 || C < 1 || n_probe < 1 || n_probe > C || max_tiles < 1) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return empty_workspace(bytes);
   DeviceInfo di;
   if ((r = device_info(di)) != DSA_OK) return r;
   IvfPlan p;
@@ -1005,6 +1058,10 @@ int dsa_index_ivf_routed(const void* Q, const float* w, const void* index, const
                          int H, int d, int64_t q_pos0, int k, int C, int n_probe, int max_tiles, int q_dtype,
                          int k_dtype, int32_t* idx, float* val, int32_t* cluster_idx, void* workspace,
                          size_t workspace_bytes, void* stream) {
+  if (T == 0) {
+    if (N < 1 || C < 1 || C > N || n_probe < 1 || n_probe > C || max_tiles < 1) return DSA_ERR_INVALID_ARG;
+    return use_tc(H, d, q_dtype, k_dtype) ? empty_prefill(N, H, d, k, q_dtype, k_dtype, q_pos0) : DSA_ERR_UNSUPPORTED;
+  }
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
   if (!Q || !w || !index || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;

@@ -168,6 +168,7 @@ int dsa_index_dense_host_staging_size(int T, int N, int H, int d, int k, int q_d
   size_t ws = 0;
   int r = dsa_index_dense_workspace_size(T, N, H, d, k, q_dtype, k_dtype, &ws);
   if (r != DSA_OK) return r;
+  if (T == 0) return (*bytes = ws, DSA_OK);  // empty call: the status word only
   Staging s;
   if ((r = prefill_staging(T, N, H, d, k, q_dtype, k_dtype, ws, s)) != DSA_OK) return r;
   *bytes = s.total;
@@ -177,6 +178,9 @@ int dsa_index_dense_host_staging_size(int T, int N, int H, int d, int k, int q_d
 int dsa_index_dense_host(const void* Q, const float* w, const void* K, const float* K_scale, int T, int N, int H,
                          int d, int64_t q_pos0, int k, int q_dtype, int k_dtype, int chunk_rows, int32_t* idx,
                          float* val, void* staging, size_t staging_bytes, void* stream) {
+  if (T == 0)  // no query rows: the device call checks the shape and launches nothing
+    return dsa_index_dense(nullptr, nullptr, nullptr, nullptr, 0, N, H, d, q_pos0, k, q_dtype, k_dtype, nullptr,
+                           nullptr, nullptr, 0, stream);
   if (!Q || !w || !K || !idx || !val || !staging || !aligned16(staging) || chunk_rows < 0) return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
   size_t ws = 0;
@@ -209,6 +213,7 @@ int dsa_index_group_host_staging_size(int T, int N, int H, int d, int k, int gro
   const int64_t per = chunk_rows_for(T, chunk_rows, group);
   int r = dsa_index_group_workspace_size((int)per, N, H, d, k, group, bank, q_dtype, k_dtype, &ws);
   if (r != DSA_OK) return r;
+  if (T == 0) return (*bytes = ws, DSA_OK);  // empty call: the status word only
   Staging s;
   if ((r = prefill_staging(T, N, H, d, k, q_dtype, k_dtype, ws, s)) != DSA_OK) return r;
   *bytes = s.total;
@@ -219,6 +224,9 @@ int dsa_index_group_host(const void* Q, const float* w, const void* K, const flo
                          int d, int64_t q_pos0, int k, int group, int bank, int mode, int q_dtype, int k_dtype,
                          int chunk_rows, int32_t* idx, float* val, void* staging, size_t staging_bytes,
                          void* stream) {
+  if (T == 0)
+    return dsa_index_group(nullptr, nullptr, nullptr, nullptr, 0, N, H, d, q_pos0, k, group, bank, mode, q_dtype,
+                           k_dtype, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, stream);
   if (!Q || !w || !K || !idx || !val || !staging || !aligned16(staging) || chunk_rows < 0 || group < 1)
     return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
@@ -252,12 +260,14 @@ int dsa_index_group_host(const void* Q, const float* w, const void* K, const flo
 
 int dsa_index_decode_host_staging_size(int B, int total_q, int64_t total_keys, int max_keys, int H, int d, int k,
                                        int q_dtype, int k_dtype, size_t* bytes) {
-  if (!bytes || B < 1 || total_q < 1 || total_keys < 1) return DSA_ERR_INVALID_ARG;
+  if (!bytes || B < 0 || total_q < 0 || total_keys < 0) return DSA_ERR_INVALID_ARG;
   const size_t qe = elem_size(q_dtype), ke = elem_size(k_dtype);
   if (!qe || !ke) return DSA_ERR_INVALID_ARG;
+  if (B == 0 && total_keys != 0) return DSA_ERR_INVALID_ARG;
   size_t ws = 0;
   int r = dsa_index_decode_workspace_size(B, total_q, max_keys, H, d, k, q_dtype, k_dtype, &ws);
   if (r != DSA_OK) return r;
+  if (B == 0) return (*bytes = ws, DSA_OK);  // empty call: the status word only
   size_t off = 0;
   off += up256((size_t)total_keys * d * ke);                                  // K
   off += k_dtype == DSA_DTYPE_FP8_E4M3 ? up256((size_t)total_keys * 4) : 0;    // K_scale
@@ -273,6 +283,9 @@ int dsa_index_decode_host(const void* Q, const float* w, const void* K, const fl
                           const int64_t* k_offsets, const int32_t* q_offsets, int B, int total_q,
                           int64_t total_keys, int max_keys, int H, int d, int k, int q_dtype, int k_dtype,
                           int32_t* idx, float* val, void* staging, size_t staging_bytes, void* stream) {
+  if (B == 0)
+    return dsa_index_decode(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, total_q, total_keys, max_keys, H,
+                            d, k, q_dtype, k_dtype, nullptr, nullptr, nullptr, 0, stream);
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !staging || !aligned16(staging))
     return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;

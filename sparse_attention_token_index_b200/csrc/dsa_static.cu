@@ -69,6 +69,10 @@ int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 
 extern "C" int dsa_index_dense_static(const void* Q, const float* w, const void* K, int T, int N, int H, int d,
                                       int64_t q_pos0, int k, int32_t* idx, float* val, void* stream) {
+  if (T == 0) {  // no query rows: nothing to compute, nothing launched
+    if (N < 0 || q_pos0 < 0 || q_pos0 > (int64_t)N || k < 1 || k > 65536) return DSA_ERR_INVALID_ARG;
+    return (H != 64 || d != 128) ? DSA_ERR_UNSUPPORTED : DSA_OK;
+  }
   if (!Q || !w || !K || !idx || !val) return DSA_ERR_INVALID_ARG;
   if (T < 1 || N < 1 || q_pos0 < 0 || q_pos0 + (int64_t)T > (int64_t)N || k < 1 || k > 65536)
     return DSA_ERR_INVALID_ARG;

@@ -119,3 +119,30 @@ def test_comparator_and_group_host_checks(L):
     gg = L.dsa_index_group
     assert gg(ok, ok, ok, None, 8, 8, 64, 128, 0, 4, 2, 8, 7, 0, 0, ok, ok, None, None, None, None, ok, 1 << 20,
               None) == -1
+
+
+def test_empty_calls_need_no_device(L):
+    # no query rows: the shape arguments are checked, nothing is launched, no
+    # device is touched, and NULL tensor pointers are accepted
+    n = ctypes.c_size_t(0)
+    assert L.dsa_index_dense_workspace_size(0, 10, 64, 128, 4, 0, 0, ctypes.byref(n)) == 0 and n.value == 256
+    assert L.dsa_index_dense(None, None, None, None, 0, 10, 64, 128, 10, 4, 0, 0, None, None, None, 0, None) == 0
+    assert L.dsa_index_dense(None, None, None, None, 0, 0, 64, 128, 0, 4, 0, 0, None, None, None, 0, None) == 0
+    assert L.dsa_index_group(None, None, None, None, 0, 10, 64, 128, 10, 4, 8, 16, 0, 0, 0, None, None, None, None,
+                             None, None, None, 0, None) == 0
+    assert L.dsa_index_decode(None, None, None, None, None, None, 0, 0, 0, 0, 64, 128, 4, 0, 0, None, None, None, 0,
+                              None) == 0
+    assert L.dsa_index_decode_group(None, None, None, None, None, None, 0, 0, 0, 0, 64, 128, 4, 16, 0, 0, 0, None,
+                                    None, None, None, None, None, None, 0, None) == 0
+    assert L.dsa_index_dense_static(None, None, None, 0, 10, 64, 128, 10, 4, None, None, None) == 0
+    assert L.dsa_index_dense_host(None, None, None, None, 0, 10, 64, 128, 10, 4, 0, 0, 0, None, None, None, 0,
+                                  None) == 0
+    assert L.dsa_index_decode_host(None, None, None, None, None, None, 0, 0, 0, 0, 64, 128, 4, 0, 0, None, None, None,
+                                   0, None) == 0
+    # still checked: k, q_pos0 against the keys, the group arguments, decode totals
+    assert L.dsa_index_dense(None, None, None, None, 0, 10, 64, 128, 10, 0, 0, 0, None, None, None, 0, None) == -1
+    assert L.dsa_index_dense(None, None, None, None, 0, 10, 64, 128, 11, 4, 0, 0, None, None, None, 0, None) == -1
+    assert L.dsa_index_group(None, None, None, None, 0, 10, 64, 128, 10, 16, 8, 8, 0, 0, 0, None, None, None, None,
+                             None, None, None, 0, None) == -1
+    assert L.dsa_index_decode(None, None, None, None, None, None, 0, 1, 0, 0, 64, 128, 4, 0, 0, None, None, None, 0,
+                              None) == -1
