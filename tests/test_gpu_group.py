@@ -10,7 +10,7 @@ import torch
 
 import sparse_attention_token_index_b200 as dsa
 from oracle import dsa_oracle as O
-from parity import check_row, RTOL, ATOL_FRAC
+from parity import check_row
 from synthetic import make_dense_inputs
 
 pytestmark = pytest.mark.gpu

@@ -7,7 +7,6 @@ cases, closed-form identities and invariants.  ``test_mutants_are_caught``
 plants plausible mistakes in the oracle (on the CPU) and requires that some pin
 fails for each.
 """
-import contextlib
 import itertools
 import json
 import math
