@@ -272,10 +272,15 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
         remaining -= above;
         prefix |= (uint64_t)dsel << shift;
         mask |= (uint64_t)0xFFu << shift;
-        if (in == remaining) break;  // the whole digit bucket is in: keys with (key & mask) >= prefix
+        // keys with (key & mask) >= prefix: the M - remaining already above
+        // this bucket plus the bucket itself.  Once they fit the sort buffer
+        // the digit steps can stop: the sort ranks the surplus below the top
+        // M, and members read the first M ranks only.
+        if (M - remaining + in <= PM) break;
       }
     }
-    // compact the top min(M, nvalid) keys (any order), then sort only them
+    // compact the keys at or above the prefix (at most PM, the top M among
+    // them; any order), then sort only them
     uint64_t* top = keys + P;
     if (tid == 0) sh_cnt = 0;
     __syncthreads();
