@@ -892,7 +892,8 @@ def main():
                 "traffic": None, "alg_per_launch": per_launch_bytes, "kernel_ms": avg_launch,
                 "note": f"algorithmic bytes = {wl.alg_bytes_note}; peak = {pk['src']} "
                         f"copy bandwidth; {scope}"}
-    roof["traffic"] = _traffic(args.config)
+    # the captures are of the workloads' own sizes: none applies to another --T
+    roof["traffic"] = _traffic(args.config) if args.T is None else None
 
     e2e = None
     if not args.no_e2e:
