@@ -739,9 +739,12 @@ def _kernel_source_hash():
     return kernel_source_hash(read)
 
 
-def _traffic(config):
+def _traffic(config, resized=False):
     """ncu DRAM bytes per scoring-kernel launch from profiles/, or None when
-    there is no capture for this workload or the kernel changed since."""
+    there is no capture for this workload, the kernel changed since, or the
+    run is resized (--T): the captures are of the workloads' own sizes."""
+    if resized:
+        return None
     p = os.path.join(ROOT, "profiles", f"{config}_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -892,8 +895,7 @@ def main():
                 "traffic": None, "alg_per_launch": per_launch_bytes, "kernel_ms": avg_launch,
                 "note": f"algorithmic bytes = {wl.alg_bytes_note}; peak = {pk['src']} "
                         f"copy bandwidth; {scope}"}
-    # the captures are of the workloads' own sizes: none applies to another --T
-    roof["traffic"] = _traffic(args.config) if args.T is None else None
+    roof["traffic"] = _traffic(args.config, resized=args.T is not None)
 
     e2e = None
     if not args.no_e2e:

@@ -42,3 +42,9 @@ def test_committed_traffic_matches_the_current_kernel():
     # the committed captures were taken on the current device code
     for cfg in ("dense_bf16_32k", "decode_bf16_32x128k", "group_bf16_128k_refine"):
         assert bench._traffic(cfg) is not None, cfg
+
+
+def test_no_traffic_for_a_resized_run():
+    # a capture of the full-size workload says nothing about a --T run
+    assert bench._traffic("dense_bf16_32k", resized=True) is None
+    assert bench._traffic("no_such_workload") is None
