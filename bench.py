@@ -641,7 +641,10 @@ WORKLOADS = {
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every 50 ms by NVML (reads only)."""
+    """SM clock and clock-event reasons sampled every 50 ms by NVML (reads only).
+
+    NVML is opened before the timed region and sampled once more when it
+    ends, so that a short timed region still has a clock record."""
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
 
@@ -653,22 +656,24 @@ class ClockSampler:
         self.max_mhz = None
         self._stop = threading.Event()
         self._thr = None
+        self._nvml = None
+        self._h = None
         self.err = None
+
+    def _sample(self):
+        N, h = self._nvml, self._h
+        self.samples.append(float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)))
+        r = int(N.nvmlDeviceGetCurrentClocksEventReasons(h))
+        for nm, bit in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(nm)
 
     def _run(self):
         try:
-            import pynvml as N
-            N.nvmlInit()
-            h = N.nvmlDeviceGetHandleByIndex(self.gpu)
-            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
-            while not self._stop.is_set():
-                self.samples.append(float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)))
-                r = int(N.nvmlDeviceGetCurrentClocksEventReasons(h))
-                for nm, bit in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(nm)
-                self._stop.wait(0.05)
-            N.nvmlShutdown()
+            while True:
+                self._sample()
+                if self._stop.wait(0.05):
+                    break
         except Exception as e:  # pragma: no cover - reported in the JSON line
             self.err = repr(e)
 
@@ -680,6 +685,16 @@ class ClockSampler:
                 self.gpu = int(vis.split(",")[self.gpu])
             except (ValueError, IndexError):
                 pass
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self._nvml = N
+            self._h = N.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = float(N.nvmlDeviceGetMaxClockInfo(self._h, N.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: the JSON line says why
+            self.err = repr(e)
+            self._nvml = None
+            return
         self._thr = threading.Thread(target=self._run, daemon=True)
         self._thr.start()
 
@@ -687,6 +702,12 @@ class ClockSampler:
         self._stop.set()
         if self._thr is not None:
             self._thr.join(timeout=5)
+        if self._nvml is not None:
+            try:
+                self._sample()  # the end of the timed region
+                self._nvml.nvmlShutdown()
+            except Exception as e:  # pragma: no cover
+                self.err = self.err or repr(e)
         out = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
                "samples": len(self.samples), "reasons": sorted(self.reasons), "source": "NVML, 50 ms"}
         if self.err:

@@ -48,3 +48,49 @@ def test_no_traffic_for_a_resized_run():
     # a capture of the full-size workload says nothing about a --T run
     assert bench._traffic("dense_bf16_32k", resized=True) is None
     assert bench._traffic("no_such_workload") is None
+
+
+class _FakeNvml:
+    """Reads only, like the sampler: a GPU at 1500 MHz of 1965 under the power cap."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self):
+        self.calls = []
+
+    def nvmlInit(self):
+        self.calls.append("init")
+
+    def nvmlShutdown(self):
+        self.calls.append("shutdown")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return 1500
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 | 0x1   # sw_power_cap, and a bit the sampler does not report
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    fake = _FakeNvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    c = bench.ClockSampler(0)
+    c.start()
+    out = c.stop()   # a timed region shorter than one interval still has samples
+    assert out["samples"] >= 1 and out["sm_mhz"] == 1500.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and "error" not in out
+    assert fake.calls == ["init", "shutdown"]
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", None)   # import fails
+    c = bench.ClockSampler(0)
+    c.start()
+    out = c.stop()
+    assert out["sm_mhz"] is None and out["samples"] == 0 and "error" in out
