@@ -50,6 +50,7 @@ def _f64(t):
 
 
 GROUP_OVERRIDE = None   # --group: group size of the group workloads
+SHARD = 0               # this rank's batch of the workload: seed = the workload's seed + SHARD
 BANK_OVERRIDE = None    # --bank: candidate bank of the group workloads
 
 
@@ -133,7 +134,8 @@ class Dense(Workload):
         self.cfg = dict(CONFIGS[self.name])
         if size:
             self.cfg["T"] = self.cfg["N"] = int(size)
-        self.inp = make_dense_inputs(self.name, device=device, T=self.cfg["T"], N=self.cfg["N"])
+        self.inp = make_dense_inputs(self.name, device=device, T=self.cfg["T"], N=self.cfg["N"],
+                                     seed=self.cfg["seed"] + SHARD)
         self.T, self.N, self.k = self.cfg["T"], self.cfg["N"], self.cfg["k"]
         q0 = self.inp.q_pos0
         self.pairs = self.alg_pairs = self.T * q0 + self.T * (self.T + 1) // 2
@@ -351,7 +353,8 @@ class Group(Workload):
         self.cfg = dict(CONFIGS[name])
         if size:
             self.cfg["T"] = self.cfg["N"] = int(size)
-        self.inp = make_dense_inputs(name, device=device, T=self.cfg["T"], N=self.cfg["N"])
+        self.inp = make_dense_inputs(name, device=device, T=self.cfg["T"], N=self.cfg["N"],
+                                     seed=self.cfg["seed"] + SHARD)
         c = self.cfg
         c["G"] = GROUP_OVERRIDE or c["G"]
         c["bank"] = BANK_OVERRIDE or c["bank"]
@@ -464,7 +467,8 @@ class Decode(Workload):
         if size:
             self.cfg["Nb"] = int(size)
         c = self.cfg
-        self.inp = make_decode_inputs(self.name, device=device, lengths=[c["Nb"]] * c["B"], m=c["m"])
+        self.inp = make_decode_inputs(self.name, device=device, lengths=[c["Nb"]] * c["B"], m=c["m"],
+                                      seed=c["seed"] + SHARD)
         self.k = c["k"]
         m = c["m"]
         self.pairs = self.alg_pairs = c["B"] * sum(c["Nb"] - m + j + 1 for j in range(m))
@@ -855,6 +859,9 @@ def main():
 
     dist, rank, world, local = _dist()
     torch.cuda.set_device(local)
+    # weak scaling: every rank indexes its own batch of the workload's shape
+    global SHARD
+    SHARD = rank
     import sparse_attention_token_index_b200 as dsa
     dsa.lib()
     wl = WORKLOADS[args.config]("cuda", args.T)
@@ -953,7 +960,8 @@ def main():
                 "rows_per_s": rows_s, "alg_pairs_per_s": alg_value * 1e9, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": wl.launches_per_step * args.steps, "clocks": clocks,
                 "launch_ms": {"min": min(per), "median": statistics.median(per), "max": max(per)}}
-        line["config"]["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+        line["config"]["parallelism"] = (f"dp{world}: rank r indexes its own batch (seed + r), no collective on "
+                                         f"the data path" if world > 1 else "single GPU")
         if hasattr(wl, "recall"):
             line["recall_vs_dense"] = recall
         print(json.dumps(line))

@@ -94,3 +94,14 @@ def test_clock_sampler_without_nvml(monkeypatch):
     c.start()
     out = c.stop()
     assert out["sm_mhz"] is None and out["samples"] == 0 and "error" in out
+
+
+def test_each_rank_indexes_its_own_batch(monkeypatch):
+    # weak scaling: rank r's inputs are the workload's shape from seed + r
+    a = bench.Dense("cpu", size=64)
+    monkeypatch.setattr(bench, "SHARD", 1)
+    b = bench.Dense("cpu", size=64)
+    assert a.inp.q.shape == b.inp.q.shape and not bool((a.inp.q == b.inp.q).all())
+    monkeypatch.setattr(bench, "SHARD", 0)
+    c = bench.Dense("cpu", size=64)
+    assert bool((a.inp.q == c.inp.q).all())
