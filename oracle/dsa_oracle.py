@@ -1,7 +1,7 @@
 """Plain CPU oracle for the DSA lightning indexer — TEST INFRASTRUCTURE ONLY.
 
-Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this module.  The product path (the CUDA library and
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline and
+reference legs of ``bench.py`` may import this module.  The product path (the CUDA library and
 its Python binding) never calls it, and it shares no code with that path.
 
 Everything here is slow and direct: float64 numpy, a full stable sort per
@@ -31,6 +31,17 @@ query row, no tiling and no fusion.  It follows the pages as follows.
   over the bank, restricted to keys the member may see, cut to k.
 * Decode (PIVOT abstract, MLI "Core Idea"): sequence b holds N_b cached keys
   and m_b new queries; new query j sits at position N_b - m_b + j.
+* Group form in decode (PIVOT abstract: the queries of one multi-token
+  prediction step are a natural group): a sequence's new queries are one
+  group.  Refine may also take each member's own stretch of the group as
+  query-specific candidates (ADIndex page, Inference).
+* Two-stage routing comparators (AttentionIndex page, Architecture): blocks
+  of 128 keys ranked by their mean key, and a plain k-means inverted file;
+  each followed by the native score on the routed keys.
+* Rounding.  Where the library stores a mean in bf16 (the proxy query, a
+  block's mean key), ``round_bf16`` rounds the float64 mean to nearest even,
+  so that the oracle can run those steps from scratch.
+* No query rows: nothing is selected; the group form has no groups.
 
 Pins: every function here is checked in ``tests/test_oracle.py`` against
 hand-worked values (``tests/golden/``), the fp8 format's published value
@@ -41,8 +52,9 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "decode_e4m3", "key_values", "score_rows", "select_topk", "dense",
-    "proxy", "group", "decode", "REFINE", "REUSE",
+    "decode_e4m3", "key_values", "score_rows", "select_topk", "dense", "round_bf16",
+    "proxy", "group", "decode", "decode_group", "block_reps", "block_routed", "kmeans", "ivf_routed",
+    "REFINE", "REUSE", "REFINE_LOCAL",
 ]
 
 REFINE = 0
