@@ -146,3 +146,33 @@ def test_empty_calls_need_no_device(L):
                              None, None, None, 0, None) == -1
     assert L.dsa_index_decode(None, None, None, None, None, None, 0, 1, 0, 0, 64, 128, 4, 0, 0, None, None, None, 0,
                               None) == -1
+
+
+def _declared_params():
+    """name -> list of parameter type strings, from the header's prototypes."""
+    out = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for m in re.finditer(r"(?:const\s+)?\w+\s*\*?\s*(dsa_\w+)\s*\(([^)]*)\)\s*;", txt):
+            params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+            out[m.group(1)] = params
+    return out
+
+
+def test_binding_prototypes_match_the_header():
+    # every ctypes prototype has the header's parameter count, and each
+    # pointer / 64-bit / 32-bit slot the matching ctypes kind
+    import ctypes as C
+    from sparse_attention_token_index_b200 import _binding as Bd
+    decl = _declared_params()
+    for name, (_, argtypes) in Bd._SIGS.items():
+        assert name in decl, name
+        params = decl[name]
+        assert len(params) == len(argtypes), (name, len(params), len(argtypes))
+        for p, t in zip(params, argtypes):
+            if "*" in p:
+                assert t in (C.c_void_p,) or issubclass(t, C._Pointer), (name, p, t)
+            elif re.match(r"(const\s+)?(int64_t|size_t)\b", p):
+                assert t in (C.c_int64, C.c_size_t), (name, p, t)
+            else:
+                assert t is C.c_int, (name, p, t)
