@@ -176,3 +176,41 @@ def test_binding_prototypes_match_the_header():
                 assert t in (C.c_int64, C.c_size_t), (name, p, t)
             else:
                 assert t is C.c_int, (name, p, t)
+
+
+def test_plain_c_program_links_and_calls(tmp_path, L):
+    # the header is C (not only C++), and a C program links against the
+    # library and calls it: version, status text, and empty calls (no device)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "dsa_index.h"
+int main(void) {
+  size_t n = 0;
+  if (dsa_version() != 100) return 1;
+  if (strcmp(dsa_status_string(DSA_ERR_INVALID_ARG), "invalid argument") != 0) return 2;
+  if (dsa_index_dense_workspace_size(0, 16, 64, 128, 8, DSA_DTYPE_BF16, DSA_DTYPE_BF16, &n) != DSA_OK || n != 256)
+    return 3;
+  if (dsa_index_dense(NULL, NULL, NULL, NULL, 0, 16, 64, 128, 16, 8, DSA_DTYPE_BF16, DSA_DTYPE_BF16, NULL, NULL,
+                      NULL, 0, NULL) != DSA_OK)
+    return 4;
+  if (dsa_index_dense(NULL, NULL, NULL, NULL, 0, 16, 64, 128, 16, 0, DSA_DTYPE_BF16, DSA_DTYPE_BF16, NULL, NULL,
+                      NULL, 0, NULL) != DSA_ERR_INVALID_ARG)
+    return 5;
+  puts("c abi ok");
+  return 0;
+}
+""")
+    lib = dsa.lib_path
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                        str(exe), lib, "-Wl,-rpath," + os.path.dirname(lib)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
