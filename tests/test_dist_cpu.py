@@ -1,10 +1,10 @@
 """Multi-rank plumbing of bench.py on CPU (gloo, world size 2).
 
-The indexer shards by independent rows and sequences, so N GPUs run N
-replicas with no data-path collective; what needs testing is the timing
-plumbing: every rank joins the same collectives, the slowest rank's time is
-the job's time, the whole-job rate counts every rank's units, and only rank 0
-of the reference arm does any work."""
+The indexer shards by independent rows and sequences, so each of N GPUs
+indexes its own batch with no data-path collective; what needs testing is
+the plumbing: every rank joins the same collectives, the slowest rank's time
+is the job's time, the whole-job rate counts every rank's units, the ranks'
+batches differ, and only rank 0 of the reference arm does any work."""
 import os
 import socket
 import sys
@@ -24,6 +24,7 @@ def _free_port():
 def _worker(rank, world, port, out):
     import datetime
 
+    import torch
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -43,8 +44,14 @@ def _worker(rank, world, port, out):
                 steps = 1
                 warmup = 3
             ref = bench.run_reference(A())
+        # each rank's own batch: a checksum of its queries, gathered
+        bench.SHARD = rank
+        wl = bench.Dense("cpu", size=64)
+        mine = torch.tensor([float(wl.inp.q.float().sum())], dtype=torch.float64)
+        sums = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(sums, mine)
         bench._barrier(dist)
-        out.put((rank, slowest, rate, ref))
+        out.put((rank, slowest, rate, ref, [float(x) for x in sums]))
     finally:
         dist.destroy_process_group()
 
@@ -60,8 +67,8 @@ def test_two_ranks_max_and_whole_job_rate():
     res = {}
     try:
         for _ in range(world):
-            r, slowest, rate, ref = q.get(timeout=120)
-            res[r] = (slowest, rate, ref)
+            r, slowest, rate, ref, sums = q.get(timeout=120)
+            res[r] = (slowest, rate, ref, sums)
     finally:
         for p in procs:
             p.join(timeout=60)
@@ -69,7 +76,8 @@ def test_two_ranks_max_and_whole_job_rate():
                 p.kill()
     assert all(p.exitcode == 0 for p in procs)
     for r in range(world):
-        slowest, rate, ref = res[r]
+        slowest, rate, ref, sums = res[r]
         assert slowest == pytest.approx(15.0)                  # max over ranks, seen by every rank
         assert rate == pytest.approx(1000 * 2 * 4 / 0.015)     # all ranks' units / slowest time
         assert ref is None
+        assert sums[0] != sums[1]                              # two ranks, two different batches
