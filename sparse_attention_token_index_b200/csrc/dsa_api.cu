@@ -241,7 +241,7 @@ int empty_decode(int total_q, int64_t total_keys, int H, int d, int k, int q_dty
 }
 
 bool group_args_ok(int k, int group, int bank, int mode) {
-  return group >= 1 && bank >= k && bank <= 16384 &&
+  return group >= 1 && bank >= k && bank <= kMaxBank &&
          (mode == DSA_GROUP_REFINE || mode == DSA_GROUP_REUSE || mode == DSA_GROUP_REFINE_LOCAL);
 }
 
@@ -417,7 +417,7 @@ int dsa_index_group_workspace_size(int T, int N, int H, int d, int k, int group,
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (T < 0 || N < 0 || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || N < 0 || group < 1 || bank < k || bank > kMaxBank) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
   if (T == 0) return empty_workspace(bytes);
   if (N < 1) return DSA_ERR_INVALID_ARG;
@@ -439,7 +439,7 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
   }
   int r = validate_dense(Q, w, K, K_scale, T, N, H, d, q_pos0, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (!idx || !val || !workspace || group < 1 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (!idx || !val || !workspace || group < 1 || bank < k || bank > kMaxBank) return DSA_ERR_INVALID_ARG;
   if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE && mode != DSA_GROUP_REFINE_LOCAL)
     return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
@@ -737,7 +737,7 @@ int dsa_index_decode_group_workspace_size(int B, int total_q, int max_keys, int 
   if (!bytes) return DSA_ERR_INVALID_ARG;
   int r = check_common(H, d, k, q_dtype, k_dtype);
   if (r != DSA_OK) return r;
-  if (B < 0 || total_q < 0 || max_keys < 0 || bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (B < 0 || total_q < 0 || max_keys < 0 || bank < k || bank > kMaxBank) return DSA_ERR_INVALID_ARG;
   if (!use_tc(H, d, q_dtype, k_dtype)) return DSA_ERR_UNSUPPORTED;
   if (B == 0) return total_q == 0 ? empty_workspace(bytes) : DSA_ERR_INVALID_ARG;
   if (total_q < 1 || max_keys < 1) return DSA_ERR_INVALID_ARG;
@@ -763,7 +763,7 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   if (r != DSA_OK) return r;
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !workspace) return DSA_ERR_INVALID_ARG;
   if (B < 1 || total_q < 1 || max_keys < 1 || total_keys < 1 || max_keys > total_keys) return DSA_ERR_INVALID_ARG;
-  if (bank < k || bank > 16384) return DSA_ERR_INVALID_ARG;
+  if (bank < k || bank > kMaxBank) return DSA_ERR_INVALID_ARG;
   if (mode != DSA_GROUP_REFINE && mode != DSA_GROUP_REUSE && mode != DSA_GROUP_REFINE_LOCAL)
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(w)) return DSA_ERR_INVALID_ARG;

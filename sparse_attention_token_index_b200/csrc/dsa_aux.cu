@@ -363,7 +363,7 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
                            const int32_t* q_off, const int64_t* k_off) {
   int P = 1;
   while (P < bank_size) P <<= 1;
-  if (P > 16384) return DSA_ERR_UNSUPPORTED;
+  if (P > kMaxBank) return DSA_ERR_UNSUPPORTED;
   int M = bank_size, PM = 0;
   if (!rank_all) {
     const int64_t m = (int64_t)k + G - 1;

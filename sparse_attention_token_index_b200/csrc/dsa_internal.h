@@ -7,6 +7,10 @@
 
 namespace dsa {
 
+// Largest candidate bank of the group form: the bank ranking holds a whole
+// bank in shared memory (8 bytes per key, 128 KB at this size).
+constexpr int kMaxBank = 16384;
+
 // Arguments of the tensor-core kernel (see dsa_tc.cu).
 //   kind 0: prefill rows.  Row r of Q sits at position
 //           pos_base + min(r * pos_mul + pos_add, pos_clamp) and sees keys
