@@ -180,12 +180,19 @@ def dsa_check_status(workspace: torch.Tensor, stream=None) -> None:
     _check(lib().dsa_check_status(_ptr(workspace), _stream(stream)), "device status")
 
 
+def _check_out(idx, val, rows, k):
+    # the library writes rows * k entries into each: a smaller buffer would overflow
+    if idx.dtype != torch.int32 or val.dtype != torch.float32:
+        raise TypeError("out must be (int32 idx, float32 val)")
+    if tuple(idx.shape) != (rows, k) or tuple(val.shape) != (rows, k):
+        raise ValueError(f"out must be two [{rows}, {k}] tensors")
+
+
 def _outputs(rows, k, device, out):
     if out is not None:
         idx, val = out
         _need_cuda(idx, val)
-        assert idx.dtype == torch.int32 and val.dtype == torch.float32
-        assert idx.shape == (rows, k) and val.shape == (rows, k)
+        _check_out(idx, val, rows, k)
         return idx, val
     return (torch.empty((rows, k), dtype=torch.int32, device=device),
             torch.empty((rows, k), dtype=torch.float32, device=device))
@@ -528,6 +535,7 @@ def _need_host(*ts):
 def _host_outputs(rows: int, k: int, out):
     if out is not None:
         _need_host(*out)
+        _check_out(out[0], out[1], rows, k)
         return out
     return (torch.empty((rows, k), dtype=torch.int32).pin_memory(),
             torch.empty((rows, k), dtype=torch.float32).pin_memory())

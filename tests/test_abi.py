@@ -214,3 +214,15 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+
+
+def test_binding_rejects_wrong_output_buffers():
+    # caller-supplied outputs are checked before the library could write past them
+    import torch
+    from sparse_attention_token_index_b200 import _binding as Bd
+    ok = (torch.empty((4, 8), dtype=torch.int32), torch.empty((4, 8), dtype=torch.float32))
+    assert Bd._host_outputs(4, 8, ok) is ok
+    with pytest.raises(ValueError):
+        Bd._host_outputs(4, 8, (torch.empty((4, 7), dtype=torch.int32), torch.empty((4, 8), dtype=torch.float32)))
+    with pytest.raises(TypeError):
+        Bd._host_outputs(4, 8, (torch.empty((4, 8), dtype=torch.int64), torch.empty((4, 8), dtype=torch.float32)))
