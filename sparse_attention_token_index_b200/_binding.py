@@ -127,6 +127,26 @@ def _dtype_code(t: torch.Tensor, allow_fp8=False) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _check_shapes(Q=None, w=None, K=None, K_scale=None, n_keys=None):
+    """Shapes the library relies on but cannot see through its pointers: a
+    mismatch would make it read past a buffer.  Q [T, H, d]; w float32
+    [T, H]; K [N, d]; K_scale float32 [N] (N = K's rows, or n_keys)."""
+    d = None
+    if Q is not None:
+        if Q.dim() != 3:
+            raise ValueError("Q must be [T, H, d]")
+        T, H, d = Q.shape
+        if w is None or w.dtype != torch.float32 or tuple(w.shape) != (T, H):
+            raise ValueError(f"w must be float32 [{T}, {H}]")
+    if K is not None:
+        if K.dim() != 2 or (d is not None and K.shape[1] != d):
+            raise ValueError(f"K must be [N, {d if d is not None else 'd'}]")
+        n_keys = K.shape[0]
+    if K_scale is not None:
+        if K_scale.dtype != torch.float32 or tuple(K_scale.shape) != (n_keys,):
+            raise ValueError(f"K_scale must be float32 [{n_keys}]")
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is None:
@@ -207,6 +227,7 @@ def dsa_index_dense(Q: torch.Tensor, w: torch.Tensor, K: torch.Tensor, k: int, q
     (then ``K_scale`` [N] fp32).  Returns (idx [T,k] int32, val [T,k] fp32);
     each row is a set, padded with -1 / -inf.
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -230,6 +251,7 @@ def dsa_index_group(Q, w, K, k: int, group: int, bank: int, mode: int = DSA_GROU
     Returns (idx, val) and, on request, (bank_idx [ng,B], bank_val [ng,B]) in
     the proxy's ranking order and (proxy_q [ng,H,d], proxy_w [ng,H]).
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -269,6 +291,7 @@ def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.
     synchronisation).  Returns (idx [sum m_b, k], val) with key indices
     local to each sequence.
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
@@ -293,6 +316,8 @@ def decode_group_workspace_bytes(B, total_q, max_keys, H, d, k, bank, q_dtype, k
 
 
 def _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys):
+    if k_offsets.numel() != q_offsets.numel() or k_offsets.numel() < 1:
+        raise ValueError("k_offsets and q_offsets must both be [B+1]")
     if max_keys is None or total_keys is None:
         ko_host = k_offsets.to("cpu", torch.int64)
         if max_keys is None:
@@ -316,6 +341,7 @@ def dsa_index_decode_group(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: 
     on request, (bank_idx [B, bank], bank_val) in the proxy's ranking order
     and (proxy_q [B, H, d], proxy_w [B, H]).
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
@@ -360,6 +386,7 @@ def dsa_index_block_routed(Q, w, K, k: int, n_blocks: int, q_pos0: Optional[int]
     Returns (idx, val) and, on request, the routed blocks [T, n_blocks] and
     the block representatives [ceil(N/128), d] (bf16).
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -421,6 +448,7 @@ class IvfIndex:
 
 def dsa_ivf_build(K, C: int, iters: int = 10, K_scale=None, stream=None, check: bool = False) -> IvfIndex:
     """Plain k-means index of the keys (Lloyd, `iters` iterations) for inverted-file routing."""
+    _check_shapes(None, None, K, K_scale)
     _need_cuda(K, K_scale)
     N, d = K.shape
     kd = _dtype_code(K, allow_fp8=True)
@@ -449,6 +477,7 @@ def dsa_index_ivf_routed(Q, w, index: IvfIndex, k: int, n_probe: int, q_pos0: Op
                          max_tiles: Optional[int] = None, out=None, return_clusters: bool = False, workspace=None,
                          stream=None, check: bool = False):
     """Inverted-file routing over `index`, then the native score on the probed clusters' keys."""
+    _check_shapes(Q, w, None, K_scale, index.N)
     _need_cuda(Q, w, K_scale)
     T, H, d = Q.shape
     N, C = index.N, index.C
@@ -470,6 +499,7 @@ def dsa_index_ivf_routed(Q, w, index: IvfIndex, k: int, n_probe: int, q_pos0: Op
 def dsa_debug_scores(Q, w, K, q_pos0: Optional[int] = None, K_scale=None, workspace=None, stream=None,
                      check: bool = False) -> torch.Tensor:
     """Test aid: the full [T, N] score matrix of the dense kernels (-inf beyond each prefix)."""
+    _check_shapes(Q, w, K, K_scale)
     _need_cuda(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -494,6 +524,7 @@ def dsa_index_dense_static(Q: torch.Tensor, w: torch.Tensor, K: torch.Tensor, k:
     overlap.  ``out`` = (idx, val) preallocated by the caller, else
     allocated here (by torch, outside the library).
     """
+    _check_shapes(Q, w, K)
     _need_cuda(Q, w, K)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -579,6 +610,7 @@ def dsa_index_dense_host(Q, w, K, k: int, q_pos0: Optional[int] = None, K_scale=
     the indexer; ``staging`` is an optional device uint8 buffer of at least
     ``dense_host_staging_bytes`` bytes.  Returns once the outputs are filled.
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_host(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -600,6 +632,7 @@ def dsa_index_group_host(Q, w, K, k: int, group: int, bank: int, mode: int = DSA
 
     Chunks hold whole groups, so the results equal one call over all rows.
     """
+    _check_shapes(Q, w, K, K_scale)
     _need_host(Q, w, K, K_scale)
     T, H, d = Q.shape
     N = K.shape[0]
@@ -620,7 +653,10 @@ def dsa_index_decode_host(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: t
     """Decode indexer on host tensors and host offsets ([B+1] int64 / int32);
     returns host (idx [sum m_b, k], val) with key indices local to each
     sequence."""
+    _check_shapes(Q, w, K, K_scale)
     _need_host(Q, w, K, K_scale, k_offsets, q_offsets)
+    if k_offsets.numel() != q_offsets.numel() or k_offsets.numel() < 1:
+        raise ValueError("k_offsets and q_offsets must both be [B+1]")
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
     ko = k_offsets.to(torch.int64).contiguous()

@@ -226,3 +226,21 @@ def test_binding_rejects_wrong_output_buffers():
         Bd._host_outputs(4, 8, (torch.empty((4, 7), dtype=torch.int32), torch.empty((4, 8), dtype=torch.float32)))
     with pytest.raises(TypeError):
         Bd._host_outputs(4, 8, (torch.empty((4, 8), dtype=torch.int64), torch.empty((4, 8), dtype=torch.float32)))
+
+
+def test_binding_rejects_mismatched_shapes_before_any_call():
+    # shapes the library cannot see through its pointers are checked first
+    import torch
+    q = torch.zeros((4, 64, 128), dtype=torch.bfloat16)
+    w = torch.zeros((4, 64), dtype=torch.float32)
+    K = torch.zeros((16, 128), dtype=torch.bfloat16)
+    for args, kw in [((q, w[:, :32], K, 2), {}),                       # w not [T, H]
+                     ((q, w.double(), K, 2), {}),                      # w not float32
+                     ((q, w, K[:, :64], 2), {}),                       # K not [N, d]
+                     ((q, w, K.to(torch.uint8), 2), {"K_scale": torch.zeros(15)})]:  # scales not [N]
+        with pytest.raises(ValueError):
+            dsa.dsa_index_dense(*args, **kw)
+        with pytest.raises(ValueError):
+            dsa.dsa_index_dense_host(*args, **kw)
+    with pytest.raises(ValueError):
+        dsa.dsa_index_decode_host(q, w, K, 2, torch.tensor([0, 8, 16]), torch.tensor([0, 4]))
