@@ -306,6 +306,27 @@ def pin_decode_group_invariants(O):
             assert np.array_equal(rf["idx"][last], dec["idx"][last]), b
             assert np.array_equal(ru["idx"][last], dec["idx"][last]), b
             assert np.allclose(ru["val"][last], dec["val"][last], rtol=1e-12), b
+    # Refine with local additions: a bank as large as every cache gives the
+    # decode indexer; with a small bank each query's candidates are the bank
+    # plus its sequence's new keys up to its own position, so its selection is
+    # causal, never worse than plain Refine, and the top-k of those candidates
+    rl_full = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE_LOCAL)
+    assert np.array_equal(rl_full["idx"], dec["idx"]) and np.array_equal(rl_full["val"], dec["val"])
+    rl = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE_LOCAL)
+    for b in range(4):
+        nb, mb = lengths[b], ms[b]
+        Kb = K[ko[b]:ko[b + 1]]
+        bank = rl["bank_idx"][b]
+        for j in range(mb):
+            r, p = qo[b] + j, nb - mb + j
+            n = rl["count"][r]
+            sel = rl["idx"][r][:n]
+            assert np.all(sel <= p), (b, j)
+            S = O.score_rows(q[r:r + 1], w[r:r + 1], Kb[:p + 1])[0]
+            assert S[sel].min() >= S[rf["idx"][r][:rf["count"][r]]].min() - 1e-15, (b, j)
+            cand = np.union1d(bank[bank <= p], np.arange(nb - mb, p + 1))
+            oi, _ = O.select_topk(S[cand], k, idx=cand)
+            assert np.array_equal(sel, oi), (b, j)
 
 
 def pin_group_local_hand(O):
