@@ -451,7 +451,8 @@ class Group(Workload):
             g = int(rng.integers(0, ng))
             r0, r1 = g * self.G, min(self.T, (g + 1) * self.G)
             O.group(_f64(i.q[r0:r1]), _f64(i.w[r0:r1]), K[:i.q_pos0 + r1], self.k, self.G, self.B, self.mode,
-                    q_pos0=i.q_pos0 + r0, k_scale=None if ks is None else ks[:i.q_pos0 + r1])
+                    q_pos0=i.q_pos0 + r0, k_scale=None if ks is None else ks[:i.q_pos0 + r1],
+                    q_dtype=self.cfg["q_dtype"])
             return sum(i.q_pos0 + t + 1 for t in range(r0, r1))
         return self._oracle_loop(budget_s, one)
 
@@ -617,7 +618,7 @@ class DecodeGroup(Decode):
             b = int(rng.integers(0, c["B"]))
             K = _f64(i.k[b * nb:(b + 1) * nb])
             O.decode_group(_f64(i.q[b * m:(b + 1) * m]), _f64(i.w[b * m:(b + 1) * m]), K, [0, nb], [0, m],
-                           self.k, self.bank, self.mode)
+                           self.k, self.bank, self.mode, q_dtype=c["q_dtype"])
             return sum(nb - m + j + 1 for j in range(m))
         return self._oracle_loop(budget_s, one)
 

@@ -38,9 +38,11 @@ query row, no tiling and no fusion.  It follows the pages as follows.
 * Two-stage routing comparators (AttentionIndex page, Architecture): blocks
   of 128 keys ranked by their mean key, and a plain k-means inverted file;
   each followed by the native score on the routed keys.
-* Rounding.  Where the library stores a mean in bf16 (the proxy query, a
-  block's mean key), ``round_bf16`` rounds the float64 mean to nearest even,
-  so that the oracle can run those steps from scratch.
+* Rounding.  The proxy query is stored in the queries' own dtype, so the
+  group form rounds the float64 member mean to that dtype (``round_q``; a
+  required ``q_dtype`` argument of ``proxy``, ``group`` and ``decode_group``).
+  A block's mean key is stored in bf16; ``round_bf16`` rounds to nearest
+  even, so that the oracle can run those steps from scratch.
 * No query rows: nothing is selected; the group form has no groups.
 
 Pins: every function here is checked in ``tests/test_oracle.py`` against
@@ -52,7 +54,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "decode_e4m3", "key_values", "score_rows", "select_topk", "dense", "round_bf16",
+    "decode_e4m3", "key_values", "score_rows", "select_topk", "dense", "round_bf16", "round_q",
     "proxy", "group", "decode", "decode_group", "block_reps", "block_routed", "kmeans", "ivf_routed",
     "REFINE", "REUSE", "REFINE_LOCAL",
 ]
@@ -202,12 +204,29 @@ def round_bf16(x):
     return out
 
 
-def proxy(q, w, G):
+def round_q(x, q_dtype):
+    """The proxy query as the library stores it: the float64 mean rounded to
+    the query's own dtype ("bf16": nearest bfloat16, ties to even; "fp32":
+    nearest float32; "f64": kept as is).  The PIVOT abstract says only that a
+    group is aggregated into one proxy query; this library keeps that query
+    in the dtype of the queries it aggregates, so the proxy scan runs on the
+    same arithmetic as every other scan."""
+    if q_dtype == "bf16":
+        return round_bf16(x)
+    if q_dtype == "fp32":
+        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+    if q_dtype == "f64":
+        return np.asarray(x, dtype=np.float64)
+    raise ValueError(f"q_dtype must be 'bf16', 'fp32' or 'f64', not {q_dtype!r}")
+
+
+def proxy(q, w, G, *, q_dtype):
     """PIVOT proxy per group of G consecutive rows: the members' mean q and mean w.
 
     A last group with fewer than G rows averages over its actual members;
-    no rows form no groups.  Returns (qbar [ng, H, d], wbar [ng, H]) in
-    float64.
+    no rows form no groups.  The mean q is rounded to ``q_dtype`` (see
+    ``round_q``); the mean w stays float64.  Returns (qbar [ng, H, d],
+    wbar [ng, H]).
     """
     q = np.asarray(q, dtype=np.float64)
     w = np.asarray(w, dtype=np.float64)
@@ -217,11 +236,11 @@ def proxy(q, w, G):
         return np.zeros((0,) + q.shape[1:]), np.zeros((0,) + w.shape[1:])
     qb = np.stack([q[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
     wb = np.stack([w[g * G:min(T, (g + 1) * G)].mean(axis=0) for g in range(ng)])
-    return qb, wb
+    return round_q(qb, q_dtype), wb
 
 
 def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=None,
-          groups=None, members=None, bank_override=None):
+          groups=None, members=None, bank_override=None, *, q_dtype):
     """PIVOT group-shared indexer (Refine or Reuse).
 
     For group g (rows gG..min(T,(g+1)G)-1) with last member position L_g:
@@ -238,8 +257,10 @@ def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=Non
          keys at positions p_first .. p_t (p_first = the group's first
          member), recent keys that the shared proxy may rank low.
 
-    ``qbar``/``wbar`` default to ``proxy(q, w, G)``; a caller may pass the
-    proxy exactly as another implementation rounded it.  ``groups`` restricts
+    ``q_dtype`` is the dtype the queries came in ("bf16", "fp32"; "f64" for
+    hand-worked float64 cases): the proxy query is the member mean rounded to
+    it (``proxy``).  ``qbar``/``wbar`` replace ``proxy(q, w, G, q_dtype)``,
+    e.g. with the proxy exactly as another implementation rounded it.  ``groups`` restricts
     the work to some groups; ``members`` (list of row indices) to some rows.
     ``bank_override`` {g: bank index array in proxy order} replaces step 1-2.
     Returns dict with ``bank_idx``/``bank_val`` {g: arrays in proxy order},
@@ -253,7 +274,7 @@ def group(q, w, K, k, G, bank, mode, q_pos0=0, k_scale=None, qbar=None, wbar=Non
     T = q.shape[0]
     ng = (T + G - 1) // G
     if qbar is None or wbar is None:
-        qb, wb = proxy(q, w, G)
+        qb, wb = proxy(q, w, G, q_dtype=q_dtype)
         qbar = qb if qbar is None else qbar
         wbar = wb if wbar is None else wbar
     qbar = np.asarray(qbar, dtype=np.float64)
@@ -337,7 +358,7 @@ def decode(q, w, K, k_offsets, q_offsets, k, k_scale=None, return_scores=False):
 
 
 def decode_group(q, w, K, k_offsets, q_offsets, k, bank, mode, k_scale=None, qbar=None, wbar=None,
-                 bank_override=None):
+                 bank_override=None, *, q_dtype):
     """PIVOT in decode: the new queries of one sequence form the group.
 
     The PIVOT abstract names the queries decoded together in one
@@ -349,8 +370,9 @@ def decode_group(q, w, K, k_offsets, q_offsets, k, bank, mode, k_scale=None, qba
     the proxy's top-`bank`, and every query refines or reuses exactly as in
     ``group``.  Indices are local to the sequence.
 
-    ``qbar`` [B, H, d] / ``wbar`` [B, H] replace the float64 means (a proxy as
-    another implementation rounded it); ``bank_override`` {b: bank indices}
+    ``q_dtype`` rounds the proxy query as in ``group``.  ``qbar`` [B, H, d] /
+    ``wbar`` [B, H] replace the proxy (e.g. as another implementation rounded
+    it); ``bank_override`` {b: bank indices}
     replaces the proxy's bank.  Returns idx/val/count over all query rows and
     bank_idx/bank_val/bank_scores {b: ...}.
     """
@@ -375,7 +397,7 @@ def decode_group(q, w, K, k_offsets, q_offsets, k, bank, mode, k_scale=None, qba
                   qbar=None if qbar is None else np.asarray(qbar)[b:b + 1],
                   wbar=None if wbar is None else np.asarray(wbar)[b:b + 1],
                   bank_override=None if bank_override is None or b not in bank_override
-                  else {0: bank_override[b]})
+                  else {0: bank_override[b]}, q_dtype=q_dtype)
         res["bank_idx"][b], res["bank_val"][b] = r["bank_idx"][0], r["bank_val"][0]
         res["bank_scores"][b] = r["bank_scores"][0]
         for j in range(mb):

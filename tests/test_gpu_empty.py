@@ -45,7 +45,8 @@ def test_group_empty(mode):
     q, w = _empty_q()
     idx, val = dsa.dsa_index_group(q, w, K, 16, 8, 64, mode=mode, q_pos0=300, check=True)
     assert idx.shape == (0, 16)
-    ref = O.group(np.zeros((0, H, D)), np.zeros((0, H)), K.cpu().double().numpy(), 16, 8, 64, mode, q_pos0=300)
+    ref = O.group(np.zeros((0, H, D)), np.zeros((0, H)), K.cpu().double().numpy(), 16, 8, 64, mode, q_pos0=300,
+                  q_dtype="bf16")
     assert len(ref["idx"]) == 0 and len(ref["bank_idx"]) == 0
 
 

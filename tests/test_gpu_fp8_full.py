@@ -54,9 +54,9 @@ def test_fp8_group_full_size_sampled(inp, keys, mode):
     for g in (0, 1000, T // G - 1):
         r0, r1 = g * G, min(T, (g + 1) * G)
         q, w = _f64(inp.q[r0:r1]), _f64(inp.w[r0:r1])
-        qb, wb = O.proxy(q, w, G)
+        qb, wb = O.proxy(q, w, G, q_dtype="bf16")
         L = inp.q_pos0 + r1 - 1
-        ps = O.score_rows(O.round_bf16(qb), wb, keys[:L + 1])[0]
+        ps = O.score_rows(qb, wb, keys[:L + 1])[0]
         bi, bv = bidx[g].cpu().numpy(), bval[g].cpu().numpy()
         check_row(bi, bv, ps, BANK, what=f"fp8 256K bank g={g}")
         bank = bi[bi >= 0].astype(np.int64)

@@ -37,11 +37,12 @@ def _check_group(inp, k, G, B, mode, what):
     T = q.shape[0]
     ng = (T + G - 1) // G
     # proxy: GPU bf16 rounding of the fp32 mean within one ulp of the fp64 mean
-    qb, wb = O.proxy(q, w, G)
+    # the unrounded float64 means, to bound the GPU's fp32 mean + bf16 rounding
+    qb, wb = O.proxy(q, w, G, q_dtype="f64")
     gq, gw = _f64(pq), _f64(pw)
     assert np.all(np.abs(gq - qb) <= _bf16_ulp(qb) + 1e-30), f"{what}: proxy q off by more than 1 bf16 ulp"
     assert np.allclose(gw, wb, rtol=1e-6, atol=1e-7), f"{what}: proxy w"
-    res = O.group(q, w, K, k, G, B, O.REFINE, q_pos0=inp.q_pos0, qbar=gq, wbar=gw)
+    res = O.group(q, w, K, k, G, B, O.REFINE, q_pos0=inp.q_pos0, qbar=gq, wbar=gw, q_dtype="bf16")
     bi, bv = bidx.cpu().numpy(), bval.cpu().numpy()
     gi, gv = idx.cpu().numpy(), val.cpu().numpy()
     for g in range(ng):

@@ -78,8 +78,7 @@ def test_group_host_chunks(mode):
     idx, val = dsa.dsa_index_group_host(_host(inp.q), _host(inp.w), _host(inp.k), k, G, B, mode=mode,
                                         q_pos0=inp.q_pos0, chunk_rows=100)
     q, w, K = _f64(inp.q), _f64(inp.w), _f64(inp.k)
-    qb, wb = O.proxy(q, w, G)
-    res = O.group(q, w, K, k, G, B, mode, q_pos0=inp.q_pos0, qbar=O.round_bf16(qb), wbar=wb)
+    res = O.group(q, w, K, k, G, B, mode, q_pos0=inp.q_pos0, q_dtype="bf16")
     gi, gv = idx.numpy(), val.numpy()
     for g in range(640 // G):
         bank = res["bank_idx"][g].astype(np.int64)

@@ -1,6 +1,7 @@
 """End-to-end parity with the oracle run entirely on its own: it forms its
-own proxies and block representatives (float64 means rounded to bf16 by
-its own round-to-nearest-even), its own banks and routed blocks, and the GPU's outputs are
+own proxies (float64 member means, rounded by the oracle to the queries'
+bf16) and block representatives (float64 means rounded to bf16 by its own
+round-to-nearest-even), its own banks and routed blocks, and the GPU's outputs are
 compared with those.  No GPU intermediate enters the oracle here (the other
 group tests also check each GPU stage on the GPU's previous stage, which
 isolates a failing stage)."""
@@ -28,8 +29,7 @@ def test_group_end_to_end(mode):
     idx, val, bi, bv = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0,
                                            return_bank=True, check=True)
     q, w, K = _f64(inp.q), _f64(inp.w), _f64(inp.k)
-    qb, wb = O.proxy(q, w, G)
-    res = O.group(q, w, K, k, G, B, mode, q_pos0=inp.q_pos0, qbar=O.round_bf16(qb), wbar=wb)
+    res = O.group(q, w, K, k, G, B, mode, q_pos0=inp.q_pos0, q_dtype="bf16")
     bi, bv, gi, gv = bi.cpu().numpy(), bv.cpu().numpy(), idx.cpu().numpy(), val.cpu().numpy()
     for g in range(q.shape[0] // G):
         ps = res["bank_scores"][g]
@@ -55,9 +55,7 @@ def test_decode_group_end_to_end(mode):
                                           check=True)
     q, w, K = _f64(inp.q), _f64(inp.w), _f64(inp.k)
     ko, qo = inp.k_offsets.numpy(), inp.q_offsets.numpy()
-    qbar = np.stack([O.round_bf16(q[qo[b]:qo[b + 1]].mean(0)) for b in range(3)])
-    wbar = np.stack([w[qo[b]:qo[b + 1]].mean(0) for b in range(3)])
-    res = O.decode_group(q, w, K, ko, qo, k, B, mode, qbar=qbar, wbar=wbar)
+    res = O.decode_group(q, w, K, ko, qo, k, B, mode, q_dtype="bf16")
     gi, gv = idx.cpu().numpy(), val.cpu().numpy()
     for b in range(3):
         k0, k1, r0, r1 = int(ko[b]), int(ko[b + 1]), int(qo[b]), int(qo[b + 1])

@@ -84,16 +84,46 @@ def pin_relu_zero_hand(O):
 def pin_group_hand(O):
     g = _load("group_hand.json")
     q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k"], float)
-    qb, wb = O.proxy(q, w, g["G"])
+    qb, wb = O.proxy(q, w, g["G"], q_dtype="bf16")
     assert np.array_equal(qb, np.array(g["proxy_q"], float)) and np.array_equal(wb, np.array(g["proxy_w"], float))
     for c in g["cases"]:
         for mode, key in ((O.REFINE, "refine"), (O.REUSE, "reuse")):
-            r = O.group(q, w, K, c["k"], g["G"], c["bank"], mode, q_pos0=g["q_pos0"])
+            r = O.group(q, w, K, c["k"], g["G"], c["bank"], mode, q_pos0=g["q_pos0"], q_dtype="bf16")
             assert list(r["bank_idx"][0]) == c["bank_idx"], (c, r["bank_idx"])
             assert list(r["bank_val"][0]) == c["bank_val"]
             for m in range(2):
                 assert list(r["idx"][m]) == c[key + "_idx"][m], (key, c, m, r["idx"][m])
                 assert list(r["val"][m]) == c[key + "_val"][m], (key, c, m, r["val"][m])
+
+
+def pin_proxy_rounding_hand(O):
+    # the proxy query is rounded to the queries' dtype before its scan: with
+    # bf16 queries the rounding turns a strict order into a tie, which moves
+    # the bank and every member's result
+    g = _load("proxy_round_hand.json")
+    q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["k_rows"], float)
+    for dt in ("bf16", "fp32"):
+        e = g[dt]
+        qb, wb = O.proxy(q, w, g["G"], q_dtype=dt)
+        assert np.array_equal(qb, np.array(e["proxy_q"], float)), (dt, qb)
+        assert np.array_equal(wb, np.array([[1.0]])), (dt, wb)
+        for mode, key in ((O.REUSE, "reuse"), (O.REFINE, "refine")):
+            r = O.group(q, w, K, g["k"], g["G"], g["bank"], mode, q_pos0=g["q_pos0"], q_dtype=dt)
+            assert list(r["bank_idx"][0]) == e["bank_idx"] and list(r["bank_val"][0]) == e["bank_val"], (dt, r)
+            for m in range(2):
+                assert list(r["idx"][m]) == e[key + "_idx"][m], (dt, key, m, r["idx"][m])
+                assert list(r["val"][m]) == e[key + "_val"][m], (dt, key, m, r["val"][m])
+    # the same group as a decode step: one sequence of 3 cached keys whose 2 new
+    # queries sit at positions 1 and 2
+    for dt in ("bf16", "fp32"):
+        e = g[dt]
+        r = O.decode_group(q, w, K, [0, 3], [0, 2], g["k"], g["bank"], O.REUSE, q_dtype=dt)
+        assert list(r["bank_idx"][0]) == e["bank_idx"], (dt, r["bank_idx"][0])
+        assert [list(x) for x in r["idx"]] == e["reuse_idx"], (dt, r["idx"])
+    # the fp32 rounding is float32's own
+    x = np.array([1.0 + 2.0 ** -30, 3.0 + 2.0 ** -23, -0.1])
+    assert np.array_equal(O.round_q(x, "fp32"), x.astype(np.float32).astype(np.float64))
+    assert np.array_equal(O.round_q(x, "f64"), x)
 
 
 def pin_decode_hand(O):
@@ -218,16 +248,16 @@ def pin_group_invariants(O):
     q0, k, G = 8, 4, 4
     dn = O.dense(q, w, K, k, q_pos0=q0)
     # Refine with a bank covering the whole prefix is dense selection
-    rf = O.group(q, w, K, k, G, 64, O.REFINE, q_pos0=q0)
+    rf = O.group(q, w, K, k, G, 64, O.REFINE, q_pos0=q0, q_dtype="f64")
     for t in range(12):
         assert np.array_equal(rf["idx"][t], dn["idx"][t])
     # G = 1: the proxy is the query itself, so Reuse == Refine == dense
     for mode in (O.REFINE, O.REUSE):
-        r1 = O.group(q, w, K, k, 1, 6, mode, q_pos0=q0)
+        r1 = O.group(q, w, K, k, 1, 6, mode, q_pos0=q0, q_dtype="f64")
         for t in range(12):
             assert np.array_equal(r1["idx"][t], dn["idx"][t]), (mode, t)
     # Reuse: the last member of a group gets exactly the proxy's top-k
-    ru = O.group(q, w, K, k, G, 7, O.REUSE, q_pos0=q0)
+    ru = O.group(q, w, K, k, G, 7, O.REUSE, q_pos0=q0, q_dtype="f64")
     for g in range(3):
         last = g * G + G - 1
         ps = ru["bank_scores"][g]
@@ -240,13 +270,13 @@ def pin_group_invariants(O):
     # the proxy of identical rows is the row; the proxy of two rows is their midpoint
     qq = np.repeat(q[:1], 4, axis=0)
     ww = np.repeat(w[:1], 4, axis=0)
-    qb, wb = O.proxy(qq, ww, 4)
+    qb, wb = O.proxy(qq, ww, 4, q_dtype="f64")
     assert np.allclose(qb[0], q[0], rtol=1e-15) and np.allclose(wb[0], w[0], rtol=1e-15)
-    qb, wb = O.proxy(q[:2], w[:2], 2)
+    qb, wb = O.proxy(q[:2], w[:2], 2, q_dtype="f64")
     assert np.allclose(qb[0], 0.5 * (q[0] + q[1]), rtol=1e-15)
     assert np.allclose(wb[0], 0.5 * (w[0] + w[1]), rtol=1e-15)
     # partial last group averages over its actual members
-    qb, _ = O.proxy(q[:5], w[:5], 4)
+    qb, _ = O.proxy(q[:5], w[:5], 4, q_dtype="f64")
     assert qb.shape[0] == 2 and np.allclose(qb[1], q[4], rtol=1e-15)
 
 
@@ -271,7 +301,7 @@ def pin_decode_group_hand(O):
     g = _load("decode_group_hand.json")
     q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["K"], float)
     for mode, key in ((O.REFINE, "refine"), (O.REUSE, "reuse")):
-        r = O.decode_group(q, w, K, g["k_offsets"], g["q_offsets"], g["k"], g["bank"], mode)
+        r = O.decode_group(q, w, K, g["k_offsets"], g["q_offsets"], g["k"], g["bank"], mode, q_dtype="bf16")
         for b in range(2):
             assert np.array_equal(r["bank_idx"][b], g["bank_idx"][b]), (key, b, r["bank_idx"][b])
             assert np.array_equal(r["bank_val"][b], g["bank_val"][b]), (key, b, r["bank_val"][b])
@@ -292,10 +322,10 @@ def pin_decode_group_invariants(O):
     qo = np.concatenate([[0], np.cumsum(ms)])
     dec = O.decode(q, w, K, ko, qo, k)
     # a bank as large as every cache makes Refine the decode indexer
-    r = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE)
+    r = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE, q_dtype="f64")
     assert np.array_equal(r["idx"], dec["idx"]) and np.array_equal(r["val"], dec["val"])
-    rf = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE)
-    ru = O.decode_group(q, w, K, ko, qo, k, 4, O.REUSE)
+    rf = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE, q_dtype="f64")
+    ru = O.decode_group(q, w, K, ko, qo, k, 4, O.REUSE, q_dtype="f64")
     for b in range(4):
         last = qo[b + 1] - 1
         # the last query may see the whole bank: Reuse gives it the proxy's top-k
@@ -310,9 +340,9 @@ def pin_decode_group_invariants(O):
     # decode indexer; with a small bank each query's candidates are the bank
     # plus its sequence's new keys up to its own position, so its selection is
     # causal, never worse than plain Refine, and the top-k of those candidates
-    rl_full = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE_LOCAL)
+    rl_full = O.decode_group(q, w, K, ko, qo, k, max(lengths), O.REFINE_LOCAL, q_dtype="f64")
     assert np.array_equal(rl_full["idx"], dec["idx"]) and np.array_equal(rl_full["val"], dec["val"])
-    rl = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE_LOCAL)
+    rl = O.decode_group(q, w, K, ko, qo, k, 4, O.REFINE_LOCAL, q_dtype="f64")
     for b in range(4):
         nb, mb = lengths[b], ms[b]
         Kb = K[ko[b]:ko[b + 1]]
@@ -333,7 +363,7 @@ def pin_group_local_hand(O):
     g = _load("group_local_hand.json")
     q, w, K = np.array(g["q"], float), np.array(g["w"], float), np.array(g["K"], float)
     for mode, key in ((O.REFINE, "refine"), (O.REFINE_LOCAL, "refine_local"), (O.REUSE, "reuse")):
-        r = O.group(q, w, K, g["k"], g["G"], g["bank"], mode, q_pos0=g["q_pos0"])
+        r = O.group(q, w, K, g["k"], g["G"], g["bank"], mode, q_pos0=g["q_pos0"], q_dtype="bf16")
         assert np.array_equal(r["bank_idx"][0], g["bank_idx"]), (key, r["bank_idx"][0])
         for t in range(2):
             assert np.array_equal(r["idx"][t], g[key + "_idx"][t]), (key, t, r["idx"][t])
@@ -344,9 +374,9 @@ def pin_group_local_invariants(O):
     q, w, K, _ = _rand_case(12, T=14, N=24, H=3, d=4, q_pos0=10)
     k, G = 4, 5
     dn = O.dense(q, w, K, k, q_pos0=10)
-    full = O.group(q, w, K, k, G, 24, O.REFINE_LOCAL, q_pos0=10)
-    rf = O.group(q, w, K, k, G, 6, O.REFINE, q_pos0=10)
-    rl = O.group(q, w, K, k, G, 6, O.REFINE_LOCAL, q_pos0=10)
+    full = O.group(q, w, K, k, G, 24, O.REFINE_LOCAL, q_pos0=10, q_dtype="f64")
+    rf = O.group(q, w, K, k, G, 6, O.REFINE, q_pos0=10, q_dtype="f64")
+    rl = O.group(q, w, K, k, G, 6, O.REFINE_LOCAL, q_pos0=10, q_dtype="f64")
     for t in range(14):
         p = 10 + t
         # a bank covering the prefix: the dense indexer
@@ -446,7 +476,7 @@ def pin_round_bf16_library(O):
 
 
 PINS = [pin_e4m3_table, pin_e4m3_library, pin_dense_hand, pin_ties_hand,
-        pin_relu_zero_hand, pin_group_hand, pin_decode_hand, pin_single_head_matmul,
+        pin_relu_zero_hand, pin_group_hand, pin_proxy_rounding_hand, pin_decode_hand, pin_single_head_matmul,
         pin_relu_odd_identity, pin_head_structure, pin_fp8_keys_scale,
         pin_topk_bruteforce, pin_causality, pin_group_invariants,
         pin_decode_matches_dense, pin_decode_group_hand, pin_decode_group_invariants,
@@ -527,7 +557,7 @@ def _m_head_mean(mp):
 
 
 def _m_proxy_sum(mp):
-    def bad(q, w, G):
+    def bad(q, w, G, *, q_dtype):
         T = q.shape[0]
         ng = (T + G - 1) // G
         return (np.stack([q[g * G:(g + 1) * G].sum(0) for g in range(ng)]),
@@ -536,7 +566,7 @@ def _m_proxy_sum(mp):
 
 
 def _m_proxy_first_member(mp):
-    def bad(q, w, G):
+    def bad(q, w, G, *, q_dtype):
         T = q.shape[0]
         ng = (T + G - 1) // G
         return (np.stack([q[g * G] for g in range(ng)]), np.stack([w[g * G] for g in range(ng)]))
@@ -574,6 +604,11 @@ def _m_decode_group_first_positions(mp):
     mp.setattr(O, "decode_group", dg)
 
 
+def _m_proxy_unrounded(mp):
+    # the proxy query kept at the float64 mean, whatever the queries' dtype
+    mp.setattr(O, "round_q", lambda x, q_dtype: np.asarray(x, dtype=np.float64))
+
+
 def _m_decode_group_scan_first_member(mp):
     # the proxy scans only its first member's prefix: the cache cut at N_b - m_b + 1
     real = O.decode_group
@@ -586,7 +621,7 @@ def _m_decode_group_scan_first_member(mp):
         for b in range(len(ko) - 1):
             Nb, mb = int(ko[b + 1] - ko[b]), int(qo[b + 1] - qo[b])
             r = real(q[qo[b]:qo[b + 1]], w[qo[b]:qo[b + 1]], K[ko[b]:ko[b] + Nb - mb + 1], [0, Nb - mb + 1],
-                     [0, mb], k, bank, mode)
+                     [0, mb], k, bank, mode, **kw)
             out_i[qo[b]:qo[b + 1]], out_v[qo[b]:qo[b + 1]] = r["idx"], r["val"]
             res["bank_idx"][b], res["bank_val"][b] = r["bank_idx"][0], r["bank_val"][0]
             res["count"][qo[b]:qo[b + 1]] = r["count"]
@@ -696,7 +731,7 @@ def _m_round_bf16_truncate(mp):
 MUTANTS = [_m_no_relu, _m_abs_relu, _m_causal_exclusive, _m_causal_plus_one,
            _m_tiebreak_high, _m_ascending, _m_e4m3_bias8, _m_e4m3_no_subnormal,
            _m_weight_outside, _m_transposed_weight, _m_head_mean, _m_proxy_sum,
-           _m_proxy_first_member, _m_decode_first_positions, _m_decode_group_first_positions,
+           _m_proxy_first_member, _m_proxy_unrounded, _m_decode_first_positions, _m_decode_group_first_positions,
            _m_decode_group_scan_first_member, _m_local_window_before_self, _m_local_window_whole_group,
            _m_block_own_block_dropped, _m_block_partial_blocks_routed, _m_kmeans_one_iteration_short,
            _m_ivf_no_causal_mask, _m_round_bf16_truncate]
