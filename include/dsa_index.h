@@ -84,8 +84,9 @@ const char* dsa_status_string(int status);
 int dsa_version(void);
 
 /* Synchronises `stream`, then reads and clears the device status word kept
- * in `workspace`.  Returns DSA_OK, the recorded DSA_ERR_TIMEOUT or
- * DSA_ERR_INTERNAL, or DSA_ERR_CUDA if the stream reported an error. */
+ * in `workspace`.  Returns DSA_OK, the recorded DSA_ERR_TIMEOUT,
+ * DSA_ERR_INTERNAL or DSA_ERR_INVALID_ARG (decode offsets that failed their
+ * device check), or DSA_ERR_CUDA if the stream reported an error. */
 int dsa_check_status(void* workspace, void* stream);
 
 /* ------------------------------------------------------------------------
@@ -157,7 +158,15 @@ int dsa_index_group(const void* Q, const float* w, const void* K,
  *   New query j of sequence b sits at position N_b - m_b + j and sees its
  *   sequence's keys 0 .. N_b - m_b + j.  Output indices are local to the
  *   sequence (0 .. N_b - 1).
- *   k_offsets [B+1] int64, q_offsets [B+1] int32: DEVICE arrays.
+ *   k_offsets [B+1] int64, q_offsets [B+1] int32: DEVICE arrays, read on
+ *          the device only (no synchronisation).  The kernels check every
+ *          sequence they read: 0 <= k_offsets[b], 1 <= N_b <= max_keys,
+ *          k_offsets[b+1] <= total_keys, 0 <= q_offsets[b], q_offsets[b+1]
+ *          <= total_q, 1 <= m_b <= min(4, N_b).  A sequence that fails is
+ *          skipped and DSA_ERR_INVALID_ARG is recorded in the status word
+ *          (dsa_check_status); the outputs of such a call are unspecified,
+ *          but no kernel reads or writes outside the buffers the sizes
+ *          describe.
  *   total_keys: k_offsets[B] (host value: rows of K; tensor copies never
  *          read beyond it).
  *   max_keys: an upper bound on every N_b (host value; sizes the split of
@@ -193,7 +202,9 @@ int dsa_index_decode(const void* Q, const float* w, const void* K,
  *           DSA_GROUP_REFINE_LOCAL: Refine whose candidates also hold the
  *           sequence's new keys N_b - m_b .. its own position.
  *   Arguments as for dsa_index_decode (1 <= m_b <= min(4, N_b), device
- *   offsets, local output indices), plus bank (k <= bank <= 16384), mode and
+ *   offsets, local output indices; a first kernel checks the offsets as
+ *   listed there plus q_offsets[B] = total_q, and when they fail no later
+ *   kernel of the call does any work), plus bank (k <= bank <= 16384), mode and
  *   the optional outputs bank_idx/bank_val [B, bank] (ranked, -1 / -inf
  *   padded; asking for them costs a sort of every bank) and proxy_q
  *   [B, H, d] (q_dtype) / proxy_w [B, H] fp32.  Tensor-core shape only (bf16

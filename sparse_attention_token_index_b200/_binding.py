@@ -295,7 +295,7 @@ def dsa_index_decode(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: torch.
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
-    ko, qo, max_keys, total_keys = _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys)
+    ko, qo, max_keys, total_keys = _decode_offsets(Q, K, k_offsets, q_offsets, max_keys, total_keys)
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     nb = decode_workspace_bytes(B, total_q, max_keys, H, d, k, qd, kd)
     ws = _workspace(nb, Q.device, workspace)
@@ -315,15 +315,40 @@ def decode_group_workspace_bytes(B, total_q, max_keys, H, d, k, bank, q_dtype, k
     return int(n.value)
 
 
-def _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys):
+def _decode_offsets(Q, K, k_offsets, q_offsets, max_keys, total_keys):
+    """Offsets on the host (or copied there because max_keys / total_keys are
+    missing) are checked here in full: k_offsets[0] = q_offsets[0] = 0,
+    q_offsets[B] = Q's rows, k_offsets[B] = total_keys <= K's rows, and every
+    sequence with 1 <= N_b <= max_keys keys and 1 <= m_b <= min(4, N_b)
+    queries.  Device offsets with both sizes given are not read back (no
+    synchronisation); the library checks them on the device and reports an
+    invalid argument through the status word."""
     if k_offsets.numel() != q_offsets.numel() or k_offsets.numel() < 1:
         raise ValueError("k_offsets and q_offsets must both be [B+1]")
-    if max_keys is None or total_keys is None:
-        ko_host = k_offsets.to("cpu", torch.int64)
+    if total_keys is not None and int(total_keys) > K.shape[0]:
+        raise ValueError(f"total_keys {int(total_keys)} exceeds the {K.shape[0]} rows of K")
+    on_host = not (k_offsets.is_cuda and q_offsets.is_cuda)
+    if on_host or max_keys is None or total_keys is None:
+        ko_h = k_offsets.to("cpu", torch.int64)
+        qo_h = q_offsets.to("cpu", torch.int64)
+        nb, mb = ko_h[1:] - ko_h[:-1], qo_h[1:] - qo_h[:-1]
         if max_keys is None:
-            max_keys = int((ko_host[1:] - ko_host[:-1]).max()) if ko_host.numel() > 1 else 0
+            max_keys = int(nb.max()) if nb.numel() else 0
         if total_keys is None:
-            total_keys = int(ko_host[-1])
+            total_keys = int(ko_h[-1])
+        bad = None
+        if int(ko_h[0]) != 0 or int(qo_h[0]) != 0:
+            bad = "offsets must start at 0"
+        elif int(qo_h[-1]) != Q.shape[0]:
+            bad = f"q_offsets[B] = {int(qo_h[-1])} is not the {Q.shape[0]} query rows"
+        elif int(ko_h[-1]) != int(total_keys) or int(total_keys) > K.shape[0]:
+            bad = f"k_offsets[B] = {int(ko_h[-1])} must equal total_keys ({int(total_keys)}) <= K's {K.shape[0]} rows"
+        elif nb.numel() and (bool((nb < 1).any()) or int(nb.max()) > int(max_keys)):
+            bad = f"every sequence needs 1 .. max_keys ({int(max_keys)}) keys"
+        elif mb.numel() and (bool((mb < 1).any()) or bool((mb > 4).any()) or bool((mb > nb).any())):
+            bad = "every sequence needs 1 <= m_b <= min(4, N_b) new queries"
+        if bad:
+            raise ValueError(bad)
     ko = k_offsets if (k_offsets.is_cuda and k_offsets.dtype == torch.int64) else \
         k_offsets.to(Q.device, torch.int64).contiguous()
     qo = q_offsets if (q_offsets.is_cuda and q_offsets.dtype == torch.int32) else \
@@ -345,7 +370,7 @@ def dsa_index_decode_group(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: 
     _need_cuda(Q, w, K, K_scale)
     total_q, H, d = Q.shape
     B = k_offsets.numel() - 1
-    ko, qo, max_keys, total_keys = _decode_offsets(Q, k_offsets, q_offsets, max_keys, total_keys)
+    ko, qo, max_keys, total_keys = _decode_offsets(Q, K, k_offsets, q_offsets, max_keys, total_keys)
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     nb = decode_group_workspace_bytes(B, total_q, max_keys, H, d, k, bank, qd, kd)
     ws = _workspace(nb, Q.device, workspace)
@@ -664,6 +689,7 @@ def dsa_index_decode_host(Q, w, K, k: int, k_offsets: torch.Tensor, q_offsets: t
     total_keys = int(ko[-1])
     if max_keys is None:
         max_keys = int((ko[1:] - ko[:-1]).max()) if ko.numel() > 1 else 0
+    _decode_offsets(Q, K, ko, qo, max_keys, total_keys)  # host offsets: checked in full
     qd, kd = _dtype_code(Q), _dtype_code(K, allow_fp8=True)
     st = _staging(decode_host_staging_bytes(B, total_q, total_keys, max_keys, H, d, k, qd, kd), device, staging)
     idx, val = _host_outputs(total_q, k, out)

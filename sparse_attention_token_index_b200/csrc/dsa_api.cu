@@ -10,59 +10,47 @@
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
-using namespace dsa;
+namespace dsa {
 
-namespace {
-
-constexpr int kMaxK = 65536;
-
-struct DeviceInfo {
-  bool ok = false;
-  int sms = 0;
-};
-
-int device_info(DeviceInfo& out) {
+int current_device(int* dev_out, int* sms_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
-  static DeviceInfo cache[64];
+  static int sms_cache[64];
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   if (dev < 0 || dev >= 64) return DSA_ERR_DEVICE;
-  if (!cache[dev].ok) {
+  if (sms_cache[dev] == 0) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return DSA_ERR_CUDA;
-    if (major != 10 || minor != 0) return DSA_ERR_DEVICE;
-    cache[dev].sms = sms;
-    cache[dev].ok = true;
+    if (major != 10 || minor != 0 || sms < 1) return DSA_ERR_DEVICE;  // only sm_100a code is built
+    sms_cache[dev] = sms;
   }
-  out = cache[dev];
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = sms_cache[dev];
   return DSA_OK;
+}
+
+void* driver_entry(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // 2-D bf16 tensor map over [rows, inner] with a box of 64 elements (128 B)
 // x box_rows rows, 128-byte swizzle (the layout the MMA descriptors expect).
 int make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t inner, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] { fn = reinterpret_cast<EncodeTiledFn>(driver_entry("cuTensorMapEncodeTiled")); });
   if (!fn) return DSA_ERR_CUDA;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
@@ -73,6 +61,20 @@ int make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t in
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_CUDA;
 }
+
+}  // namespace dsa
+
+using namespace dsa;
+
+namespace {
+
+constexpr int kMaxK = 65536;
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+int device_info(DeviceInfo& out) { return current_device(nullptr, &out.sms); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -582,7 +584,7 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
 // idx / val [rows, k].  K is bf16 (fp8 keys already widened).
 int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void* K, const float* K_scale,
                   const int64_t* k_offsets, const int32_t* q_offsets, int B, int rows, int64_t total_keys, int H,
-                  int d, int k, int32_t* idx, float* val, uint8_t* ws, cudaStream_t st) {
+                  int d, int k, int32_t* idx, float* val, uint8_t* ws, cudaStream_t st, const int* ok = nullptr) {
   int r;
   uint2* ppair = reinterpret_cast<uint2*>(ws + p.ppair_off);
   int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
@@ -610,8 +612,10 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
   a.q_off = q_offsets;
   a.splits = p.splits;
   a.tiles_per_split = p.tiles_per_split;
+  a.total_keys = total_keys;
+  a.offsets_ok = ok;
   if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
-  return launch_decode_merge(ppair, pcnt, rows, p.splits, k, idx, val, status, st);
+  return launch_decode_merge(ppair, pcnt, rows, p.splits, k, idx, val, status, st, ok);
 }
 
 }  // namespace
@@ -688,6 +692,7 @@ int dsa_index_decode(const void* Q, const float* w, const void* K, const float* 
     a.B = B;
     a.splits = p.splits;
     a.keys_per_split = p.tiles_per_split * 128;
+    a.total_keys = total_keys;
     if ((r = launch_simt_index(a, p.grid, st)) != DSA_OK) return r;
   }
   return launch_decode_merge(ppair, pcnt, total_q, p.splits, k, idx, val, status, st);
@@ -782,17 +787,22 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   float* wbar = proxy_w ? proxy_w : reinterpret_cast<float*>(ws + gp.wbar_off);
   int32_t* bi = bank_idx ? bank_idx : reinterpret_cast<int32_t*>(ws + gp.bidx_off);
   float* bv = bank_val ? bank_val : reinterpret_cast<float*>(ws + gp.bval_off);
-  // 0. fp8 keys: exact bf16 copy, the per-key scale goes to the epilogue
+  // 0. the offsets, checked once on the device: every later kernel that
+  // reads them does nothing if they failed (invalid argument in the status)
+  if ((r = launch_decode_offsets_check(k_offsets, q_offsets, B, total_keys, total_q, max_keys, ws, st)) != DSA_OK)
+    return r;
+  const int* ok = &reinterpret_cast<const WsHeader*>(ws)->offsets_ok;
+  // fp8 keys: exact bf16 copy, the per-key scale goes to the epilogue
   if (needs_widen(H, d, q_dtype, k_dtype)) {
     if ((r = widen_keys(K, total_keys, d, ws, gp.scan.widen_off, st)) != DSA_OK) return r;
     K = ws + gp.scan.widen_off;
   }
   // 1. proxies: the mean of each sequence's new queries
-  if ((r = launch_proxy_mean(Q, w, total_q, H, d, 1, q_dtype, qbar, wbar, st, q_offsets, B)) != DSA_OK) return r;
+  if ((r = launch_proxy_mean(Q, w, total_q, H, d, 1, q_dtype, qbar, wbar, st, q_offsets, B, ok)) != DSA_OK) return r;
   // 2. one scan of each cache by its proxy, which sits at the last query's
   // position N_b - 1: bank = its top-`bank` keys (local indices)
   if ((r = run_decode_tc(gp.scan, qbar, wbar, K, K_scale, k_offsets, nullptr, B, B, total_keys, H, d, bank, bi, bv,
-                         ws, st)) != DSA_OK)
+                         ws, st, ok)) != DSA_OK)
     return r;
   // 3. Reuse ranks the bank and finishes here; Refine ranks it only for the
   // caller's bank output.  A sequence's queries drop at most 3 bank keys
@@ -800,7 +810,7 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   const bool want_bank = bank_idx != nullptr || bank_val != nullptr;
   if (mode == DSA_GROUP_REUSE || want_bank) {
     if ((r = launch_bank_rank_reuse(bi, bv, B, bank, 4, total_q, 0, k, idx, val, mode == DSA_GROUP_REUSE, want_bank,
-                                    st, q_offsets, k_offsets)) != DSA_OK)
+                                    st, q_offsets, k_offsets, ok)) != DSA_OK)
       return r;
   }
   if (mode == DSA_GROUP_REUSE) return DSA_OK;
@@ -811,11 +821,12 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   const int32_t* kmap = bi;
   if (local) {
     int32_t* map = reinterpret_cast<int32_t*>(ws + gp.map_off);
-    if ((r = launch_local_extend(bi, B, bank, 4, total_q, 0, q_offsets, k_offsets, S, map, st)) != DSA_OK) return r;
+    if ((r = launch_local_extend(bi, B, bank, 4, total_q, 0, q_offsets, k_offsets, S, map, st, ok)) != DSA_OK)
+      return r;
     kmap = map;
   }
   void* Kg = ws + gp.kg_off;
-  if ((r = launch_bank_gather(K, DSA_DTYPE_BF16, d, kmap, B, S, Kg, st, k_offsets)) != DSA_OK) return r;
+  if ((r = launch_bank_gather(K, DSA_DTYPE_BF16, d, kmap, B, S, Kg, st, k_offsets, ok)) != DSA_OK) return r;
   CUtensorMap tmQ, tmK;
   if ((r = make_map_bf16(&tmQ, Q, (uint64_t)total_q * H, (uint64_t)d, 64)) != DSA_OK) return r;
   if ((r = make_map_bf16(&tmK, Kg, (uint64_t)B * S, (uint64_t)d, 128)) != DSA_OK) return r;
@@ -840,6 +851,8 @@ int dsa_index_decode_group(const void* Q, const float* w, const void* K, const f
   a.T = total_q;
   a.k_off = k_offsets;
   a.q_off = q_offsets;
+  a.total_keys = total_keys;
+  a.offsets_ok = ok;
   return launch_tc_index(tmQ, tmK, a, gp.ref_grid, st);
 }
 

@@ -24,7 +24,8 @@ namespace dsa {
 // seg (per-group row offsets, e.g. a decode batch's query offsets) is given.
 __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __restrict__ w, int T, int H, int d,
                                   int G, const int32_t* __restrict__ seg, int q_dtype, void* __restrict__ qbar,
-                                  float* __restrict__ wbar) {
+                                  float* __restrict__ wbar, const int* ok) {
+  if (offsets_bad(ok)) return;
   const int g = blockIdx.y;
   const int r0 = seg ? seg[g] : g * G, r1 = seg ? seg[g + 1] : min(T, r0 + G);
   const float n = (float)(r1 - r0);
@@ -75,11 +76,11 @@ __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __res
 }
 
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
-                      float* wbar, cudaStream_t stream, const int32_t* seg, int nseg) {
+                      float* wbar, cudaStream_t stream, const int32_t* seg, int nseg, const int* ok) {
   const int ng = seg ? nseg : (T + G - 1) / G;
   const int64_t chunks = ((int64_t)H * d + 7) / 8;
   const dim3 grid((unsigned)((chunks + 127) / 128), (unsigned)ng);
-  proxy_mean_kernel<<<grid, 128, 0, stream>>>(Q, w, T, H, d, G, seg, q_dtype, qbar, wbar);
+  proxy_mean_kernel<<<grid, 128, 0, stream>>>(Q, w, T, H, d, G, seg, q_dtype, qbar, wbar, ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -116,7 +117,8 @@ int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, voi
 // ---------------------------------------------------------------------------
 __global__ void bank_gather_kernel(const uint4* __restrict__ K, int row_vecs, const int32_t* __restrict__ bank,
                                    int64_t n_rows, int bank_size, const int64_t* __restrict__ row_off,
-                                   uint4* __restrict__ Kg) {
+                                   uint4* __restrict__ Kg, const int* ok) {
+  if (offsets_bad(ok)) return;
   const int64_t total = n_rows * row_vecs;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / row_vecs;
@@ -128,12 +130,12 @@ __global__ void bank_gather_kernel(const uint4* __restrict__ K, int row_vecs, co
 }
 
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size, void* Kg,
-                       cudaStream_t stream, const int64_t* row_off) {
+                       cudaStream_t stream, const int64_t* row_off, const int* ok) {
   const int elt = (k_dtype == DSA_DTYPE_FP32) ? 4 : (k_dtype == DSA_DTYPE_BF16 ? 2 : 1);
   const int row_vecs = d * elt / 16;
   bank_gather_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), row_vecs, bank,
                                                    (int64_t)ng * bank_size, bank_size, row_off,
-                                                   static_cast<uint4*>(Kg));
+                                                   static_cast<uint4*>(Kg), ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -146,8 +148,9 @@ int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, i
 // ---------------------------------------------------------------------------
 __global__ void local_extend_kernel(const int32_t* __restrict__ bank, int B, int G, int T, int64_t q_pos0,
                                     const int32_t* __restrict__ q_off, const int64_t* __restrict__ k_off, int S,
-                                    int32_t* __restrict__ map) {
+                                    int32_t* __restrict__ map, const int* ok) {
   extern __shared__ int in_bank[];  // [S - B]
+  if (offsets_bad(ok)) return;
   const int g = blockIdx.x, tid = threadIdx.x;
   const int W = S - B;
   int r0, r1;
@@ -176,10 +179,10 @@ __global__ void local_extend_kernel(const int32_t* __restrict__ bank, int B, int
 }
 
 int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
-                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream) {
+                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream, const int* ok) {
   if (S - B < 1 || S - B > 4096) return DSA_ERR_INVALID_ARG;
   local_extend_kernel<<<ng, 256, (size_t)(S - B) * sizeof(int), stream>>>(bank, B, G, T, q_pos0, q_off, k_off, S,
-                                                                          map);
+                                                                          map, ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -202,10 +205,12 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
                                                                        int k, int32_t* __restrict__ out_idx,
                                                                        float* __restrict__ out_val, int do_reuse,
                                                                        const int32_t* __restrict__ q_off,
-                                                                       const int64_t* __restrict__ k_off) {
+                                                                       const int64_t* __restrict__ k_off,
+                                                                       const int* ok) {
   extern __shared__ uint64_t keys[];  // [P] the bank; then [PM] its top M when M < B
   __shared__ uint32_t hist[256];
   __shared__ int sh_digit, sh_above, sh_in, sh_cnt;
+  if (offsets_bad(ok)) return;
   const int g = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   int32_t* bi = bank_idx + (int64_t)g * B;
@@ -360,7 +365,7 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
 
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T, int64_t q_pos0,
                            int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all, cudaStream_t stream,
-                           const int32_t* q_off, const int64_t* k_off) {
+                           const int32_t* q_off, const int64_t* k_off, const int* ok) {
   int P = 1;
   while (P < bank_size) P <<= 1;
   if (P > kMaxBank) return DSA_ERR_UNSUPPORTED;
@@ -379,7 +384,7 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
                                                (int)smem) != cudaSuccess)
     return DSA_ERR_CUDA;
   bank_rank_reuse_kernel<<<ng, kRankThreads, smem, stream>>>(bank_idx, bank_val, bank_size, P, M, PM, G, T, q_pos0, k,
-                                                             out_idx, out_val, do_reuse, q_off, k_off);
+                                                             out_idx, out_val, do_reuse, q_off, k_off, ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -400,16 +405,25 @@ struct MergeSmem {
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const uint2* __restrict__ parts,
                                                                      const int* __restrict__ part_cnt, int splits,
                                                                      int k, int32_t* __restrict__ out_idx,
-                                                                     float* __restrict__ out_val, int* status) {
+                                                                     float* __restrict__ out_val, int* status,
+                                                                     const int* ok) {
   __shared__ MergeSmem M;
+  __shared__ int cnt[256];
+  if (offsets_bad(ok)) return;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   RowState& st = M.st;
   row_reset(st, tid, kMergeThreads);
+  // a split holds at most k entries; a count outside [0, k] (a slice the scan
+  // skipped because its sequence's offsets were invalid) reads as empty
+  for (int s = tid; s < splits; s += kMergeThreads) {
+    const int c = __ldcg(part_cnt + (int64_t)row * splits + s);
+    cnt[s] = (c >= 0 && c <= k) ? c : 0;
+  }
   CandList cl;
   cl.base = parts + (int64_t)row * splits * k;
   cl.stride = k;
   cl.nseg = splits;
-  cl.cnt = part_cnt + (int64_t)row * splits;
+  cl.cnt = cnt;
   cl.l2 = true;  // written by the scoring kernel's other CTAs
   __syncthreads();
   for_each_cand(cl, tid, kMergeThreads, [&](uint2 e, bool v) {
@@ -429,9 +443,42 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const uint2
 }
 
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
-                        float* out_val, int* status, cudaStream_t stream) {
+                        float* out_val, int* status, cudaStream_t stream, const int* ok) {
   if (splits > 256) return DSA_ERR_UNSUPPORTED;
-  decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(parts, part_cnt, splits, k, out_idx, out_val, status);
+  decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(parts, part_cnt, splits, k, out_idx, out_val, status,
+                                                             ok);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Device check of a decode batch's offsets, before any kernel that reads them
+// (the group form in decode runs several).  Sequence b: k_off[b] >= 0,
+// 1 <= N_b = k_off[b+1] - k_off[b] <= max_keys, k_off[b+1] <= total_keys,
+// q_off[b] >= 0, 1 <= m_b = q_off[b+1] - q_off[b] <= min(4, N_b), and
+// q_off[B] = total_q.  Writes the verdict to hdr->offsets_ok; a failure is
+// also recorded as an invalid argument in the status word.
+// ---------------------------------------------------------------------------
+__global__ void decode_offsets_check_kernel(const int64_t* __restrict__ k_off, const int32_t* __restrict__ q_off,
+                                            int B, int64_t total_keys, int total_q, int max_keys, WsHeader* hdr) {
+  bool ok = true;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t k0 = k_off[b], k1 = k_off[b + 1];
+    const int64_t q0 = q_off[b], q1 = q_off[b + 1];
+    ok = ok && k0 >= 0 && k1 - k0 >= 1 && k1 - k0 <= max_keys && k1 <= total_keys && q0 >= 0 && q1 - q0 >= 1 &&
+         q1 - q0 <= 4 && q1 - q0 <= k1 - k0;
+  }
+  if (threadIdx.x == 0) ok = ok && q_off[B] == total_q;
+  ok = __syncthreads_and(ok) != 0;
+  if (threadIdx.x == 0) {
+    hdr->offsets_ok = ok ? 1 : 0;
+    if (!ok) report_error(&hdr->status, DSA_ERR_INVALID_ARG, 6);
+  }
+}
+
+int launch_decode_offsets_check(const int64_t* k_off, const int32_t* q_off, int B, int64_t total_keys, int total_q,
+                                int max_keys, void* workspace, cudaStream_t stream) {
+  decode_offsets_check_kernel<<<1, 256, 0, stream>>>(k_off, q_off, B, total_keys, total_q, max_keys,
+                                                     static_cast<WsHeader*>(workspace));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

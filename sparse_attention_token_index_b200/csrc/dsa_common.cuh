@@ -23,12 +23,19 @@ namespace dsa {
 struct WsHeader {
   int status;      // first device-side error (0 = none)
   int info;        // where it happened
-  int pad[62];
+  int offsets_ok;  // decode groups: 1 when the call's offsets passed their device check
+  int pad[61];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 __device__ __forceinline__ void report_error(int* status, int code, int info) {
   if (atomicCAS(status, 0, code) == 0) status[1] = info;
+}
+
+// A call whose device offsets failed their check (offsets_ok == 0) runs none
+// of its later kernels' work; null means the kernel checks its own.
+__device__ __forceinline__ bool offsets_bad(const int* ok) {
+  return ok != nullptr && *(volatile const int*)ok == 0;
 }
 
 // ----------------------------------------------------------------------------

@@ -289,12 +289,19 @@ int dsa_index_decode_host(const void* Q, const float* w, const void* K, const fl
   if (!Q || !w || !K || !k_offsets || !q_offsets || !idx || !val || !staging || !aligned16(staging))
     return DSA_ERR_INVALID_ARG;
   if ((k_dtype == DSA_DTYPE_FP8_E4M3) != (K_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+  // the offsets are in host memory here: check all of them before anything
+  // else (sequence b: 1 <= N_b <= max_keys, 1 <= m_b <= min(4, N_b))
+  if (B < 0 || k_offsets[0] != 0 || k_offsets[B] != total_keys || q_offsets[0] != 0 || q_offsets[B] != total_q)
+    return DSA_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b) {
+    const int64_t nb = k_offsets[b + 1] - k_offsets[b];
+    const int64_t mb = (int64_t)q_offsets[b + 1] - q_offsets[b];
+    if (nb < 1 || nb > max_keys || mb < 1 || mb > 4 || mb > nb) return DSA_ERR_INVALID_ARG;
+  }
   size_t need = 0;
   int r = dsa_index_decode_host_staging_size(B, total_q, total_keys, max_keys, H, d, k, q_dtype, k_dtype, &need);
   if (r != DSA_OK) return r;
   if (staging_bytes < need) return DSA_ERR_WORKSPACE;
-  if (k_offsets[0] != 0 || k_offsets[B] != total_keys || q_offsets[0] != 0 || q_offsets[B] != total_q)
-    return DSA_ERR_INVALID_ARG;
   size_t ws = 0;
   if ((r = dsa_index_decode_workspace_size(B, total_q, max_keys, H, d, k, q_dtype, k_dtype, &ws)) != DSA_OK) return r;
   const size_t qe = elem_size(q_dtype), ke = elem_size(k_dtype);

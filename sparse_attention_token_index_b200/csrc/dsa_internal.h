@@ -48,6 +48,8 @@ struct TcArgs {
   const int32_t* q_off;
   int splits;
   int tiles_per_split;
+  int64_t total_keys;     // rows of K: every k_off[b + 1] must stay within it
+  const int* offsets_ok;  // decode groups: the call's device check of its offsets (null: none)
   // refine
   const int32_t* key_map;   // [ng, bank] bank key positions (-1 = empty)
   int bank;        // key slots per group in the gathered bank (its row stride)
@@ -71,6 +73,14 @@ struct TcArgs {
   const int32_t* ivf_tiles;
   int ivf_max_tiles;  // candidate lists hold this many tiles per query
 };
+
+// The current device, checked once: compute capability 10.0 (only sm_100a
+// code is built) and its multiprocessor count.
+int current_device(int* dev, int* sms);
+// A driver entry point (resolved through the runtime, no libcuda link).
+void* driver_entry(const char* name);
+// 2-D bf16 tensor map over [rows, inner], box 64 x box_rows, 128-byte swizzle.
+int make_map_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t inner, uint32_t box_rows);
 
 // Event pair for timing one scoring-kernel launch (dsa_timer.cu); both null
 // unless dsa_kernel_timer_start armed the timer and a slot is left.
@@ -110,6 +120,7 @@ struct SimtArgs {
   int B;
   int splits;
   int keys_per_split;
+  int64_t total_keys;     // rows of K: every k_off[b + 1] must stay within it
 };
 int launch_simt_index(const SimtArgs& a, int grid, cudaStream_t stream);
 size_t simt_smem_bytes(int H, int d);
@@ -117,24 +128,31 @@ size_t simt_smem_bytes(int H, int d);
 // Auxiliary kernels.
 // Groups of G consecutive rows, or (seg given) rows seg[g] .. seg[g+1]-1 of
 // nseg groups.
+// `ok` (decode groups): the call's offsets check; the kernels that read device
+// offsets do nothing when it failed.
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
-                      float* wbar, cudaStream_t stream, const int32_t* seg = nullptr, int nseg = 0);
+                      float* wbar, cudaStream_t stream, const int32_t* seg = nullptr, int nseg = 0,
+                      const int* ok = nullptr);
 // row_off (decode): bank indices are local to sequence g, whose rows start at row_off[g].
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
-                       void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr);
+                       void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr, const int* ok = nullptr);
 // rank_all: sort and write back the whole bank; otherwise only the top
 // k + G - 1 entries are ranked (enough for Reuse) and the bank is not written.
 // Refine with query-specific additions: map [ng, S] = bank (B) + own stretch (S - B).
 int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
-                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream);
+                        const int64_t* k_off, int S, int32_t* map, cudaStream_t stream, const int* ok = nullptr);
 // q_off / k_off (decode): group g is sequence g with members q_off[g] ..
 // q_off[g+1]-1 at positions N_g - m_g + j (local key indices).
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T,
                            int64_t q_pos0, int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all,
-                           cudaStream_t stream, const int32_t* q_off = nullptr, const int64_t* k_off = nullptr);
+                           cudaStream_t stream, const int32_t* q_off = nullptr, const int64_t* k_off = nullptr,
+                           const int* ok = nullptr);
 // parts [total_q, splits, k] {score bits, index} pairs, part_cnt [total_q, splits]
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
-                        float* out_val, int* status, cudaStream_t stream);
+                        float* out_val, int* status, cudaStream_t stream, const int* ok = nullptr);
+// Device check of decode offsets into the workspace header (offsets_ok + status word).
+int launch_decode_offsets_check(const int64_t* k_off, const int32_t* q_off, int B, int64_t total_keys, int total_q,
+                                int max_keys, void* workspace, cudaStream_t stream);
 int launch_fill_scores(float* S, int64_t n, cudaStream_t stream);
 // Block representatives of bf16 keys (fp8 keys widened; K_scale applied when given).
 int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, void* R, cudaStream_t stream);

@@ -62,10 +62,22 @@ __global__ void __launch_bounds__(kSimtThreads) simt_index_kernel(const SimtArgs
     } else {
       const int qrow = task / a.splits, sp = task % a.splits;
       int b = 0;
-      while (a.q_off[b + 1] <= qrow) ++b;
-      const int64_t k0 = a.k_off[b], k1 = a.k_off[b + 1];
-      const int mb = a.q_off[b + 1] - a.q_off[b];
-      const int j = qrow - a.q_off[b];
+      while (b < a.B && a.q_off[b + 1] <= qrow) ++b;
+      const int64_t k0 = b < a.B ? a.k_off[b] : 0, k1 = b < a.B ? a.k_off[b + 1] : 0;
+      const int q0 = b < a.B ? a.q_off[b] : 0;
+      const int mb = b < a.B ? a.q_off[b + 1] - q0 : 0;
+      // the row's sequence must exist, lie inside K, fit this plan's slices
+      // (N_b <= max_keys) and have 1 <= m_b <= min(4, N_b): otherwise its
+      // partial lists stay empty and the call reports an invalid argument
+      if (b >= a.B || k0 < 0 || k1 - k0 < 1 || k1 > a.total_keys || k1 - k0 > (int64_t)a.splits * a.keys_per_split ||
+          q0 < 0 || qrow < q0 || mb < 1 || mb > 4 || (int64_t)mb > k1 - k0) {
+        if (tid == 0) {
+          report_error(a.status, DSA_ERR_INVALID_ARG, 7);
+          a.out_cnt[(int64_t)qrow * a.splits + sp] = 0;
+        }
+        continue;
+      }
+      const int j = qrow - q0;
       const int nb = (int)(k1 - k0);
       row = qrow;
       pos = (int64_t)nb - mb + j;

@@ -24,45 +24,31 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices];  // device address of g_static_scratch, per device
+// Device address of g_static_scratch per device, with the context it was
+// resolved in: a device reset makes a new context (and loads the module
+// again), so the address is resolved once per device and context.
+void* g_scratch_ptr[kMaxDevices];
+CUcontext g_scratch_ctx[kMaxDevices];
 
-// Once per device, with that device current: the device address of the
-// array (the host-side name is only a stand-in, not a device address).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// With the device current: the device address of the array (its host-side
+// name is only a stand-in, not a device address).
 int scratch_address(int dev, void** out) {
+  static CtxGetCurrentFn ctx_fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] { ctx_fn = reinterpret_cast<CtxGetCurrentFn>(dsa::driver_entry("cuCtxGetCurrent")); });
+  CUcontext ctx = nullptr;
+  if (!ctx_fn || ctx_fn(&ctx) != CUDA_SUCCESS || ctx == nullptr) return DSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return DSA_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return DSA_OK;
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t inner, uint32_t box_rows) {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  if (!fn) return DSA_ERR_CUDA;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
-             ? DSA_OK
-             : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -79,12 +65,10 @@ extern "C" int dsa_index_dense_static(const void* Q, const float* w, const void*
   if (((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(w)) & 15u) != 0)
     return DSA_ERR_INVALID_ARG;
   if (H != 64 || d != 128) return DSA_ERR_UNSUPPORTED;  // bf16 tensor-core shape only
-  int dev = 0, sms = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  if (major != 10) return DSA_ERR_DEVICE;
+  int dev = 0, sms = 0;
+  int r = dsa::current_device(&dev, &sms);  // compute capability 10.0, as every entry
+  if (r != DSA_OK) return r;
+  if (dev >= kMaxDevices) return DSA_ERR_DEVICE;
 
   // Each CTA of the kernel keeps 4 candidate lists of round_up(N, 512)
   // entries (whole groups of 4 key tiles); the grid shrinks to what the
@@ -98,15 +82,14 @@ extern "C" int dsa_index_dense_static(const void* Q, const float* w, const void*
   if (grid > fit) grid = (int)fit;
 
   void* base = nullptr;
-  int r = scratch_address(dev, &base);
-  if (r != DSA_OK) return r;
+  if ((r = scratch_address(dev, &base)) != DSA_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word must start at zero; candidate lists need no clearing
   if (cudaMemsetAsync(base, 0, 256, st) != cudaSuccess) return DSA_ERR_CUDA;
 
   CUtensorMap tmQ, tmK;
-  if ((r = encode_bf16_map(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
-  if ((r = encode_bf16_map(&tmK, K, (uint64_t)N, (uint64_t)d, 128)) != DSA_OK) return r;
+  if ((r = dsa::make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
+  if ((r = dsa::make_map_bf16(&tmK, K, (uint64_t)N, (uint64_t)d, 128)) != DSA_OK) return r;
   dsa::TcArgs a;
   memset(&a, 0, sizeof(a));
   a.kind = 0;

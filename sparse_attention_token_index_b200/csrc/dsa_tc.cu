@@ -176,23 +176,26 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
     const int64_t k0 = a.k_off[b], k1 = a.k_off[b + 1];
     // no query offsets: one query row per sequence (decode proxies)
     const int q0 = a.q_off ? a.q_off[b] : b, q1 = a.q_off ? a.q_off[b + 1] : b + 1;
-    const int nb = (int)(k1 - k0);
-    u.row0 = q0;
-    u.nq = q1 - q0;
+    // the sequence must lie inside K and Q, fit this plan's slices
+    // (N_b <= max_keys) and have 1 <= m_b <= min(4, N_b); otherwise the unit
+    // does nothing and the call reports an invalid argument
+    const int64_t nb64 = k1 - k0;
+    const bool seq_ok = k0 >= 0 && nb64 >= 1 && k1 <= a.total_keys &&
+                        nb64 <= (int64_t)a.splits * a.tiles_per_split * kTileKeys && q0 >= 0 && q1 <= a.n_rows &&
+                        q1 - q0 >= 1 && q1 - q0 <= kQB && (int64_t)(q1 - q0) <= nb64;
+    const int nb = seq_ok ? (int)nb64 : 0;
+    u.row0 = seq_ok ? q0 : 0;
+    u.nq = seq_ok ? q1 - q0 : 0;
     const int tiles_b = (nb + kTileKeys - 1) / kTileKeys;
     const int t0 = min(tiles_b, sp * a.tiles_per_split);
     const int t1 = min(tiles_b, t0 + a.tiles_per_split);
-    u.key_row0 = (int)k0;
+    u.key_row0 = seq_ok ? (int)k0 : 0;
     u.tile0 = t0;
     u.ntiles = t1 - t0;
     u.nkeys = nb;
     u.seq_split = sp;
     u.partial = 1;
-    if (u.nq < 1 || u.nq > kQB || u.nq > nb) {  // 1 <= m_b <= min(4, N_b) is required
-      if (threadIdx.x == 0) report_error(a.status, DSA_ERR_INTERNAL, 3);
-      u.nq = 0;
-      u.ntiles = 0;
-    }
+    if (!seq_ok && threadIdx.x == 0) report_error(a.status, DSA_ERR_INVALID_ARG, 3);
   } else {
     // group refine: members of group g against the group's gathered bank
     const int unit = a.n_units - 1 - v;
@@ -202,15 +205,16 @@ __device__ __forceinline__ bool unit_at(const TcArgs& a, int round, UnitInfo& u)
       // decode groups: group g is sequence g, its queries at N_g - m_g + j,
       // its bank indices local to the sequence
       const int q0 = a.q_off[g], q1 = a.q_off[g + 1];
-      const int nb = (int)(a.k_off[g + 1] - a.k_off[g]);
-      u.row0 = q0 + mbk * kQB;
-      u.nq = max(0, min(kQB, q1 - u.row0));
-      u.pos0 = nb - (q1 - q0) + (u.row0 - q0);
+      const int64_t k0 = a.k_off[g], k1 = a.k_off[g + 1];
+      const bool seq_ok = k0 >= 0 && k1 - k0 >= 1 && k1 <= a.total_keys && q0 >= 0 && q1 <= a.T &&
+                          q1 - q0 >= 1 && q1 - q0 <= kQB * a.mblocks && (int64_t)(q1 - q0) <= k1 - k0;
+      const int nb = seq_ok ? (int)(k1 - k0) : 0;
+      u.row0 = seq_ok ? q0 + mbk * kQB : 0;
+      u.nq = seq_ok ? max(0, min(kQB, q1 - u.row0)) : 0;
+      u.pos0 = seq_ok ? nb - (q1 - q0) + (u.row0 - q0) : 0;
       nbk = min(a.bank, nb);
-      if (q1 - q0 < 1 || q1 - q0 > kQB * a.mblocks || q1 - q0 > nb) {  // 1 <= m_b <= min(4, N_b) is required
-        if (threadIdx.x == 0) report_error(a.status, DSA_ERR_INTERNAL, 4);
-        u.nq = 0;
-      }
+      // 1 <= m_b <= min(4, N_b), sequence inside K and Q: else no work, invalid argument
+      if (!seq_ok && threadIdx.x == 0) report_error(a.status, DSA_ERR_INVALID_ARG, 4);
     } else {
       const int r_end = min(a.T, (g + 1) * a.group);
       u.row0 = g * a.group + mbk * kQB;
@@ -302,6 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // access (a detour through an integer address would make them generic)
   TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (offsets_bad(a.offsets_ok)) return;  // the whole CTA, before any barrier or TMEM
   volatile int* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {

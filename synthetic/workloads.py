@@ -55,6 +55,7 @@ class DenseInputs:
     q_pos0: int                # query row t sits at key position q_pos0 + t
     q_dtype: str
     k_dtype: str
+    needles: Optional[torch.Tensor] = None  # [n] int64 (host): positions of planted keys, ascending
 
 
 @dataclass
@@ -67,6 +68,7 @@ class DecodeInputs:
     q_offsets: torch.Tensor    # [B+1] int32 (host)
     q_dtype: str
     k_dtype: str
+    needles: Optional[torch.Tensor] = None  # [n] int64 (host): planted key rows of K, ascending
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -158,20 +160,24 @@ def make_dense_inputs(cfg: str | dict, device="cpu", T: Optional[int] = None,
     g = _gen(device, seed)
     kind = c["kind"]
     k_scale = None
+    needles = None
     if kind == "planted":
         sig = 1.0 / math.sqrt(d)
         u = _unit(_randn(g, (d,), device))
         kf = _randn(g, (N, d), device) * sig
         qf = _randn(g, (T, H, d), device) * sig
         # 16 planted keys (and query rows) per 256-position block, +3 sigma along u.
+        planted = []
         for arr, n in ((kf, N), (qf, T)):
             for b0 in range(0, n, 256):
                 nb = min(256, n - b0)
                 pick = torch.randperm(nb, generator=g, device=device)[:min(16, nb)] + b0
                 if arr.dim() == 2:
                     arr[pick] += 3.0 * sig * u
+                    planted.append(pick)
                 else:
                     arr[pick] += 3.0 * sig * u[None, :]
+        needles = torch.sort(torch.cat(planted)).values
         w = torch.rand((T, H), generator=g, device=device, dtype=torch.float32)
         q = _cast(qf, qd)
         k = _cast(kf, kd)
@@ -197,6 +203,7 @@ def make_dense_inputs(cfg: str | dict, device="cpu", T: Optional[int] = None,
         u = _unit(q[rows].float().sum(dim=(0, 1)))
         pos = torch.randperm(N, generator=g, device=device)[:nneedle]
         kf[pos] += 4.0 * sig * u
+        needles = torch.sort(pos).values
         w = torch.rand((T, H), generator=g, device=device, dtype=torch.float32)
         if kd == "fp8":
             k, k_scale = encode_e4m3(kf)
@@ -205,7 +212,8 @@ def make_dense_inputs(cfg: str | dict, device="cpu", T: Optional[int] = None,
     else:
         raise ValueError(f"not a prefill recipe: {kind}")
     return DenseInputs(q=q.contiguous(), w=w.contiguous(), k=k, k_scale=k_scale,
-                       q_pos0=int(q_pos0), q_dtype=qd, k_dtype=kd)
+                       q_pos0=int(q_pos0), q_dtype=qd, k_dtype=kd,
+                       needles=None if needles is None else needles.to("cpu", torch.int64))
 
 
 def make_decode_inputs(cfg: str | dict = "decode_bf16_32x128k", device="cpu",
@@ -236,12 +244,14 @@ def make_decode_inputs(cfg: str | dict = "decode_bf16_32x128k", device="cpu",
     qf = _randn(g, (Mtot, H, d), device) * sig
     kf = torch.empty((Ntot, d), device=device, dtype=torch.float32)
     ko, qo = 0, 0
+    planted = []
     for nb, mb in zip(lengths, ms):
         kb = _randn(g, (nb, d), device) * sig
         u = _unit(qf[qo:qo + mb].sum(dim=(0, 1)))
         npl = max(1, int(round(0.01 * nb)))
         pos = torch.randperm(nb, generator=g, device=device)[:npl]
         kb[pos] += 4.0 * sig * u
+        planted.append(torch.sort(pos).values + ko)
         kf[ko:ko + nb] = kb
         ko += nb
         qo += mb
@@ -256,4 +266,5 @@ def make_decode_inputs(cfg: str | dict = "decode_bf16_32x128k", device="cpu",
     q_off = torch.zeros(B + 1, dtype=torch.int32)
     q_off[1:] = torch.cumsum(torch.tensor(ms, dtype=torch.int64), 0).to(torch.int32)
     return DecodeInputs(q=_cast(qf, qd), w=w.contiguous(), k=k, k_scale=k_scale,
-                        k_offsets=k_off, q_offsets=q_off, q_dtype=qd, k_dtype=kd)
+                        k_offsets=k_off, q_offsets=q_off, q_dtype=qd, k_dtype=kd,
+                        needles=torch.cat(planted).to("cpu", torch.int64))

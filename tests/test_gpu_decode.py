@@ -75,10 +75,11 @@ def test_decode_matches_dense_tail():
         assert set(a[t].tolist()) == set(b[t].tolist())
 
 
-def test_decode_full_size_sampled():
-    # 32 caches x 131072 keys, 2 queries each, k = 2048; 8 sampled rows
+def test_decode_full_size_all_rows():
+    # 32 caches x 131072 keys, 2 queries each, k = 2048: every one of the 64 rows
     inp = make_decode_inputs(device=DEV)
-    _check(inp, 2048, rows=[0, 1, 17, 30, 41, 50, 62, 63], what="decode 32x128K")
+    assert int(inp.q_offsets[-1]) == 64
+    _check(inp, 2048, rows=None, what="decode 32x128K")
 
 
 def test_decode_fp8_keys_tensor_core():

@@ -10,7 +10,7 @@ import torch
 
 import sparse_attention_token_index_b200 as dsa
 from oracle import dsa_oracle as O
-from parity import check_row
+from parity import check_group_sample, check_row, sample_groups
 from synthetic import make_dense_inputs
 
 pytestmark = pytest.mark.gpu
@@ -126,36 +126,23 @@ def test_group_without_bank_output(mode, shape):
     _same_rows(fi, fv, pi, pv)
 
 
-def test_group_full_size_sampled():
-    # the 128K group workload (G = 64, B = 8192, k = 2048), sampled groups
+@pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
+def test_group_full_size_sampled(mode):
+    # the 128K group workload (G = 64, B = 8192, k = 2048) at full size: eight
+    # whole groups in adjacent pairs (512 members, group boundaries included)
     inp = make_dense_inputs("group_bf16_128k", device=DEV)
     G, B, k = 64, 8192, 2048
     T = inp.q.shape[0]
-    for mode in (0, 1):
-        idx, val, bidx, bval, pq, pw = _run_group(inp, k, G, B, mode)
-        # the bench's call (no bank output) gives the same member sets
-        pi, pv = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0, check=True)
-        _same_rows(idx, val, pi, pv)
-        del pi, pv
-        K = _f64(inp.k)
-        gq, gw = _f64(pq), _f64(pw)
-        bi, bv = bidx.cpu().numpy(), bval.cpu().numpy()
-        gi, gv = idx.cpu().numpy(), val.cpu().numpy()
-        for g in [0, 1, 31, 1000, T // G - 1]:
-            L = inp.q_pos0 + min(T, (g + 1) * G) - 1
-            ps = O.score_rows(gq[g:g + 1], gw[g:g + 1], K[:L + 1])[0]
-            check_row(bi[g], bv[g], ps, B, what=f"bank g={g}")
-            bank = bi[g][bi[g] >= 0].astype(np.int64)
-            for t in (g * G, g * G + 37, min(T, (g + 1) * G) - 1):
-                p = inp.q_pos0 + t
-                cand = bank[bank <= p]
-                if mode == 0:
-                    q = inp.q[t:t + 1].double().cpu().numpy()
-                    w = inp.w[t:t + 1].double().cpu().numpy()
-                    S = O.score_rows(q, w, K[:p + 1])[0]
-                    check_row(gi[t], gv[t], S[cand], k, what=f"refine t={t}", idx_map=cand)
-                else:
-                    check_row(gi[t], gv[t], ps[cand], k, what=f"reuse t={t}", idx_map=cand)
+    idx, val, bidx, bval = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0,
+                                               return_bank=True, check=True)
+    # the bench's call (no bank output) gives the same member sets
+    pi, pv = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=mode, q_pos0=inp.q_pos0, check=True)
+    _same_rows(idx, val, pi, pv)
+    del pi, pv
+    groups = sample_groups(T // G, G, q_pos0=inp.q_pos0, seed=3)
+    assert len(groups) == 8 and groups[0] == 0 and groups[-1] == T // G - 1
+    check_group_sample(inp.q, inp.w, _f64(inp.k), idx.cpu().numpy(), val.cpu().numpy(), bidx.cpu().numpy(),
+                       bval.cpu().numpy(), groups, G, B, k, mode, inp.q_pos0, "bf16", what=f"128K mode {mode}")
 
 
 @pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])
@@ -182,23 +169,16 @@ def test_group_fp8_keys(mode):
 
 
 def test_refine_local_full_size_sampled():
-    # the 128K group workload with query-specific additions, sampled groups
+    # the 128K group workload with query-specific additions: eight whole groups
     inp = make_dense_inputs("group_bf16_128k", device=DEV)
     G, B, k = 64, 8192, 2048
     T = inp.q.shape[0]
     idx, val, bidx, bval = dsa.dsa_index_group(inp.q, inp.w, inp.k, k, G, B, mode=dsa.DSA_GROUP_REFINE_LOCAL,
                                                q_pos0=inp.q_pos0, return_bank=True, check=True)
-    K = _f64(inp.k)
-    bi, gi, gv = bidx.cpu().numpy(), idx.cpu().numpy(), val.cpu().numpy()
-    for g in [0, 777, T // G - 1]:
-        bank = bi[g][bi[g] >= 0].astype(np.int64)
-        for t in (g * G, g * G + 40, min(T, (g + 1) * G) - 1):
-            p = inp.q_pos0 + t
-            cand = np.union1d(bank[bank <= p], np.arange(inp.q_pos0 + g * G, p + 1))
-            q = inp.q[t:t + 1].double().cpu().numpy()
-            w = inp.w[t:t + 1].double().cpu().numpy()
-            S = O.score_rows(q, w, K[:p + 1])[0]
-            check_row(gi[t], gv[t], S[cand], k, what=f"refine_local t={t}", idx_map=cand)
+    groups = sample_groups(T // G, G, q_pos0=inp.q_pos0, seed=4)
+    check_group_sample(inp.q, inp.w, _f64(inp.k), idx.cpu().numpy(), val.cpu().numpy(), bidx.cpu().numpy(),
+                       bval.cpu().numpy(), groups, G, B, k, O.REFINE_LOCAL, inp.q_pos0, "bf16",
+                       what="128K refine_local")
 
 
 @pytest.mark.parametrize("mode", [0, 1], ids=["refine", "reuse"])

@@ -59,3 +59,21 @@ def test_decode_recipe():
     assert x.k.shape == (1317, 64) and x.q.shape == (6, 8, 64)
     assert x.k_offsets.tolist() == [0, 300, 317, 1317]
     assert x.q_offsets.tolist() == [0, 2, 3, 6]
+
+
+def test_needle_positions_reported():
+    # the recipes report where they planted keys (data for choosing parity rows)
+    x = make_dense_inputs("fp8_256k", T=512, N=4000)
+    n = x.needles.numpy()
+    assert n.shape == (20,) and np.all(np.diff(n) > 0) and n[0] >= 0 and n[-1] < 4000
+    y = make_decode_inputs(lengths=[300, 17, 1000], m=[2, 1, 3], H=8, d=64)
+    ny = y.needles.numpy()
+    assert ny.shape == (3 + 1 + 10,)
+    assert np.all((ny[:3] < 300)) and ny[3] in range(300, 317) and np.all((ny[4:] >= 317) & (ny[4:] < 1317))
+    z = make_dense_inputs("tiny_fp32_2k", T=512, N=512)
+    assert z.needles.shape == (32,)                     # 16 keys per 256-position block
+    assert make_dense_inputs("dense_bf16_32k", T=64, N=256).needles is None
+    # the planted decode keys lean along the sequence's query direction
+    u = y.q[:2].float().sum(dim=(0, 1))
+    proj = (y.k[:300].float() @ (u / u.norm())).numpy()
+    assert proj[ny[:3]].min() > np.median(proj)

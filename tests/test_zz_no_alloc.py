@@ -17,7 +17,8 @@ import pytest
 import torch
 
 import sparse_attention_token_index_b200 as dsa
-from parity import RTOL
+from oracle import dsa_oracle as O
+from parity import RTOL, check_rows
 from synthetic import make_dense_inputs
 
 pytestmark = pytest.mark.gpu
@@ -60,6 +61,10 @@ def test_static_scratch_matches_workspace_entry_point_twice():
         si, sv = _static_call(inp.q, inp.w, inp.k, c["k"], inp.q_pos0)
         ri, rv = dsa.dsa_index_dense(inp.q, inp.w, inp.k, c["k"], q_pos0=inp.q_pos0, check=True)
         _same(si, sv, ri, rv)
+        # and against the CPU oracle itself, every row
+        r = O.dense(inp.q.double().cpu().numpy(), inp.w.double().cpu().numpy(), inp.k.double().cpu().numpy(),
+                    c["k"], q_pos0=inp.q_pos0, return_scores=True)
+        check_rows(si.cpu().numpy(), sv.cpu().numpy(), r["scores"], c["k"], what="static entry")
 
 
 def test_static_scratch_rejects_oversize():
