@@ -38,6 +38,7 @@ from ._binding import (  # noqa: F401
     dsa_kernel_timer_start,
     dsa_kernel_timer_stop,
     dsa_check_status,
+    dsa_debug_set_wait,
     dense_workspace_bytes,
     group_workspace_bytes,
     decode_workspace_bytes,

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.environ.get("DSA_LIB") or os.path.join(_HERE, "libdsa_index.so")
 
 EXPORTED_SYMBOLS = (
-    "dsa_status_string", "dsa_version", "dsa_check_status",
+    "dsa_status_string", "dsa_version", "dsa_check_status", "dsa_debug_set_wait",
     "dsa_index_dense_workspace_size", "dsa_index_dense",
     "dsa_index_group_workspace_size", "dsa_index_group",
     "dsa_index_decode_workspace_size", "dsa_index_decode",
@@ -49,6 +49,7 @@ _c_int, _c_i64, _c_sz, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctyp
 _SIGS = {
     "dsa_status_string": (ctypes.c_char_p, [_c_int]),
     "dsa_version": (_c_int, []),
+    "dsa_debug_set_wait": (_c_int, [ctypes.c_uint, _c_int]),
     "dsa_check_status": (_c_int, [_vp, _vp]),
     "dsa_index_dense_workspace_size": (_c_int, [_c_int] * 7 + [ctypes.POINTER(_c_sz)]),
     "dsa_index_dense": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_i64, _c_int, _c_int,
@@ -198,6 +199,15 @@ def decode_workspace_bytes(B, total_q, max_keys, H, d, k, q_dtype, k_dtype) -> i
 def dsa_check_status(workspace: torch.Tensor, stream=None) -> None:
     """Waits for the stream and raises if a kernel recorded a device-side failure."""
     _check(lib().dsa_check_status(_ptr(workspace), _stream(stream)), "device status")
+
+
+def dsa_debug_set_wait(polls: int = 0, hold_first_tile: bool = False) -> None:
+    """Failure-path control for tests: the poll budget of the tensor-core
+    kernel's inter-role waits (0 = the default, about a second) and, with
+    ``hold_first_tile``, a first key tile that the first CTA of the next
+    dense-kind launches never loads, so that a wait runs out and the launch
+    reports DSA_ERR_TIMEOUT through the status word.  Process-wide."""
+    _check(lib().dsa_debug_set_wait(int(polls), 1 if hold_first_tile else 0), "dsa_debug_set_wait")
 
 
 def _check_out(idx, val, rows, k):

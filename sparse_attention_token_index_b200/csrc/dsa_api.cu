@@ -279,6 +279,11 @@ const char* dsa_status_string(int status) {
 
 int dsa_version(void) { return 100; }
 
+int dsa_debug_set_wait(unsigned int polls, int hold_first_tile) {
+  set_wait_controls(polls, hold_first_tile);
+  return DSA_OK;
+}
+
 int dsa_check_status(void* workspace, void* stream) {
   if (!workspace) return DSA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

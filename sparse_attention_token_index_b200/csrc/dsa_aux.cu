@@ -77,6 +77,7 @@ __global__ void proxy_mean_kernel(const void* __restrict__ Q, const float* __res
 
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
                       float* wbar, cudaStream_t stream, const int32_t* seg, int nseg, const int* ok) {
+  const NvtxRange nvtx("dsa.proxy_mean");
   const int ng = seg ? nseg : (T + G - 1) / G;
   const int64_t chunks = ((int64_t)H * d + 7) / 8;
   const dim3 grid((unsigned)((chunks + 127) / 128), (unsigned)ng);
@@ -104,6 +105,7 @@ __global__ void block_mean_kernel(const __nv_bfloat16* __restrict__ K, const flo
 }
 
 int launch_block_mean(const void* K, const float* K_scale, int64_t N, int d, void* R, cudaStream_t stream) {
+  const NvtxRange nvtx("dsa.block_mean");
   const int64_t nb = (N + 127) / 128;
   block_mean_kernel<<<(unsigned)nb, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(K), K_scale, N, d,
                                                       static_cast<__nv_bfloat16*>(R));
@@ -131,6 +133,7 @@ __global__ void bank_gather_kernel(const uint4* __restrict__ K, int row_vecs, co
 
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size, void* Kg,
                        cudaStream_t stream, const int64_t* row_off, const int* ok) {
+  const NvtxRange nvtx("dsa.bank_gather");
   const int elt = (k_dtype == DSA_DTYPE_FP32) ? 4 : (k_dtype == DSA_DTYPE_BF16 ? 2 : 1);
   const int row_vecs = d * elt / 16;
   bank_gather_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), row_vecs, bank,
@@ -180,6 +183,7 @@ __global__ void local_extend_kernel(const int32_t* __restrict__ bank, int B, int
 
 int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
                         const int64_t* k_off, int S, int32_t* map, cudaStream_t stream, const int* ok) {
+  const NvtxRange nvtx("dsa.local_extend");
   if (S - B < 1 || S - B > 4096) return DSA_ERR_INVALID_ARG;
   local_extend_kernel<<<ng, 256, (size_t)(S - B) * sizeof(int), stream>>>(bank, B, G, T, q_pos0, q_off, k_off, S,
                                                                           map, ok);
@@ -366,6 +370,7 @@ __global__ void __launch_bounds__(kRankThreads) bank_rank_reuse_kernel(int32_t* 
 int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_size, int G, int T, int64_t q_pos0,
                            int k, int32_t* out_idx, float* out_val, int do_reuse, int rank_all, cudaStream_t stream,
                            const int32_t* q_off, const int64_t* k_off, const int* ok) {
+  const NvtxRange nvtx("dsa.bank_rank_reuse");
   int P = 1;
   while (P < bank_size) P <<= 1;
   if (P > kMaxBank) return DSA_ERR_UNSUPPORTED;
@@ -444,6 +449,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const uint2
 
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
                         float* out_val, int* status, cudaStream_t stream, const int* ok) {
+  const NvtxRange nvtx("dsa.decode_merge");
   if (splits > 256) return DSA_ERR_UNSUPPORTED;
   decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(parts, part_cnt, splits, k, out_idx, out_val, status,
                                                              ok);
@@ -477,6 +483,7 @@ __global__ void decode_offsets_check_kernel(const int64_t* __restrict__ k_off, c
 
 int launch_decode_offsets_check(const int64_t* k_off, const int32_t* q_off, int B, int64_t total_keys, int total_q,
                                 int max_keys, void* workspace, cudaStream_t stream) {
+  const NvtxRange nvtx("dsa.decode_offsets_check");
   decode_offsets_check_kernel<<<1, 256, 0, stream>>>(k_off, q_off, B, total_keys, total_q, max_keys,
                                                      static_cast<WsHeader*>(workspace));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -507,6 +514,7 @@ __global__ void e4m3_to_bf16_kernel(const uint4* __restrict__ src, int64_t n16, 
 }
 
 int launch_e4m3_to_bf16(const uint8_t* src, int64_t n, void* dst, cudaStream_t stream) {
+  const NvtxRange nvtx("dsa.e4m3_to_bf16");
   e4m3_to_bf16_kernel<<<148 * 8, 256, 0, stream>>>(reinterpret_cast<const uint4*>(src), n / 16,
                                                     static_cast<uint4*>(dst));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -519,6 +527,7 @@ __global__ void fill_neg_inf_kernel(float* S, int64_t n) {
 }
 
 int launch_fill_scores(float* S, int64_t n, cudaStream_t stream) {
+  const NvtxRange nvtx("dsa.fill_scores");
   fill_neg_inf_kernel<<<592, 256, 0, stream>>>(S, n);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

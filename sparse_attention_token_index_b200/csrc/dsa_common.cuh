@@ -110,19 +110,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint32_t kWaitPolls = 1u << 22;
 
 // Returns false when the wait gave up (abort raised elsewhere, or the poll
-// budget ran out — then the status word and the abort flag are set).
+// budget `limit` ran out — then the status word and the abort flag are set).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int where) {
+                                          int* status, int where, uint32_t limit = kWaitPolls) {
   const uint32_t a = smem_u32(bar);
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 255u) == 255u) {
       if (*abort_flag) return false;
-      if (it >= kWaitPolls) {
+      if (it >= limit) {
         report_error(status, DSA_ERR_TIMEOUT, where);
         *abort_flag = 1;
         return false;
       }
+    }
+  }
+}
+
+// The wait for work this CTA has already issued (a TMA copy, an MMA) before
+// it leaves: it ignores the abort flag, since a copy in flight must land
+// before the CTA's shared memory is released, and keeps the full budget.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status, int where) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 255u) == 255u && it >= kWaitPolls) {
+      report_error(status, DSA_ERR_TIMEOUT, where);
+      return false;
     }
   }
 }

@@ -3,9 +3,21 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace dsa {
+
+// An NVTX range around one kernel launch on the host, named for the step it
+// runs, so that a profiler's timeline shows candidate scoring, selection,
+// merging and the group steps apart (ADIndex — Deployment Guidance: profile
+// the indexer's parts separately).  Costs a few nanoseconds without a tool.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Largest candidate bank of the group form: the bank ranking holds a whole
 // bank in shared memory (8 bytes per key, 128 KB at this size).
@@ -72,6 +84,11 @@ struct TcArgs {
   const int32_t* ivf_off;
   const int32_t* ivf_tiles;
   int ivf_max_tiles;  // candidate lists hold this many tiles per query
+  // failure-path controls (dsa_debug_set_wait; zero in normal calls): the
+  // poll budget of the waits between roles (0 = the default), and a first
+  // key tile that CTA 0's producer never loads, so that a wait runs out
+  uint32_t wait_polls;
+  int hold_first_tile;
 };
 
 // The current device, checked once: compute capability 10.0 (only sm_100a
@@ -92,6 +109,9 @@ TimerSlot timer_acquire();
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream);
+// dsa_debug_set_wait: poll budget of the tensor-core kernel's inter-role
+// waits (0 = default) and the held first tile of the failure-path test.
+void set_wait_controls(uint32_t polls, int hold_first_tile);
 size_t tc_smem_bytes();
 
 // Exact fp32 CUDA-core path (any H <= 128, d <= 256, H*d <= 8192).

@@ -166,6 +166,7 @@ size_t ivf_build_scratch_bytes(int d, int C) { return (size_t)C * d * 4 + (size_
 
 int ivf_build(const void* K, const float* K_scale, int64_t N, int d, int C, int iters, const IvfIndex& x,
               uint8_t* scratch, cudaStream_t st) {
+  const NvtxRange nvtx("dsa.ivf_build");
   const __nv_bfloat16* Kb = static_cast<const __nv_bfloat16*>(K);
   float* sum = reinterpret_cast<float*>(scratch);
   int32_t* count = reinterpret_cast<int32_t*>(sum + (size_t)C * d);
@@ -188,6 +189,7 @@ int ivf_build(const void* K, const float* K_scale, int64_t N, int d, int C, int 
 }
 
 int launch_ivf_tiles(const int32_t* list, int n_probe, int T, const int32_t* off, int32_t* tiles, cudaStream_t st) {
+  const NvtxRange nvtx("dsa.ivf_tiles");
   ivf_tiles_kernel<<<(T + 255) / 256, 256, 0, st>>>(list, n_probe, T, off, tiles);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

@@ -122,6 +122,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_index_kernel(const SimtArgs
 }
 
 int launch_simt_index(const SimtArgs& a, int grid, cudaStream_t stream) {
+  const NvtxRange nvtx(a.kind == 1 ? "dsa.score_topk.decode.fp32" : "dsa.score_topk.fp32");
   const size_t smem = simt_smem_bytes(a.H, a.d);
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(simt_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (offsets_bad(a.offsets_ok)) return;  // the whole CTA, before any barrier or TMEM
+  const uint32_t polls = a.wait_polls ? a.wait_polls : kWaitPolls;
   volatile int* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
@@ -346,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       UnitInfo u;
       for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
-        if (qi > 0 && !(ok = mbar_wait(&S.q_empty, (qi - 1) & 1, abort_flag, a.status, 10))) break;
+        if (qi > 0 && !(ok = mbar_wait(&S.q_empty, (qi - 1) & 1, abort_flag, a.status, 10, polls))) break;
         mbar_arrive_expect_tx(&S.q_full, (uint32_t)(u.nq * 2 * kQHeadBlockBytes));
         for (int q = 0; q < u.nq; ++q)
           for (int c = 0; c < 2; ++c)
@@ -356,7 +357,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ClusterWalk walk;
         if constexpr (kKind == 4) walk.start(a, u.row0);
         for (int j = 0; j < u.ntiles; ++j) {
-          if (!(ok = mbar_wait(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11))) break;
+          if (!(ok = mbar_wait(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11, polls))) break;
+          if (kKind == 0 && a.hold_first_tile && blockIdx.x == 0 && round == 0 && j == 0) {
+            // failure-path test: this stage is never armed nor loaded, so the
+            // MMA issuer's wait for it runs out
+            if (++s == kStages) {
+              s = 0;
+              ph ^= 1u;
+            }
+            continue;
+          }
           mbar_arrive_expect_tx(&S.k_full[s], (uint32_t)kKStageBytes);
           int row;
           if constexpr (kKind == 4) {
@@ -377,8 +387,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // never leave with a copy in flight
       for (int t = 0; t < kStages; ++t)
-        if ((armed >> t) & 1u) mbar_wait(&S.k_full[t], (armed_ph >> t) & 1u, abort_flag, a.status, 12);
-      if (qi > 0) mbar_wait(&S.q_full, (qi - 1) & 1, abort_flag, a.status, 13);
+        if ((armed >> t) & 1u) mbar_wait_drain(&S.k_full[t], (armed_ph >> t) & 1u, a.status, 12);
+      if (qi > 0) mbar_wait_drain(&S.q_full, (qi - 1) & 1, a.status, 13);
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
@@ -391,13 +401,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       UnitInfo u;
       const uint32_t q_addr = smem_u32(S.q);
       for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
-        if (!(ok = mbar_wait(&S.q_full, qi & 1, abort_flag, a.status, 20))) break;
+        if (!(ok = mbar_wait(&S.q_full, qi & 1, abort_flag, a.status, 20, polls))) break;
         ++qi;
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_f32(128, u.nq * kHeads);
         for (int j = 0; j < u.ntiles; ++j) {
-          if (!(ok = mbar_wait(&S.k_full[s], ph, abort_flag, a.status, 21))) break;
-          if (!(ok = mbar_wait(&S.t_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort_flag, a.status, 22))) break;
+          if (!(ok = mbar_wait(&S.k_full[s], ph, abort_flag, a.status, 21, polls))) break;
+          if (!(ok = mbar_wait(&S.t_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort_flag, a.status, 22, polls))) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
           const uint32_t k_addr = smem_u32(S.k[s]);
@@ -424,7 +434,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // never leave with an MMA in flight
       tc_commit(&S.drain);
-      mbar_wait(&S.drain, 0, abort_flag, a.status, 23);
+      mbar_wait_drain(&S.drain, 0, a.status, 23);
     }
   } else if (warp == kThreshWarp) {
     // ---------------- threshold warp ----------------
@@ -491,7 +501,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ClusterWalk walk;
       if constexpr (kKind == 4) walk.start(a, u.row0);
       for (int jt = 0; jt < ntiles; ++jt) {
-        if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30)) {
+        if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30, polls)) {
           ok = false;
           break;
         }
@@ -595,8 +605,24 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
+// Failure-path controls set by dsa_debug_set_wait (process-wide).
+static std::atomic<uint32_t> g_wait_polls{0};
+static std::atomic<int> g_hold_first_tile{0};
+
+void set_wait_controls(uint32_t polls, int hold_first_tile) {
+  g_wait_polls.store(polls);
+  g_hold_first_tile.store(hold_first_tile ? 1 : 0);
+}
+
+int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& args, int grid,
                     cudaStream_t stream) {
+  static const char* const kNames[5] = {"dsa.score_topk.prefill", "dsa.score_topk.decode",
+                                         "dsa.score_topk.group_refine", "dsa.score_topk.block_refine",
+                                         "dsa.score_topk.ivf_refine"};
+  const NvtxRange nvtx(args.kind >= 0 && args.kind <= 4 ? kNames[args.kind] : "dsa.score_topk");
+  TcArgs a = args;
+  a.wait_polls = g_wait_polls.load();
+  a.hold_first_tile = g_hold_first_tile.load();
   if (a.kind < 0 || a.kind > 4 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
   const TimerSlot ts = timer_acquire();
   if (ts.start) cudaEventRecord(ts.start, stream);

@@ -174,6 +174,8 @@ def test_binding_prototypes_match_the_header():
                 assert t in (C.c_void_p,) or issubclass(t, C._Pointer), (name, p, t)
             elif re.match(r"(const\s+)?(int64_t|size_t)\b", p):
                 assert t in (C.c_int64, C.c_size_t), (name, p, t)
+            elif re.match(r"unsigned\s+int\b", p):
+                assert t is C.c_uint, (name, p, t)
             else:
                 assert t is C.c_int, (name, p, t)
 
