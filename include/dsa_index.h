@@ -88,15 +88,16 @@ int dsa_version(void);
  * Every wait of the tensor-core kernel is bounded: when it runs out, the
  * kernel records DSA_ERR_TIMEOUT in the status word, lets the copies and MMAs
  * it already issued land, frees its tensor memory and returns, so the device
- * stays usable.  `polls` sets the budget of the waits between the kernel's
- * roles for the tensor-core launches that follow (0 restores the default of
- * about a second; the final drain of issued work always keeps the default).
+ * stays usable.  `budget_us` sets the time budget, in microseconds, of the
+ * waits between the kernel's roles for the tensor-core launches that follow
+ * (0 restores the default of 2 s; the final drain of issued work always
+ * keeps the default).
  * With `hold_first_tile` nonzero, the first CTA of the following dense-kind
  * launches never loads its first key tile, so the wait for it runs out and
  * that launch reports DSA_ERR_TIMEOUT (its outputs are then unspecified).
  * Process-wide, read at each launch; call it between calls, never while
  * another thread launches.  Returns DSA_OK. */
-int dsa_debug_set_wait(unsigned int polls, int hold_first_tile);
+int dsa_debug_set_wait(unsigned int budget_us, int hold_first_tile);
 
 /* Synchronises `stream`, then reads and clears the device status word kept
  * in `workspace`.  Returns DSA_OK, the recorded DSA_ERR_TIMEOUT,

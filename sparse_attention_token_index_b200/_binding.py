@@ -201,13 +201,13 @@ def dsa_check_status(workspace: torch.Tensor, stream=None) -> None:
     _check(lib().dsa_check_status(_ptr(workspace), _stream(stream)), "device status")
 
 
-def dsa_debug_set_wait(polls: int = 0, hold_first_tile: bool = False) -> None:
-    """Failure-path control for tests: the poll budget of the tensor-core
-    kernel's inter-role waits (0 = the default, about a second) and, with
+def dsa_debug_set_wait(budget_us: int = 0, hold_first_tile: bool = False) -> None:
+    """Failure-path control for tests: the time budget in microseconds of the
+    tensor-core kernel's inter-role waits (0 = the default, 2 s) and, with
     ``hold_first_tile``, a first key tile that the first CTA of the next
     dense-kind launches never loads, so that a wait runs out and the launch
     reports DSA_ERR_TIMEOUT through the status word.  Process-wide."""
-    _check(lib().dsa_debug_set_wait(int(polls), 1 if hold_first_tile else 0), "dsa_debug_set_wait")
+    _check(lib().dsa_debug_set_wait(int(budget_us), 1 if hold_first_tile else 0), "dsa_debug_set_wait")
 
 
 def _check_out(idx, val, rows, k):

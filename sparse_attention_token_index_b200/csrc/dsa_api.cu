@@ -279,8 +279,8 @@ const char* dsa_status_string(int status) {
 
 int dsa_version(void) { return 100; }
 
-int dsa_debug_set_wait(unsigned int polls, int hold_first_tile) {
-  set_wait_controls(polls, hold_first_tile);
+int dsa_debug_set_wait(unsigned int budget_us, int hold_first_tile) {
+  set_wait_controls(budget_us, hold_first_tile);
   return DSA_OK;
 }
 

@@ -2,9 +2,10 @@
 //
 // PTX wrappers for mbarriers, TMA tile loads and tcgen05 (TMEM allocation,
 // MMA issue, commit, TMEM loads), order-preserving float keys, and the
-// bounded-wait error protocol: every spin on an mbarrier gives up after a
-// fixed number of polls, records DSA_ERR_TIMEOUT in the workspace status word
-// and raises a per-CTA abort flag so that all roles leave their loops.
+// bounded-wait error protocol: a wait on an mbarrier sleeps in the hardware
+// until the phase completes and gives up after a time budget, records
+// DSA_ERR_TIMEOUT in the workspace status word and raises a per-CTA abort
+// flag so that all roles leave their loops.
 #pragma once
 
 #include <cuda.h>
@@ -92,37 +93,61 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Longest single suspension of a waiting thread when the wait is far off the
+// critical path (the TMA producer, drains): try_wait sleeps until the phase
+// completes or this many nanoseconds pass, so the warp takes no issue slots
+// meanwhile.  Waits on the critical path use the plain form, whose short
+// hardware suspension wakes sooner.
+constexpr uint32_t kSuspendNs = 20000;
+
+template <bool kLongSleep>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (kLongSleep) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
-// Poll budget of one bounded wait.  try_wait suspends for a short hardware
-// time slice per poll, so 2^22 polls last well beyond any legitimate wait of
-// these kernels (microseconds) and still end in about a second.
-constexpr uint32_t kWaitPolls = 1u << 22;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
-// Returns false when the wait gave up (abort raised elsewhere, or the poll
-// budget `limit` ran out — then the status word and the abort flag are set).
+// Time budget of one bounded wait: far beyond any legitimate wait of these
+// kernels (microseconds), short enough that a failure returns promptly.
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+// Returns false when the wait gave up (abort raised elsewhere, or the
+// `budget_ns` ran out — then the status word and the abort flag are set).
+template <bool kLongSleep = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int where, uint32_t limit = kWaitPolls) {
+                                          int* status, int where, uint64_t budget_ns = kWaitNs) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (*abort_flag) return false;
-      if (it >= limit) {
-        report_error(status, DSA_ERR_TIMEOUT, where);
-        *abort_flag = 1;
-        return false;
-      }
+  if (mbar_try_wait<kLongSleep>(a, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait<kLongSleep>(a, parity)) return true;
+    if (global_ns() - t0 > budget_ns) {
+      report_error(status, DSA_ERR_TIMEOUT, where);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -132,9 +157,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // before the CTA's shared memory is released, and keeps the full budget.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* status, int where) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((it & 255u) == 255u && it >= kWaitPolls) {
+  if (mbar_try_wait<true>(a, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait<true>(a, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) {
       report_error(status, DSA_ERR_TIMEOUT, where);
       return false;
     }

@@ -85,9 +85,9 @@ struct TcArgs {
   const int32_t* ivf_tiles;
   int ivf_max_tiles;  // candidate lists hold this many tiles per query
   // failure-path controls (dsa_debug_set_wait; zero in normal calls): the
-  // poll budget of the waits between roles (0 = the default), and a first
-  // key tile that CTA 0's producer never loads, so that a wait runs out
-  uint32_t wait_polls;
+  // time budget of the waits between roles in ns (0 = the default), and a
+  // first key tile that CTA 0's producer never loads, so that a wait runs out
+  uint64_t wait_ns;
   int hold_first_tile;
 };
 
@@ -109,9 +109,9 @@ TimerSlot timer_acquire();
 
 int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid,
                     cudaStream_t stream);
-// dsa_debug_set_wait: poll budget of the tensor-core kernel's inter-role
-// waits (0 = default) and the held first tile of the failure-path test.
-void set_wait_controls(uint32_t polls, int hold_first_tile);
+// dsa_debug_set_wait: time budget (microseconds) of the tensor-core kernel's
+// inter-role waits (0 = default) and the held first tile of the failure-path test.
+void set_wait_controls(uint32_t budget_us, int hold_first_tile);
 size_t tc_smem_bytes();
 
 // Exact fp32 CUDA-core path (any H <= 128, d <= 256, H*d <= 8192).
@@ -153,12 +153,12 @@ size_t simt_smem_bytes(int H, int d);
 int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G, int q_dtype, void* qbar,
                       float* wbar, cudaStream_t stream, const int32_t* seg = nullptr, int nseg = 0,
                       const int* ok = nullptr);
-// row_off (decode): bank indices are local to sequence g, whose rows start at row_off[g].
-int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
-                       void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr, const int* ok = nullptr);
 // rank_all: sort and write back the whole bank; otherwise only the top
 // k + G - 1 entries are ranked (enough for Reuse) and the bank is not written.
 // Refine with query-specific additions: map [ng, S] = bank (B) + own stretch (S - B).
+// row_off (decode): bank indices are local to sequence g, whose rows start at row_off[g].
+int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
+                       void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr, const int* ok = nullptr);
 int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
                         const int64_t* k_off, int S, int32_t* map, cudaStream_t stream, const int* ok = nullptr);
 // q_off / k_off (decode): group g is sequence g with members q_off[g] ..

@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (offsets_bad(a.offsets_ok)) return;  // the whole CTA, before any barrier or TMEM
-  const uint32_t polls = a.wait_polls ? a.wait_polls : kWaitPolls;
+  const uint64_t budget = a.wait_ns ? a.wait_ns : kWaitNs;  // budget of the inter-role waits
   volatile int* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       UnitInfo u;
       for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
-        if (qi > 0 && !(ok = mbar_wait(&S.q_empty, (qi - 1) & 1, abort_flag, a.status, 10, polls))) break;
+        if (qi > 0 && !(ok = mbar_wait<true>(&S.q_empty, (qi - 1) & 1, abort_flag, a.status, 10, budget))) break;
         mbar_arrive_expect_tx(&S.q_full, (uint32_t)(u.nq * 2 * kQHeadBlockBytes));
         for (int q = 0; q < u.nq; ++q)
           for (int c = 0; c < 2; ++c)
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ClusterWalk walk;
         if constexpr (kKind == 4) walk.start(a, u.row0);
         for (int j = 0; j < u.ntiles; ++j) {
-          if (!(ok = mbar_wait(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11, polls))) break;
+          if (!(ok = mbar_wait<true>(&S.k_empty[s], ph ^ 1u, abort_flag, a.status, 11, budget))) break;
           if (kKind == 0 && a.hold_first_tile && blockIdx.x == 0 && round == 0 && j == 0) {
             // failure-path test: this stage is never armed nor loaded, so the
             // MMA issuer's wait for it runs out
@@ -401,13 +401,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       UnitInfo u;
       const uint32_t q_addr = smem_u32(S.q);
       for (int round = 0; ok && unit_at<kKind>(a, round, u); ++round) {
-        if (!(ok = mbar_wait(&S.q_full, qi & 1, abort_flag, a.status, 20, polls))) break;
+        if (!(ok = mbar_wait(&S.q_full, qi & 1, abort_flag, a.status, 20, budget))) break;
         ++qi;
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_f32(128, u.nq * kHeads);
         for (int j = 0; j < u.ntiles; ++j) {
-          if (!(ok = mbar_wait(&S.k_full[s], ph, abort_flag, a.status, 21, polls))) break;
-          if (!(ok = mbar_wait(&S.t_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort_flag, a.status, 22, polls))) break;
+          if (!(ok = mbar_wait(&S.k_full[s], ph, abort_flag, a.status, 21, budget))) break;
+          if (!(ok = mbar_wait(&S.t_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort_flag, a.status, 22, budget))) break;
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
           const uint32_t k_addr = smem_u32(S.k[s]);
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ClusterWalk walk;
       if constexpr (kKind == 4) walk.start(a, u.row0);
       for (int jt = 0; jt < ntiles; ++jt) {
-        if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30, polls)) {
+        if (!mbar_wait(&S.t_full[buf], (eph >> buf) & 1u, abort_flag, a.status, 30, budget)) {
           ok = false;
           break;
         }
@@ -606,11 +606,11 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
 }
 
 // Failure-path controls set by dsa_debug_set_wait (process-wide).
-static std::atomic<uint32_t> g_wait_polls{0};
+static std::atomic<uint32_t> g_wait_us{0};
 static std::atomic<int> g_hold_first_tile{0};
 
-void set_wait_controls(uint32_t polls, int hold_first_tile) {
-  g_wait_polls.store(polls);
+void set_wait_controls(uint32_t budget_us, int hold_first_tile) {
+  g_wait_us.store(budget_us);
   g_hold_first_tile.store(hold_first_tile ? 1 : 0);
 }
 
@@ -621,7 +621,7 @@ int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs
                                          "dsa.score_topk.ivf_refine"};
   const NvtxRange nvtx(args.kind >= 0 && args.kind <= 4 ? kNames[args.kind] : "dsa.score_topk");
   TcArgs a = args;
-  a.wait_polls = g_wait_polls.load();
+  a.wait_ns = (uint64_t)g_wait_us.load() * 1000u;
   a.hold_first_tile = g_hold_first_tile.load();
   if (a.kind < 0 || a.kind > 4 || (a.dbg_scores != nullptr && a.kind != 0)) return DSA_ERR_INVALID_ARG;
   const TimerSlot ts = timer_acquire();

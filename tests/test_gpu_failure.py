@@ -32,7 +32,7 @@ def test_wait_runs_out_then_device_serves_a_normal_call():
     inp = make_dense_inputs("dense_bf16_32k", device=DEV, T=64, N=4096, seed=61)
     k = 64
     ws = torch.zeros(dsa.dense_workspace_bytes(64, 4096, 64, 128, k, 0, 0), dtype=torch.uint8, device=DEV)
-    dsa.dsa_debug_set_wait(1 << 12, hold_first_tile=True)   # about a millisecond
+    dsa.dsa_debug_set_wait(1000, hold_first_tile=True)   # a millisecond
     try:
         dsa.dsa_index_dense(inp.q, inp.w, inp.k, k, q_pos0=inp.q_pos0, workspace=ws)
         with pytest.raises(dsa.DsaError) as e:
@@ -47,9 +47,9 @@ def test_wait_runs_out_then_device_serves_a_normal_call():
 
 
 def test_short_budget_alone_keeps_results():
-    # a budget of a few milliseconds is far above any wait of a working launch
+    # a budget of 20 ms is far above any wait of a working launch
     inp = make_dense_inputs("dense_bf16_32k", device=DEV, T=130, N=2000, seed=62)
-    dsa.dsa_debug_set_wait(1 << 14)
+    dsa.dsa_debug_set_wait(20000)
     try:
         idx, val = dsa.dsa_index_dense(inp.q, inp.w, inp.k, 100, q_pos0=inp.q_pos0, check=True)
     finally:
