@@ -534,7 +534,7 @@ struct DecodePlan {
   int grid;
   int64_t cand_cap;
   int splits, tiles_per_split;
-  size_t cand_off, ppair_off, pcnt_off, total;
+  size_t cand_off, ppair_off, pcnt_off, hdr_off, hist_off, total;
 };
 
 void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, int max_keys, int H, int d, int k,
@@ -565,7 +565,14 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
     p.cand_cap = (int64_t)((p.tiles_per_split + 3) / 4 * 4) * 128;
     const int64_t units = (int64_t)B * p.splits;
     p.grid = units < di.sms ? (int)units : di.sms;
-    p.cand_off = L.take((size_t)p.grid * 4 * p.cand_cap * sizeof(uint2));
+    // every (row, slice) keeps its whole candidate list, segment header and
+    // histogram for the merge
+    const size_t lists = (size_t)total_q * p.splits;
+    p.cand_off = L.take(lists * p.cand_cap * sizeof(uint2));
+    p.hdr_off = L.take(lists * kSegHdr * sizeof(int));
+    p.hist_off = L.take(lists * kBins * sizeof(uint32_t));
+    p.total = L.off;
+    return;
   } else {
     int s = (int)((2 * (int64_t)di.sms * 2 + total_q - 1) / total_q);
     if (s < 1) s = 1;
@@ -585,14 +592,16 @@ void plan_decode(const DeviceInfo& di, int B, int total_q, int64_t total_keys, i
 }
 
 // Tensor-core decode scan of `rows` query rows (q_offsets == nullptr: one row
-// per sequence) followed by the merge of the splits' partial lists into
-// idx / val [rows, k].  K is bf16 (fp8 keys already widened).
+// per sequence), whose slices leave their whole candidate lists, followed by
+// the merge that selects each row's top k from them into idx / val [rows, k].
+// K is bf16 (fp8 keys already widened).
 int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void* K, const float* K_scale,
                   const int64_t* k_offsets, const int32_t* q_offsets, int B, int rows, int64_t total_keys, int H,
                   int d, int k, int32_t* idx, float* val, uint8_t* ws, cudaStream_t st, const int* ok = nullptr) {
   int r;
-  uint2* ppair = reinterpret_cast<uint2*>(ws + p.ppair_off);
-  int* pcnt = reinterpret_cast<int*>(ws + p.pcnt_off);
+  uint2* cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+  int* hdr = reinterpret_cast<int*>(ws + p.hdr_off);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + p.hist_off);
   int* status = reinterpret_cast<int*>(ws);
   CUtensorMap tmQ, tmK;
   if ((r = make_map_bf16(&tmQ, Q, (uint64_t)rows * H, (uint64_t)d, 64)) != DSA_OK) return r;
@@ -607,10 +616,10 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
   a.n_units = B * p.splits;
   a.k = k;
   a.w = w;
-  a.out_pair = ppair;
   a.out_ld = k;
-  a.out_cnt = pcnt;
-  a.cand = reinterpret_cast<uint2*>(ws + p.cand_off);
+  a.out_cnt = hdr;
+  a.out_hist = hist;
+  a.cand = cand;
   a.cand_cap = p.cand_cap;
   a.status = status;
   a.k_off = k_offsets;
@@ -620,7 +629,7 @@ int run_decode_tc(const DecodePlan& p, const void* Q, const float* w, const void
   a.total_keys = total_keys;
   a.offsets_ok = ok;
   if ((r = launch_tc_index(tmQ, tmK, a, p.grid, st)) != DSA_OK) return r;
-  return launch_decode_merge(ppair, pcnt, rows, p.splits, k, idx, val, status, st, ok);
+  return launch_decode_merge_lists(cand, p.cand_cap, hdr, hist, rows, p.splits, k, idx, val, status, st, ok);
 }
 
 }  // namespace

@@ -8,6 +8,8 @@
 //   * decode_merge: combines the per-split top-k lists of a decode query;
 //   * local_extend: bank + a group's own stretch (Refine with local additions);
 //   * block_mean: block representatives for block routing.
+#include <atomic>
+
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
 #include "dsa_internal.h"
@@ -453,6 +455,103 @@ int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, in
   if (splits > 256) return DSA_ERR_UNSUPPORTED;
   decode_merge_kernel<<<total_q, kMergeThreads, 0, stream>>>(parts, part_cnt, splits, k, out_idx, out_val, status,
                                                              ok);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// decode merge of the tensor-core scan's raw slice lists: a decode row's
+// slices left their whole candidate lists (no per-slice selection) with a bin
+// histogram each.  The histograms add up to the row's, whose exact threshold
+// bin is read off it; one classify pass over every slice's segments (dealt
+// out to the warps) emits the entries above it and stages the bin, which the
+// same exact resolve as the scan kernel's select finishes.
+// ---------------------------------------------------------------------------
+constexpr int kMergeListThreads = 1024;
+
+__global__ void __launch_bounds__(kMergeListThreads) decode_merge_lists_kernel(
+    const uint2* __restrict__ cand, int64_t cand_cap, const int* __restrict__ hdr, const uint32_t* __restrict__ hist,
+    int splits, int k, int32_t* __restrict__ out_idx, float* __restrict__ out_val, int* status, const int* ok) {
+  __shared__ MergeSmem M;
+  extern __shared__ uint8_t dyn[];  // [splits * 16] segment starts, then [splits * 16] counts
+  if (offsets_bad(ok)) return;
+  const uint2** segp = reinterpret_cast<const uint2**>(dyn);
+  int* segn = reinterpret_cast<int*>(dyn + sizeof(const uint2*) * splits * 16);
+  __shared__ int row_nseg;
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  RowState& st = M.st;
+  if (tid == 0) {
+    st.outpos = 0;
+    st.stage_cnt = 0;
+    // a row's slices come from one sequence and share its segment count
+    const int ns = __ldcg(hdr + (int64_t)row * splits * kSegHdr);
+    row_nseg = (ns == 4 || ns == 8 || ns == 16) ? ns : 0;
+  }
+  // the row's histogram: the sum of its slices' (loads in flight together)
+  for (int b = tid; b < kBins; b += kMergeListThreads) {
+    const uint32_t* hb = hist + (int64_t)row * splits * kBins + b;
+    uint32_t h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+    int sp = 0;
+    for (; sp + 4 <= splits; sp += 4) {
+      h0 += __ldcg(hb + (int64_t)(sp + 0) * kBins);
+      h1 += __ldcg(hb + (int64_t)(sp + 1) * kBins);
+      h2 += __ldcg(hb + (int64_t)(sp + 2) * kBins);
+      h3 += __ldcg(hb + (int64_t)(sp + 3) * kBins);
+    }
+    for (; sp < splits; ++sp) h0 += __ldcg(hb + (int64_t)sp * kBins);
+    st.hist[b] = (h0 + h1) + (h2 + h3);
+  }
+  __syncthreads();
+  // the segment table, segment j of slice sp at s = j * splits + sp; a slice
+  // whose header disagrees (skipped on invalid offsets) reads as empty
+  const int ns = row_nseg;
+  const int nseg_total = ns * splits;
+  const int64_t stride = ns ? cand_cap / ns : 0;
+  for (int s = tid; s < nseg_total; s += kMergeListThreads) {
+    const int j = s / splits, sp = s - j * splits;
+    const int64_t o = (int64_t)row * splits + sp;
+    const int c = __ldcg(hdr + o * kSegHdr + 1 + j);
+    const bool same = __ldcg(hdr + o * kSegHdr) == ns;
+    segp[s] = cand + o * cand_cap + j * stride;
+    segn[s] = (same && c >= 0 && c <= stride) ? c : 0;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int2 r = hist_scan(st, 0, kBins - 1, k, lane);
+    if (lane == 0) {
+      st.bstar = r.x >= 0 ? r.x : 0;
+      st.cge = r.y;
+    }
+  }
+  __syncthreads();
+  CandList cl;
+  cl.base = cand;
+  cl.stride = 0;
+  cl.nseg = nseg_total;
+  cl.cnt = segn;
+  cl.l2 = true;  // written by the scan kernel's CTAs
+  cl.segp = segp;
+  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k), M.stage, kMergeStage, tid,
+             kMergeListThreads, 1, status);
+}
+
+int launch_decode_merge_lists(const uint2* cand, int64_t cand_cap, const int* hdr, const uint32_t* hist, int total_q,
+                              int splits, int k, int32_t* out_idx, float* out_val, int* status, cudaStream_t stream,
+                              const int* ok) {
+  const NvtxRange nvtx("dsa.decode_merge");
+  if (splits < 1 || splits > 256) return DSA_ERR_UNSUPPORTED;
+  const size_t dyn = (size_t)splits * 16 * (sizeof(const uint2*) + sizeof(int));
+  const size_t total = dyn + sizeof(MergeSmem) + 64;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+  if (total > 48 * 1024 && !(configured.load() & (uint64_t(1) << dev))) {
+    if (cudaFuncSetAttribute(decode_merge_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(64 * 1024 + 1024)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    configured.fetch_or(uint64_t(1) << dev);
+  }
+  decode_merge_lists_kernel<<<total_q, kMergeListThreads, dyn, stream>>>(cand, cand_cap, hdr, hist, splits, k,
+                                                                         out_idx, out_val, status, ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

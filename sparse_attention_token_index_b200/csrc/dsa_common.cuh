@@ -59,6 +59,21 @@ __device__ __forceinline__ int score_bin(float f) {
   return key < 0 ? 0 : (key > kBins - 1 ? kBins - 1 : key);
 }
 
+// The smallest score whose bin is b: for every finite score f,
+// score_bin(f) >= b  <=>  f >= bin_floor(b).  (Bin 0 holds every score up to
+// 2^-40, negatives included, so its floor is -inf; inside bins 1..1023 the
+// bin is the score's top 13 bits offset by the exponent floor, and positive
+// floats order like their bits.)
+__device__ __forceinline__ float bin_floor(int b) {
+  return b <= 0 ? __int_as_float(0xff800000) : __uint_as_float((uint32_t)(b + kBinExpLo * 16) << 19);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
 // 64-bit selection key: larger = better (higher score, then lower index).
 __device__ __forceinline__ uint64_t sel_key(uint2 e) {
   return ((uint64_t)f2o(__uint_as_float(e.x)) << 32) | (uint64_t)(~e.y);

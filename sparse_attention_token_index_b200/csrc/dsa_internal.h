@@ -23,13 +23,18 @@ struct NvtxRange {
 // bank in shared memory (8 bytes per key, 128 KB at this size).
 constexpr int kMaxBank = 16384;
 
+// Decode slices hand their raw candidate lists to the merge: per (row, slice)
+// a header {nseg, count of segment 0 .. 15} and a kBins histogram; segment j
+// of (row, slice) o starts at cand + o * cand_cap + j * (cand_cap / nseg).
+constexpr int kSegHdr = 17;
+
 // Arguments of the tensor-core kernel (see dsa_tc.cu).
 //   kind 0: prefill rows.  Row r of Q sits at position
 //           pos_base + min(r * pos_mul + pos_add, pos_clamp) and sees keys
 //           0..pos (dense: pos_mul 1, pos_add 0; group proxies: pos_mul G,
 //           pos_add G-1 so the proxy scans its group's last member's prefix).
 //   kind 1: decode segments; unit v = (sequence v / splits, split v % splits);
-//           each leaves a partial top-k list that decode_merge combines.
+//           each leaves its candidate list (no selection) for decode_merge.
 //   kind 3: routed refine; unit v = query row v over its routed key blocks.
 //   kind 2: group refine; unit v = (group v / mblocks, member block v % mblocks);
 //           keys are the group's gathered bank rows, key_map gives their
@@ -47,9 +52,10 @@ struct TcArgs {
   const float* w;
   int32_t* out_idx;
   float* out_val;
-  uint2* out_pair;   // decode: partial lists as {score bits, index} pairs
+  uint2* out_pair;   // decode (fp32 kernel): partial lists as {score bits, index} pairs
   int64_t out_ld;
-  int* out_cnt;
+  int* out_cnt;      // decode (tensor-core kernel): per (row, slice) segment header, kSegHdr ints
+  uint32_t* out_hist;  // decode (tensor-core kernel): per (row, slice) bin histogram of its candidates
   uint2* cand;
   int64_t cand_cap;
   int* status;
@@ -170,6 +176,11 @@ int launch_bank_rank_reuse(int32_t* bank_idx, float* bank_val, int ng, int bank_
 // parts [total_q, splits, k] {score bits, index} pairs, part_cnt [total_q, splits]
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
                         float* out_val, int* status, cudaStream_t stream, const int* ok = nullptr);
+// The tensor-core decode scan's raw slice lists: cand [total_q, splits, cand_cap],
+// hdr [total_q, splits, kSegHdr], hist [total_q, splits, kBins].
+int launch_decode_merge_lists(const uint2* cand, int64_t cand_cap, const int* hdr, const uint32_t* hist, int total_q,
+                              int splits, int k, int32_t* out_idx, float* out_val, int* status, cudaStream_t stream,
+                              const int* ok = nullptr);
 // Device check of decode offsets into the workspace header (offsets_ok + status word).
 int launch_decode_offsets_check(const int64_t* k_off, const int32_t* q_off, int B, int64_t total_keys, int total_q,
                                 int max_keys, void* workspace, cudaStream_t stream);

@@ -473,11 +473,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       RowState& st = S.rows[q];
       const int nseg = 4 * team;
       const int64_t seg_stride = a.cand_cap / nseg;
-      uint2* const cand0 = a.cand + ((int64_t)blockIdx.x * kQB + q) * a.cand_cap;
+      const int64_t row = (int64_t)u.row0 + q;
+      // decode: a list per (row, slice), read later by the merge; else a
+      // list per (CTA, query slot), reused by the CTA's next unit
+      uint2* const cand0 = a.cand + (kKind == 1 ? (active ? row * a.splits + u.seq_split : 0)
+                                                : (int64_t)blockIdx.x * kQB + q) * a.cand_cap;
       uint2* const my_seg = cand0 + (member * 4 + lq) * seg_stride;
       const ulonglong2* w2 = reinterpret_cast<const ulonglong2*>(S.w[q]);
       // per-unit scalars (kept in registers through the tile loop)
-      const int64_t row = (int64_t)u.row0 + q;
       // keys 0 .. pos are visible (pos = -1: none); positions fit in int (N <= INT_MAX)
       const int pos = active ? (int)slot_pos<kKind>(a, u, q) : -1;
       const unsigned n_vis = (unsigned)(pos + 1);
@@ -507,6 +510,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const bool mine = active && (jt & (team - 1)) == member;
+        const float thr = row_threshold(st);  // read early: its latency hides behind the tile's loads
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
         if (mine) {
@@ -545,7 +549,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && (unsigned)kpos < n_vis;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
-          row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, lane);
+          row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, thr, lane);
         }
         if constexpr (kKind == 4) walk.next(a);
       }
@@ -556,6 +560,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // the whole team agrees on success before any further barrier
       ok = group_and(tbar, tthr, ok);
       if (!ok) break;
+      if constexpr (kKind == 1) {
+        // decode: no selection here.  The slice's raw candidate list goes to
+        // the merge with its segment counts and its bin histogram, so the
+        // key stream never pauses for a select.
+        const int64_t o = row * a.splits + u.seq_split;
+        if (lane == 0) a.out_cnt[o * kSegHdr + 1 + member * 4 + lq] = count;
+        if (ttid == 0) {
+          a.out_cnt[o * kSegHdr] = nseg;
+          tb_close(st);
+        }
+        named_bar(tbar, tthr);  // every append of the team has landed in the histogram
+        for (int b = ttid; b < kBins; b += tthr) a.out_hist[o * kBins + b] = st.hist[b];
+        named_bar(tbar, tthr);  // the histogram is read out before any member resets it
+        continue;
+      }
       if (lane == 0) st.seg_cnt[member * 4 + lq] = count;
       if (ttid == 0) tb_close(st);
       named_bar(tbar, tthr);
@@ -567,16 +586,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cl.nseg = nseg;
       cl.cnt = st.seg_cnt;
       cl.l2 = false;
-      if constexpr (kKind == 1) {
-        // decode: this split's local top-k, combined later by decode_merge
-        const int64_t o = row * a.splits + u.seq_split;
-        const int cnt = row_select(st, cl, a.k, RowOut{nullptr, nullptr, a.out_pair + o * a.out_ld},
-                                   S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
-        if (ttid == 0) a.out_cnt[o] = cnt;
-      } else {
-        row_select(st, cl, a.k, row_out(a.out_idx + row * a.out_ld, a.out_val + row * a.out_ld), S.stage[q],
-                   kStageCap, ttid, tthr, tbar, a.status);
-      }
+      row_select(st, cl, a.k, row_out(a.out_idx + row * a.out_ld, a.out_val + row * a.out_ld), S.stage[q],
+                 kStageCap, ttid, tthr, tbar, a.status);
     }
     if (tid == 0) atomicAdd(&S.epi_done, 1);
   }

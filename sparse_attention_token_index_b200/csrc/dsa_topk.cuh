@@ -37,17 +37,20 @@ struct RowState {
 
 constexpr uint32_t kTbActive = 1u << 16;
 
-// Candidate list: nseg segments of `stride` entries each; cnt[s] (shared
-// memory) entries used in segment s.
+// Candidate list: nseg segments; segment s starts at segp[s] (a table in
+// shared memory) or, without a table, at base + s * stride; cnt[s] entries
+// are used in segment s.
 struct CandList {
   const uint2* __restrict__ base;
   int64_t stride;
   int nseg;
   const int* cnt;
   bool l2;  // entries written by other CTAs: read them through L2
+  const uint2* const* segp = nullptr;
   // counts may live in shared or global memory (written by other CTAs):
   // read them with volatile loads
   __device__ __forceinline__ int count(int s) const { return *(volatile const int*)(cnt + s); }
+  __device__ __forceinline__ const uint2* seg(int s) const { return segp ? segp[s] : base + s * stride; }
   __device__ __forceinline__ int total() const {
     int n = 0;
     for (int s = 0; s < nseg; ++s) n += count(s);
@@ -59,7 +62,7 @@ struct CandList {
       i -= count(s);
       ++s;
     }
-    return l2 ? __ldcg(base + s * stride + i) : base[s * stride + i];
+    return l2 ? __ldcg(seg(s) + i) : seg(s)[i];
   }
 };
 
@@ -93,21 +96,31 @@ __device__ __forceinline__ void row_append(RowState& st, uint2* __restrict__ can
   }
 }
 
+// The row's current threshold as a score bound (see bin_floor): read once
+// per tile by each appending warp.  A stale read is a lower bound, which only
+// lets more candidates through.
+__device__ __forceinline__ float row_threshold(const RowState& st) {
+  return bin_floor((int)(*(volatile const uint32_t*)&st.tb & 0xFFFFu));
+}
+
 // Appends to a warp-private segment: `count` (a register, warp-uniform) is
-// the segment's fill; only the histogram and the top bin are shared.  All 32
-// lanes call it.
+// the segment's fill; only the histogram and the top bin are shared.  `thr`
+// is row_threshold(st): a score passes if it is at least the floor of the
+// threshold bin, exactly as if its bin were compared; the bin itself is
+// computed for passing scores only.  All 32 lanes call it.
 __device__ __forceinline__ void row_append_seg(RowState& st, uint2* __restrict__ seg, int& count, float score,
-                                               uint32_t key_out, bool valid, int lane) {
-  const int bin = score_bin(score);
-  const bool pass = valid && (bin >= (int)(*(volatile uint32_t*)&st.tb & 0xFFFFu));
+                                               uint32_t key_out, bool valid, float thr, int lane) {
+  const bool pass = valid && score >= thr;
   const unsigned m = __ballot_sync(0xffffffffu, pass);
   if (m == 0u) return;
   if (pass) {
-    seg[count + __popc(m & ((1u << lane) - 1u))] = make_uint2(__float_as_uint(score), key_out);
+    const int bin = score_bin(score);
+    seg[count + __popc(m & lanemask_lt())] = make_uint2(__float_as_uint(score), key_out);
     atomicAdd(&st.hist[bin], 1u);
     // the top bin rises after the histogram: a raise reading an older top
     // only skips bins, which undercounts and stays safe
-    if (bin > *(volatile int*)&st.top) atomicMax(&st.top, bin);
+    const int wmax = __reduce_max_sync(m, bin);
+    if (lane == __ffs(m) - 1 && wmax > *(volatile int*)&st.top) atomicMax(&st.top, wmax);
   }
   count += __popc(m);
 }
@@ -395,22 +408,24 @@ __device__ __forceinline__ int warp_excl_scan(int x, int lane, int& total) {
 constexpr int kBatch = 8;
 
 // Calls f(e, valid) for every entry of the list, kBatch independent loads in
-// flight per thread; every thread of the group runs the same number of calls
-// (valid = false past the end) so that f may use warp collectives.
+// flight per thread.  The segments are dealt out to the group's warps (a warp
+// streams whole segments), and every lane of a warp runs the same number of
+// calls (valid = false past a segment's end), so f may use warp collectives.
 template <class F>
 __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nthr, F&& f) {
-  for (int s = 0; s < c.nseg; ++s) {
-    const uint2* seg = c.base + s * c.stride;
+  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  for (int s = warp; s < c.nseg; s += nw) {
+    const uint2* seg = c.seg(s);
     const int n = c.count(s);
-    for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
+    for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
       uint2 e[kBatch];
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        const int i = i0 + j * nthr + tid;
+        const int i = i0 + j * 32 + lane;
         e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) f(e[j], i0 + j * nthr + tid < n);
+      for (int j = 0; j < kBatch; ++j) f(e[j], i0 + j * 32 + lane < n);
     }
   }
 }
@@ -418,27 +433,28 @@ __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nt
 // Streams the candidate list in batches of kBatch entries per thread and
 // classifies each entry with cls(e) -> 0 drop, 1 emit to the output, 2 stage
 // into shared memory (entries beyond stage_cap are counted, not stored).
-// Output and stage slots are taken with one warp scan and one atomic per
-// warp and batch.  All nthr threads call it (nthr a multiple of 32).
+// Segments are dealt out to the group's warps; output and stage slots are
+// taken with one warp scan and one atomic per warp and batch.  All nthr
+// threads call it (nthr a multiple of 32).
 template <class Cls>
 __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nthr, RowState& st, const RowOut& out,
                                               uint2* stage, int stage_cap, Cls&& cls) {
-  const int lane = tid & 31;
-  for (int s = 0; s < c.nseg; ++s) {
-    const uint2* seg = c.base + s * c.stride;
+  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  for (int s = warp; s < c.nseg; s += nw) {
+    const uint2* seg = c.seg(s);
     const int n = c.count(s);
-    for (int i0 = 0; i0 < n; i0 += nthr * kBatch) {
+    for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
       uint2 e[kBatch];
       int cat[kBatch];
       int ne = 0, ns = 0;
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        const int i = i0 + j * nthr + tid;
+        const int i = i0 + j * 32 + lane;
         e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        const int i = i0 + j * nthr + tid;
+        const int i = i0 + j * 32 + lane;
         cat[j] = (i < n) ? cls(e[j]) : 0;
         ne += cat[j] == 1;
         ns += cat[j] == 2;
