@@ -84,6 +84,7 @@ def _f64(t):
 GROUP_OVERRIDE = None   # --group: group size of the group workloads
 SHARD = 0               # this rank's batch of the workload: seed = the workload's seed + SHARD
 BANK_OVERRIDE = None    # --bank: candidate bank of the group workloads
+M_OVERRIDE = None       # --m: new queries per sequence of the decode workloads
 
 
 def _row_recall(got_idx, ref_idx):
@@ -499,6 +500,8 @@ class Decode(Workload):
         self.cfg = dict(CONFIGS[self.name])
         if size:
             self.cfg["Nb"] = int(size)
+        if M_OVERRIDE:
+            self.cfg["m"] = int(M_OVERRIDE)
         c = self.cfg
         self.inp = make_decode_inputs(self.name, device=device, lengths=[c["Nb"]] * c["B"], m=c["m"],
                                       seed=c["seed"] + SHARD)
@@ -880,12 +883,13 @@ def main():
                     help="other T = N (prefill) or cache length (decode), e.g. for profiling captures")
     ap.add_argument("--group", type=int, default=None, help="group size G of the group workloads")
     ap.add_argument("--bank", type=int, default=None, help="candidate bank B of the group workloads")
+    ap.add_argument("--m", type=int, default=None, help="new queries per sequence (1..4) of the decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    global GROUP_OVERRIDE, BANK_OVERRIDE
-    GROUP_OVERRIDE, BANK_OVERRIDE = args.group, args.bank
+    global GROUP_OVERRIDE, BANK_OVERRIDE, M_OVERRIDE
+    GROUP_OVERRIDE, BANK_OVERRIDE, M_OVERRIDE = args.group, args.bank, args.m
     if args.bank:
         DecodeGroup.bank = args.bank
     if args.impl == "reference":

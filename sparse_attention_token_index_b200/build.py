@@ -1,10 +1,15 @@
 """Builds the in-tree C-ABI library ``libdsa_index.so`` for sm_100a.
 
-Usage: ``python -m sparse_attention_token_index_b200.build [--verbose]``.
+Usage: ``python -m sparse_attention_token_index_b200.build [--verbose] [--debug-bounds]``.
 Each ``csrc/*.cu`` is compiled with nvcc (``-gencode
 arch=compute_100a,code=sm_100a``) in parallel and linked into one shared
 library next to this file; the CUDA runtime is linked statically, so the
 library loads without a GPU (only calls into it need one).
+
+``--debug-bounds`` builds ``libdsa_index_debug.so`` instead: the same
+library compiled with ``-DDSA_DEBUG_BOUNDS=1``, whose kernels check every
+index they are about to use against its buffer and record a failing check in
+the status word (``DSA_LIB`` selects it at load time).
 """
 from __future__ import annotations
 
@@ -20,6 +25,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdsa_index.so")
+DEBUG_LIB = os.path.join(PKG, "libdsa_index_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -46,22 +52,24 @@ def _deps():
         os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, force: bool = False, extra_flags=None, debug_bounds: bool = False) -> str:
+    lib = DEBUG_LIB if debug_bounds else LIB
+    if not force and up_to_date(lib):
+        return lib
+    build_dir = BUILD + ("_debug" if debug_bounds else "")
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
-    flags = NVCC_FLAGS + list(extra_flags or [])
+    flags = NVCC_FLAGS + (["-DDSA_DEBUG_BOUNDS=1"] if debug_bounds else []) + list(extra_flags or [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         cmd = [nvcc, *flags, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
@@ -76,15 +84,16 @@ def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
         for _, log in results:
             if log.strip():
                 print(log)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
            "-o", tmp, *[o for o, _ in results]]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv,
+                debug_bounds="--debug-bounds" in sys.argv))

@@ -445,8 +445,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const uint2
     }
   }
   __syncthreads();
-  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k), M.stage, kMergeStage, tid,
-             kMergeThreads, 1, status);
+  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k, k, status), M.stage,
+             kMergeStage, tid, kMergeThreads, 1, status);
 }
 
 int launch_decode_merge(const uint2* parts, const int* part_cnt, int total_q, int splits, int k, int32_t* out_idx,
@@ -530,8 +530,8 @@ __global__ void __launch_bounds__(kMergeListThreads) decode_merge_lists_kernel(
   cl.cnt = segn;
   cl.l2 = true;  // written by the scan kernel's CTAs
   cl.segp = segp;
-  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k), M.stage, kMergeStage, tid,
-             kMergeListThreads, 1, status);
+  row_select(st, cl, k, row_out(out_idx + (int64_t)row * k, out_val + (int64_t)row * k, k, status), M.stage,
+             kMergeStage, tid, kMergeListThreads, 1, status);
 }
 
 int launch_decode_merge_lists(const uint2* cand, int64_t cand_cap, const int* hdr, const uint32_t* hist, int total_q,

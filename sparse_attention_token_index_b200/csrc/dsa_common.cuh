@@ -33,6 +33,25 @@ __device__ __forceinline__ void report_error(int* status, int code, int info) {
   if (atomicCAS(status, 0, code) == 0) status[1] = info;
 }
 
+// Debug bounds checks, compiled in by -DDSA_DEBUG_BOUNDS=1 (the library's
+// debug build, libdsa_index_debug.so): an index a kernel is about to use is
+// checked against the extent of its buffer; a failing check records
+// DSA_ERR_INTERNAL with info 100 + site in the status word and the access is
+// skipped.  In the normal build in_bounds is constant true and costs nothing.
+#ifndef DSA_DEBUG_BOUNDS
+#define DSA_DEBUG_BOUNDS 0
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, int* status, int site) {
+  if constexpr (DSA_DEBUG_BOUNDS != 0) {
+    if (!ok) report_error(status, DSA_ERR_INTERNAL, 100 + site);
+    return ok;
+  } else {
+    (void)status;
+    (void)site;
+    return true;
+  }
+}
+
 // A call whose device offsets failed their check (offsets_ok == 0) runs none
 // of its later kernels' work; null means the kernel checks its own.
 __device__ __forceinline__ bool offsets_bad(const int* ok) {
@@ -193,6 +212,49 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "[%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// L2 eviction policies (cache hints for loads and stores): data read once
+// (queries, outputs, streamed decode keys) goes first, data read again (the
+// prefill keys, the candidate lists until the final select) stays.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// A 2-D TMA tile load with an L2 eviction policy.
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                 uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_global_hint(uint2* p, uint2 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x), "r"(v.y), "l"(pol)
+               : "memory");
+}
+
+__device__ __forceinline__ uint2 ld_global_hint(const uint2* p, uint64_t pol) {
+  uint2 v;
+  asm volatile("ld.global.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;" : "=r"(v.x), "=r"(v.y) : "l"(p), "l"(pol));
+  return v;
+}
+
+// Brings a tile into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

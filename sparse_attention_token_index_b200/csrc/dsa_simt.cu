@@ -107,13 +107,14 @@ __global__ void __launch_bounds__(kSimtThreads) simt_index_kernel(const SimtArgs
         score = score + 0.0f;
         if (a.dbg_scores != nullptr) a.dbg_scores[row * a.dbg_ld + key] = score;
       }
-      row_append(G.st, cand, score, (uint32_t)key, valid, lane);
+      row_append(G.st, cand, score, (uint32_t)key, valid, lane, a.cand_cap, a.status);
       named_bar(bar, 128);
       if (lw == 0) row_update(G.st, a.k, lane);
       named_bar(bar, 128);
     }
-    const RowOut out = a.kind == 1 ? RowOut{nullptr, nullptr, a.out_pair + out_row * a.out_ld}
-                                   : row_out(a.out_idx + out_row * a.out_ld, a.out_val + out_row * a.out_ld);
+    const RowOut out = a.kind == 1 ? pair_out(a.out_pair + out_row * a.out_ld, a.k, a.status)
+                                   : row_out(a.out_idx + out_row * a.out_ld, a.out_val + out_row * a.out_ld, a.k,
+                                             a.status);
     const int cnt =
         row_select(G.st, single_list(cand, &G.st.cnt), a.k, out, G.stage, kSimtStageCap, tid, 128, bar, a.status);
     if (a.kind == 1 && tid == 0) a.out_cnt[out_row] = cnt;

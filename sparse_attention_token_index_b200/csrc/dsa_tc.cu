@@ -340,6 +340,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      const uint64_t pol_first = l2_evict_first(), pol_last = l2_evict_last();
       int s = 0;
       uint32_t ph = 0;
       int qi = 0;
@@ -351,9 +352,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_arrive_expect_tx(&S.q_full, (uint32_t)(u.nq * 2 * kQHeadBlockBytes));
         for (int q = 0; q < u.nq; ++q)
           for (int c = 0; c < 2; ++c)
-            tma_load_2d(S.q + c * kQChunkBytes + q * kQHeadBlockBytes, &tmQ, &S.q_full, c * 64,
-                        (u.row0 + q) * kHeads);
+            tma_load_2d_hint(S.q + c * kQChunkBytes + q * kQHeadBlockBytes, &tmQ, &S.q_full, c * 64,
+                             (u.row0 + q) * kHeads, pol_first);
         ++qi;
+        {
+          // the next unit's queries into L2 now, so that its load (issued
+          // only once this unit's last MMA is done) does not wait on HBM
+          UnitInfo un;
+          if (unit_at<kKind>(a, round + 1, un))
+            for (int q = 0; q < un.nq; ++q)
+              for (int c = 0; c < 2; ++c) tma_prefetch_l2_2d(&tmQ, c * 64, (un.row0 + q) * kHeads);
+        }
         ClusterWalk walk;
         if constexpr (kKind == 4) walk.start(a, u.row0);
         for (int j = 0; j < u.ntiles; ++j) {
@@ -375,8 +384,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else {
             row = (kKind == 3) ? routed_block(a, u, j) * kTileKeys : u.key_row0 + (u.tile0 + j) * kTileKeys;
           }
-          for (int c = 0; c < 2; ++c)
-            tma_load_2d(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row);
+          for (int c = 0; c < 2; ++c) {
+            // prefill keys are read by every unit: they stay in L2; a decode
+            // cache streams by once; a gathered bank is left to the default
+            if (kKind == 1)
+              tma_load_2d_hint(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row, pol_first);
+            else if (kKind == 2)
+              tma_load_2d(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row);
+            else
+              tma_load_2d_hint(S.k[s] + c * kKChunkBytes, &tmK, &S.k_full[s], c * 64, row, pol_last);
+          }
           armed |= 1u << s;
           armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
           if (++s == kStages) {
@@ -457,6 +474,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // barrier inside the tile loop: the threshold warp raises the thresholds.
     const int slot = warp >> 2, lq = warp & 3, tid = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)(lq * 32) << 16;
+    const uint64_t pol_keep = l2_evict_last();  // candidate lists: kept in L2 until the row's select reads them
     uint32_t eph = 0u;  // bit b: phase of accumulator buffer b
     int buf = 0;
     UnitInfo u;
@@ -501,6 +519,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (ttid == 0) tb_open(st);
       }
       int count = 0;  // my segment's fill
+      // group refine: the bank slot -> key position of this warp's next tile,
+      // loaded a whole tile ahead so its latency never sits on the tile's path
+      int kp_next = -1;
+      if (kKind == 2 && active && member < ntiles && key0 + member * kTileKeys < nkeys)
+        kp_next = kmap[key0 + member * kTileKeys];
       ClusterWalk walk;
       if constexpr (kKind == 4) walk.start(a, u.row0);
       for (int jt = 0; jt < ntiles; ++jt) {
@@ -542,14 +565,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             in_range = key < nkeys;
           }
           int kpos = key;
-          if (kmap != nullptr) kpos = in_range ? kmap[key] : -1;
+          if constexpr (kKind == 2) {
+            kpos = in_range ? kp_next : -1;
+            const int nkey = key + team * kTileKeys;  // this warp's next tile
+            kp_next = (nkey < nkeys && in_bounds(nkey < a.bank, a.status, 6)) ? kmap[nkey] : -1;
+          } else if (kmap != nullptr) {
+            kpos = in_range ? kmap[key] : -1;
+          }
           const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
           float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
           if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && (unsigned)kpos < n_vis;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
-          row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, thr, lane);
+          row_append_seg(st, my_seg, count, score, (uint32_t)kpos, valid, thr, pol_keep, lane, seg_stride, a.status);
         }
         if constexpr (kKind == 4) walk.next(a);
       }
@@ -561,16 +590,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = group_and(tbar, tthr, ok);
       if (!ok) break;
       if constexpr (kKind == 1) {
-        // decode: no selection here.  The slice's raw candidate list goes to
-        // the merge with its segment counts and its bin histogram, so the
-        // key stream never pauses for a select.
+        // decode: no selection here.  The slice's candidate list goes to the
+        // merge with its segment counts and its bin histogram, so the key
+        // stream pauses only for one short pass: an entry below the slice's
+        // own exact threshold bin has k entries of the slice above it, so
+        // it cannot be in the row's top k, and each warp drops those from
+        // its segment (compacting in place) before the merge reads it.
         const int64_t o = row * a.splits + u.seq_split;
-        if (lane == 0) a.out_cnt[o * kSegHdr + 1 + member * 4 + lq] = count;
-        if (ttid == 0) {
-          a.out_cnt[o * kSegHdr] = nseg;
-          tb_close(st);
-        }
+        if (ttid == 0) tb_close(st);
         named_bar(tbar, tthr);  // every append of the team has landed in the histogram
+        if (ttid < 32) tb_finish(st, a.k, lane);
+        named_bar(tbar, tthr);
+        if (st.cge >= a.k) {
+          const float keep_at = bin_floor(st.bstar);
+          int kept = 0;
+          for (int i0 = 0; i0 < count; i0 += 32 * 8) {
+            uint2 e[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int i = i0 + j * 32 + lane;
+              e[j] = i < count ? my_seg[i] : make_uint2(0u, 0u);
+            }
+            // every entry of this batch is in registers before any write,
+            // and writes land below i0 + 256: no entry is lost
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const bool keep = (i0 + j * 32 + lane < count) && __uint_as_float(e[j].x) >= keep_at;
+              const unsigned m = __ballot_sync(0xffffffffu, keep);
+              if (keep) st_global_hint(my_seg + kept + __popc(m & lanemask_lt()), e[j], pol_keep);
+              kept += __popc(m);
+            }
+          }
+          count = kept;
+        }
+        if (lane == 0) a.out_cnt[o * kSegHdr + 1 + member * 4 + lq] = count;
+        if (ttid == 0) a.out_cnt[o * kSegHdr] = nseg;
         for (int b = ttid; b < kBins; b += tthr) a.out_hist[o * kBins + b] = st.hist[b];
         named_bar(tbar, tthr);  // the histogram is read out before any member resets it
         continue;
@@ -586,8 +640,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cl.nseg = nseg;
       cl.cnt = st.seg_cnt;
       cl.l2 = false;
-      row_select(st, cl, a.k, row_out(a.out_idx + row * a.out_ld, a.out_val + row * a.out_ld), S.stage[q],
-                 kStageCap, ttid, tthr, tbar, a.status);
+      row_select<8>(st, cl, a.k, row_out(a.out_idx + row * a.out_ld, a.out_val + row * a.out_ld, a.k, a.status),
+                    S.stage[q], kStageCap, ttid, tthr, tbar, a.status);
     }
     if (tid == 0) atomicAdd(&S.epi_done, 1);
   }

@@ -47,10 +47,14 @@ struct CandList {
   const int* cnt;
   bool l2;  // entries written by other CTAs: read them through L2
   const uint2* const* segp = nullptr;
+  uint64_t pol = 0;  // nonzero: the L2 policy of the reads (a final read lets the lines go)
   // counts may live in shared or global memory (written by other CTAs):
   // read them with volatile loads
   __device__ __forceinline__ int count(int s) const { return *(volatile const int*)(cnt + s); }
   __device__ __forceinline__ const uint2* seg(int s) const { return segp ? segp[s] : base + s * stride; }
+  __device__ __forceinline__ uint2 load(const uint2* p) const {
+    return pol ? ld_global_hint(p, pol) : (l2 ? __ldcg(p) : *p);
+  }
   __device__ __forceinline__ int total() const {
     int n = 0;
     for (int s = 0; s < nseg; ++s) n += count(s);
@@ -62,7 +66,7 @@ struct CandList {
       i -= count(s);
       ++s;
     }
-    return l2 ? __ldcg(seg(s) + i) : seg(s)[i];
+    return load(seg(s) + i);
   }
 };
 
@@ -80,7 +84,8 @@ __device__ __forceinline__ void row_reset(RowState& st, int tid, int nthr) {
 
 // Called by all 32 lanes of one warp for one score per lane.
 __device__ __forceinline__ void row_append(RowState& st, uint2* __restrict__ cand, float score,
-                                           uint32_t key_out, bool valid, int lane) {
+                                           uint32_t key_out, bool valid, int lane, int64_t cap = 0,
+                                           int* status = nullptr) {
   const int bin = score_bin(score);
   const bool pass = valid && (bin >= *(volatile int*)&st.bstar);
   const unsigned m = __ballot_sync(0xffffffffu, pass);
@@ -90,7 +95,7 @@ __device__ __forceinline__ void row_append(RowState& st, uint2* __restrict__ can
   base = __shfl_sync(0xffffffffu, base, 0);
   if (pass) {
     const int r = __popc(m & ((1u << lane) - 1u));
-    cand[base + r] = make_uint2(__float_as_uint(score), key_out);
+    if (in_bounds(base + r < cap, status, 1)) cand[base + r] = make_uint2(__float_as_uint(score), key_out);
     const unsigned mm = __match_any_sync(m, bin);
     if ((__ffs(mm) - 1) == lane) atomicAdd(&st.hist[bin], (uint32_t)__popc(mm));
   }
@@ -107,22 +112,27 @@ __device__ __forceinline__ float row_threshold(const RowState& st) {
 // the segment's fill; only the histogram and the top bin are shared.  `thr`
 // is row_threshold(st): a score passes if it is at least the floor of the
 // threshold bin, exactly as if its bin were compared; the bin itself is
-// computed for passing scores only.  All 32 lanes call it.
+// computed for passing scores only.  `pol`: the L2 policy of the stores (the
+// list is read back once, at the row's end).  All 32 lanes call it.
 __device__ __forceinline__ void row_append_seg(RowState& st, uint2* __restrict__ seg, int& count, float score,
-                                               uint32_t key_out, bool valid, float thr, int lane) {
+                                               uint32_t key_out, bool valid, float thr, uint64_t pol, int lane,
+                                               int64_t seg_cap = 0, int* status = nullptr) {
   const bool pass = valid && score >= thr;
   const unsigned m = __ballot_sync(0xffffffffu, pass);
-  if (m == 0u) return;
-  if (pass) {
+  if (m != 0u) {  // warp-uniform: the warp's collectives stay outside any divergent region
     const int bin = score_bin(score);
-    seg[count + __popc(m & lanemask_lt())] = make_uint2(__float_as_uint(score), key_out);
-    atomicAdd(&st.hist[bin], 1u);
+    const int wmax = __reduce_max_sync(0xffffffffu, pass ? bin : -1);
+    const int at = count + __popc(m & lanemask_lt());
+    if (pass) {
+      if (in_bounds(at < seg_cap, status, 2))
+        st_global_hint(seg + at, make_uint2(__float_as_uint(score), key_out), pol);
+      atomicAdd(&st.hist[bin], 1u);
+    }
     // the top bin rises after the histogram: a raise reading an older top
     // only skips bins, which undercounts and stays safe
-    const int wmax = __reduce_max_sync(m, bin);
-    if (lane == __ffs(m) - 1 && wmax > *(volatile int*)&st.top) atomicMax(&st.top, wmax);
+    if (lane == 0 && wmax > *(volatile int*)&st.top) atomicMax(&st.top, wmax);
+    count += __popc(m);
   }
-  count += __popc(m);
 }
 
 // Largest bin b in [b0, top] with sum_{b' >= b} hist[b'] >= k, reading the
@@ -285,25 +295,35 @@ struct RowOut {
   int32_t* __restrict__ idx;
   float* __restrict__ val;
   uint2* __restrict__ pair;
+  int k = 0;             // the row's slots (bounds checks of the debug build)
+  int* status = nullptr;
+  // outputs are written once and not read here again: streaming stores
   __device__ __forceinline__ void put(int p, uint2 e) const {
+    if (!in_bounds((unsigned)p < (unsigned)k, status, 3)) return;
     if (pair != nullptr) {
-      pair[p] = e;
+      __stcs(pair + p, e);
     } else {
-      idx[p] = (int32_t)e.y;
-      val[p] = __uint_as_float(e.x);
+      __stcs(idx + p, (int32_t)e.y);
+      __stcs(val + p, __uint_as_float(e.x));
     }
   }
   __device__ __forceinline__ void pad(int p) const {
+    if (!in_bounds((unsigned)p < (unsigned)k, status, 4)) return;
     if (pair != nullptr) {
-      pair[p] = make_uint2(0xff800000u, 0xffffffffu);
+      __stcs(pair + p, make_uint2(0xff800000u, 0xffffffffu));
     } else {
-      idx[p] = -1;
-      val[p] = __int_as_float(0xff800000);
+      __stcs(idx + p, -1);
+      __stcs(val + p, __int_as_float(0xff800000));
     }
   }
 };
 
-__device__ __forceinline__ RowOut row_out(int32_t* idx, float* val) { return RowOut{idx, val, nullptr}; }
+__device__ __forceinline__ RowOut row_out(int32_t* idx, float* val, int k, int* status) {
+  return RowOut{idx, val, nullptr, k, status};
+}
+__device__ __forceinline__ RowOut pair_out(uint2* pair, int k, int* status) {
+  return RowOut{nullptr, nullptr, pair, k, status};
+}
 
 __device__ __forceinline__ void emit(RowState& st, uint2 e, const RowOut& out) {
   const int p = atomicAdd(&st.outpos, 1);
@@ -422,7 +442,7 @@ __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nt
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * 32 + lane;
-        e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
+        e[j] = (i < n) ? c.load(seg + i) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) f(e[j], i0 + j * 32 + lane < n);
@@ -450,7 +470,7 @@ __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nt
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * 32 + lane;
-        e[j] = (i < n) ? (c.l2 ? __ldcg(seg + i) : seg[i]) : make_uint2(0u, 0u);
+        e[j] = (i < n) ? c.load(seg + i) : make_uint2(0u, 0u);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
@@ -489,14 +509,13 @@ __device__ __forceinline__ uint2 key_entry(uint64_t key) {
   return make_uint2(u, ~(uint32_t)key);
 }
 
-constexpr int kResolvePerThread = 8;  // staged entries per thread: stage_cap <= 8 * nthr
-
-// Emits the `need` best of the ns staged entries (need <= ns <= stage_cap).
-// Entries move into registers; MSD digit steps of 8 bits, starting at bit
-// `shift` of the 64-bit key (bits above it are equal for all entries or
-// already decided), drop or emit whole digit buckets until at most 128
-// entries remain undecided; those are ranked exactly by counting.
-// Group-wide (nthr threads, barrier `bar`).
+// Emits the `need` best of the ns staged entries (need <= ns <= stage_cap,
+// stage_cap <= kPer * nthr).  Entries move into registers (kPer a thread);
+// MSD digit steps of 8 bits, starting at bit `shift` of the 64-bit key (bits
+// above it are equal for all entries or already decided), drop or emit whole
+// digit buckets until at most 128 entries remain undecided; those are ranked
+// exactly by counting.  Group-wide (nthr threads, barrier `bar`).
+template <int kResolvePerThread>
 static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, int ns, int need, int shift,
                                                   const RowOut out, int tid, int nthr, int bar) {
   const int lane = tid & 31;
@@ -545,8 +564,8 @@ static __device__ __noinline__ void stage_resolve(RowState& st, uint2* stage, in
     if (live[j]) kk[base + __popc(m & ((1u << lane) - 1u))] = key[j];
   }
   named_bar(bar, nthr);
-  if (tid < nlive) {
-    const uint64_t mine = kk[tid];
+  for (int i = tid; i < nlive; i += nthr) {
+    const uint64_t mine = kk[i];
     int rank = 0;
     for (int j = 0; j < nlive; ++j) rank += kk[j] > mine;
     if (rank < remaining) {
@@ -565,8 +584,9 @@ __device__ __forceinline__ int digit_shift_below(int bin) { return (bin > 0 && b
 // Final selection of one row: writes min(k, visible) entries to
 // out[0..k) (any order), pads the rest with -1 / -inf, and
 // returns the number of real entries.  Group-wide call (nthr threads, a
-// multiple of 32, stage_cap <= 8 * nthr).  Expects st.bstar / st.cge exact
-// (no appends in flight).
+// multiple of 32, stage_cap <= kPer * nthr).  Expects st.bstar / st.cge
+// exact (no appends in flight).
+template <int kPer = 8>
 static __device__ __noinline__ int row_select(RowState& st, const CandList cand, int k, const RowOut out,
                                               uint2* __restrict__ stage, int stage_cap, int tid, int nthr, int bar,
                                               int* status) {
@@ -597,7 +617,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
   const int ns = st.stage_cnt;
   if (tid == 0 && (ns != hb || st.outpos != cge - hb)) report_error(status, DSA_ERR_INTERNAL, 1);
   if (ns <= stage_cap) {
-    stage_resolve(st, stage, ns, need, digit_shift_below(bstar), out, tid, nthr, bar);
+    stage_resolve<kPer>(st, stage, ns, need, digit_shift_below(bstar), out, tid, nthr, bar);
     return k;
   }
   // The threshold bin holds more entries than the stage.  Inside bins
@@ -627,7 +647,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
       });
       named_bar(bar, nthr);
       if (tid == 0 && (st.stage_cnt != hsel || st.outpos != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
-      stage_resolve(st, stage, hsel, need - above, 35, out, tid, nthr, bar);
+      stage_resolve<kPer>(st, stage, hsel, need - above, 35, out, tid, nthr, bar);
       return k;
     }
     named_bar(bar, nthr);
@@ -659,11 +679,12 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
         if (km > prefix) {
           emit(st, e, out);
         } else if (km == prefix) {
-          stage[atomicAdd(&st.stage_cnt, 1)] = e;
+          const int at = atomicAdd(&st.stage_cnt, 1);
+          if (in_bounds(at < stage_cap, status, 5)) stage[at] = e;
         }
       }
       named_bar(bar, nthr);
-      stage_resolve(st, stage, hsel, remaining, shift - 8, out, tid, nthr, bar);
+      stage_resolve<kPer>(st, stage, hsel, remaining, shift - 8, out, tid, nthr, bar);
       return k;
     }
   }
