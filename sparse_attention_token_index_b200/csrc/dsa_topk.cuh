@@ -450,9 +450,14 @@ __device__ __forceinline__ void for_each_cand(const CandList& c, int tid, int nt
   }
 }
 
+// Classify outcomes as packed counter increments, so that one warp scan
+// counts both: selected entries in the low 16 bits, staged ones in the high.
+constexpr int kCatSel = 1, kCatStage = 1 << 16;
+
 // Streams the candidate list in batches of kBatch entries per thread and
-// classifies each entry with cls(e) -> 0 drop, 1 emit to the output, 2 stage
-// into shared memory (entries beyond stage_cap are counted, not stored).
+// classifies each entry with cls(e) -> 0 drop, kCatSel emit to the output,
+// kCatStage stage into shared memory (entries beyond stage_cap are counted,
+// not stored).
 // Segments are dealt out to the group's warps; output and stage slots are
 // taken with one warp scan and one atomic per warp and batch.  All nthr
 // threads call it (nthr a multiple of 32).
@@ -466,7 +471,7 @@ __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nt
     for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
       uint2 e[kBatch];
       int cat[kBatch];
-      int ne = 0, ns = 0;
+      int acc = 0;  // selected | staged << 16 (at most 8 of each a lane, 256 a warp)
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * 32 + lane;
@@ -476,25 +481,24 @@ __device__ __forceinline__ void classify_pass(const CandList& c, int tid, int nt
       for (int j = 0; j < kBatch; ++j) {
         const int i = i0 + j * 32 + lane;
         cat[j] = (i < n) ? cls(e[j]) : 0;
-        ne += cat[j] == 1;
-        ns += cat[j] == 2;
+        acc += cat[j];
       }
-      int te, ts;
-      int pe = warp_excl_scan(ne, lane, te);
-      int ps = warp_excl_scan(ns, lane, ts);
+      int tot;
+      const int p = warp_excl_scan(acc, lane, tot);
+      const int te = tot & 0xFFFF, ts = tot >> 16;
       int be = 0, bs = 0;
       if (lane == 0) {
         if (te) be = atomicAdd(&st.outpos, te);
         if (ts) bs = atomicAdd(&st.stage_cnt, ts);
       }
-      be = __shfl_sync(0xffffffffu, be, 0) + pe;
-      bs = __shfl_sync(0xffffffffu, bs, 0) + ps;
+      be = __shfl_sync(0xffffffffu, be, 0) + (p & 0xFFFF);
+      bs = __shfl_sync(0xffffffffu, bs, 0) + (p >> 16);
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        if (cat[j] == 1) {
+        if (cat[j] == kCatSel) {
           out.put(be, e[j]);
           ++be;
-        } else if (cat[j] == 2) {
+        } else if (cat[j] == kCatStage) {
           if (bs < stage_cap) stage[bs] = e[j];
           ++bs;
         }
@@ -601,7 +605,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
   named_bar(bar, nthr);
   if (cge < k) {
     // b* never moved: every visible key was appended (n == cge < k)
-    classify_pass(cand, tid, nthr, st, out, stage, 0, [](uint2) { return 1; });
+    classify_pass(cand, tid, nthr, st, out, stage, 0, [](uint2) { return kCatSel; });
     named_bar(bar, nthr);
     for (int i = n + tid; i < k; i += nthr) out.pad(i);
     named_bar(bar, nthr);
@@ -609,9 +613,12 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
   }
   const int need = k - (cge - hb);
   // entries above the threshold bin are selected; the bin itself is staged
-  classify_pass(cand, tid, nthr, st, out, stage, stage_cap, [bstar](uint2 e) {
-    const int b = score_bin(__uint_as_float(e.x));
-    return b > bstar ? 1 : (b == bstar ? 2 : 0);
+  // score_bin(f) > b*  <=>  f >= bin_floor(b* + 1) (none when b* is the top bin);
+  // score_bin(f) == b* <=>  f >= bin_floor(b*) and not above
+  const float f_hi = bstar >= kBins - 1 ? __int_as_float(0x7f800000) : bin_floor(bstar + 1), f_lo = bin_floor(bstar);
+  classify_pass(cand, tid, nthr, st, out, stage, stage_cap, [f_hi, f_lo](uint2 e) {
+    const float f = __uint_as_float(e.x);
+    return f >= f_hi ? kCatSel : (f >= f_lo ? kCatStage : 0);
   });
   named_bar(bar, nthr);
   const int ns = st.stage_cnt;
@@ -643,7 +650,7 @@ static __device__ __noinline__ int row_select(RowState& st, const CandList cand,
       classify_pass(cand, tid, nthr, st, out, stage, stage_cap, [bstar, dsel](uint2 e) {
         if (score_bin(__uint_as_float(e.x)) != bstar) return 0;
         const int dg = (int)((e.x >> 11) & 255u);
-        return dg > dsel ? 1 : (dg == dsel ? 2 : 0);
+        return dg > dsel ? kCatSel : (dg == dsel ? kCatStage : 0);
       });
       named_bar(bar, nthr);
       if (tid == 0 && (st.stage_cnt != hsel || st.outpos != cge - hb + above)) report_error(status, DSA_ERR_INTERNAL, 2);
