@@ -133,14 +133,36 @@ __global__ void bank_gather_kernel(const uint4* __restrict__ K, int row_vecs, co
   }
 }
 
+// The tensor-core path's rows (bf16, d = 128: 16 vectors of 16 bytes): a warp
+// copies two whole rows per step, one bank entry read per row and no
+// division per element, so the copy runs at the write bandwidth.
+__global__ void bank_gather_rows16_kernel(const uint4* __restrict__ K, const int32_t* __restrict__ bank,
+                                          int64_t n_rows, int bank_size, const int64_t* __restrict__ row_off,
+                                          uint4* __restrict__ Kg, const int* ok) {
+  if (offsets_bad(ok)) return;
+  const int lane = threadIdx.x & 31, c = lane & 15;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp0 * 2 + (lane >> 4); r < n_rows; r += nwarps * 2) {
+    const int32_t src = bank[r];
+    const int64_t base = row_off ? row_off[r / bank_size] : 0;
+    Kg[r * 16 + c] = src >= 0 ? K[(base + src) * 16 + c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size, void* Kg,
                        cudaStream_t stream, const int64_t* row_off, const int* ok) {
   const NvtxRange nvtx("dsa.bank_gather");
   const int elt = (k_dtype == DSA_DTYPE_FP32) ? 4 : (k_dtype == DSA_DTYPE_BF16 ? 2 : 1);
   const int row_vecs = d * elt / 16;
-  bank_gather_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), row_vecs, bank,
-                                                   (int64_t)ng * bank_size, bank_size, row_off,
-                                                   static_cast<uint4*>(Kg), ok);
+  if (row_vecs == 16)
+    bank_gather_rows16_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), bank,
+                                                           (int64_t)ng * bank_size, bank_size, row_off,
+                                                           static_cast<uint4*>(Kg), ok);
+  else
+    bank_gather_kernel<<<148 * 8, 256, 0, stream>>>(static_cast<const uint4*>(K), row_vecs, bank,
+                                                     (int64_t)ng * bank_size, bank_size, row_off,
+                                                     static_cast<uint4*>(Kg), ok);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
