@@ -496,7 +496,15 @@ int dsa_index_group(const void* Q, const float* w, const void* K, const float* K
     kmap = map;
   }
   void* Kg = ws + gp.kg_off;
-  if ((r = launch_bank_gather(K, k_dtype, d, kmap, gp.ng, S, Kg, st)) != DSA_OK) return r;
+  if (!local && bank <= 8192) {
+    // the bank in descending order of the proxy's score bin: members meet
+    // their likely top keys first (the set, and so the results, unchanged)
+    int32_t* map = reinterpret_cast<int32_t*>(ws + gp.map_off);
+    if ((r = launch_bank_order_gather(K, bi, bv, gp.ng, bank, map, Kg, st)) != DSA_OK) return r;
+    kmap = map;
+  } else if ((r = launch_bank_gather(K, k_dtype, d, kmap, gp.ng, S, Kg, st)) != DSA_OK) {
+    return r;
+  }
   CUtensorMap tmQ, tmK;
   if ((r = make_map_bf16(&tmQ, Q, (uint64_t)T * H, (uint64_t)d, 64)) != DSA_OK) return r;
   if ((r = make_map_bf16(&tmK, Kg, (uint64_t)gp.ng * S, (uint64_t)d, 128)) != DSA_OK) return r;

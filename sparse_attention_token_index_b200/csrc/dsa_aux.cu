@@ -150,6 +150,76 @@ __global__ void bank_gather_rows16_kernel(const uint4* __restrict__ K, const int
   }
 }
 
+// Refine's bank in descending order of the proxy's score bin, then gathered:
+// map[g, :] = the group's bank indices ordered by score_bin(proxy score),
+// highest bin first (any order inside a bin), and Kg the matching key rows
+// (bf16, d = 128).  Members then meet their likely top keys early, so their
+// streaming threshold rises sooner and fewer candidates reach the select.
+// The bank stays the same set: the order changes nothing in the results.
+// One block of kOrderThreads per group.
+constexpr int kOrderThreads = 512;
+constexpr int kOrderMaxBank = 8192;  // bank entries a block orders in shared memory
+
+__global__ void __launch_bounds__(kOrderThreads) bank_order_gather_kernel(const uint4* __restrict__ K,
+                                                                           const int32_t* __restrict__ bank_idx,
+                                                                           const float* __restrict__ bank_val,
+                                                                           int bank_size, int32_t* __restrict__ map,
+                                                                           uint4* __restrict__ Kg) {
+  __shared__ int hist[kBins];
+  __shared__ int32_t smap[kOrderMaxBank];
+  const int g = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* bi = bank_idx + (int64_t)g * bank_size;
+  const float* bv = bank_val + (int64_t)g * bank_size;
+  for (int b = tid; b < kBins; b += kOrderThreads) hist[b] = 0;
+  __syncthreads();
+  for (int j = tid; j < bank_size; j += kOrderThreads) atomicAdd(&hist[score_bin(bv[j])], 1);
+  __syncthreads();
+  if (warp == 0) {
+    // start of each bin in descending bin order: lane l owns bins 1023 - 32l - 31 .. 1023 - 32l
+    int c[32];
+    int tot = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      c[i] = hist[kBins - 1 - 32 * lane - i];
+      tot += c[i];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - tot;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      hist[kBins - 1 - 32 * lane - i] = run;  // becomes the bin's next free slot
+      run += c[i];
+    }
+  }
+  __syncthreads();
+  for (int j = tid; j < bank_size; j += kOrderThreads) smap[atomicAdd(&hist[score_bin(bv[j])], 1)] = bi[j];
+  __syncthreads();
+  int32_t* mg = map + (int64_t)g * bank_size;
+  for (int j = tid; j < bank_size; j += kOrderThreads) mg[j] = smap[j];
+  // the key rows, two 256-byte rows a warp step
+  const int c16 = lane & 15;
+  uint4* kg = Kg + (int64_t)g * bank_size * 16;
+  for (int r = warp * 2 + (lane >> 4); r < bank_size; r += (kOrderThreads / 32) * 2) {
+    const int32_t src = smap[r];
+    kg[(int64_t)r * 16 + c16] = src >= 0 ? K[(int64_t)src * 16 + c16] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+int launch_bank_order_gather(const void* K, const int32_t* bank_idx, const float* bank_val, int ng, int bank_size,
+                             int32_t* map, void* Kg, cudaStream_t stream) {
+  const NvtxRange nvtx("dsa.bank_order_gather");
+  if (bank_size > kOrderMaxBank) return DSA_ERR_UNSUPPORTED;
+  if (ng == 0) return DSA_OK;
+  bank_order_gather_kernel<<<ng, kOrderThreads, 0, stream>>>(static_cast<const uint4*>(K), bank_idx, bank_val,
+                                                             bank_size, map, static_cast<uint4*>(Kg));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size, void* Kg,
                        cudaStream_t stream, const int64_t* row_off, const int* ok) {
   const NvtxRange nvtx("dsa.bank_gather");

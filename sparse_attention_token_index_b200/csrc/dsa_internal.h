@@ -165,6 +165,10 @@ int launch_proxy_mean(const void* Q, const float* w, int T, int H, int d, int G,
 // row_off (decode): bank indices are local to sequence g, whose rows start at row_off[g].
 int launch_bank_gather(const void* K, int k_dtype, int d, const int32_t* bank, int ng, int bank_size,
                        void* Kg, cudaStream_t stream, const int64_t* row_off = nullptr, const int* ok = nullptr);
+// Refine (prefill, bf16 keys with d = 128, bank_size <= 8192): map = the bank
+// ordered by the proxy's score bin, highest first; Kg the matching key rows.
+int launch_bank_order_gather(const void* K, const int32_t* bank_idx, const float* bank_val, int ng, int bank_size,
+                             int32_t* map, void* Kg, cudaStream_t stream);
 int launch_local_extend(const int32_t* bank, int ng, int B, int G, int T, int64_t q_pos0, const int32_t* q_off,
                         const int64_t* k_off, int S, int32_t* map, cudaStream_t stream, const int* ok = nullptr);
 // q_off / k_off (decode): group g is sequence g with members q_off[g] ..
