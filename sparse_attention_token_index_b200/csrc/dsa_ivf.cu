@@ -67,6 +67,92 @@ __global__ void ivf_assign_kernel(const __nv_bfloat16* __restrict__ K, const flo
   if (lane == 0) assign[r] = bi;
 }
 
+// The same assignment as a tiled product: a block takes 64 keys against the
+// centroids 64 at a time, d in chunks of 32 staged in shared memory, each
+// thread 4 keys x 4 centroids; the nearest centroid (lowest index among
+// equals) is kept per key across tiles and then across the 16 threads that
+// share a key.  d must be a multiple of 32.
+constexpr int kAsgKeys = 64, kAsgCen = 64, kAsgD = 32;
+
+__global__ void __launch_bounds__(256) ivf_assign_tiled_kernel(const __nv_bfloat16* __restrict__ K,
+                                                               const float* __restrict__ ks, int64_t N, int d,
+                                                               const float* __restrict__ cen,
+                                                               const float* __restrict__ norm, int C,
+                                                               int32_t* __restrict__ assign) {
+  // chunks stored transposed; rows padded by 4 floats (16-byte reads stay
+  // aligned, the transposing stores spread over 8 banks instead of one)
+  __shared__ __align__(16) float As[kAsgD][kAsgKeys + 4];
+  __shared__ __align__(16) float Bs[kAsgD][kAsgCen + 4];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int64_t r0 = (int64_t)blockIdx.x * kAsgKeys;
+  float best[4];
+  int bi[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    best[i] = __int_as_float(0x7f800000);
+    bi[i] = 0x7fffffff;
+  }
+  for (int c0 = 0; c0 < C; c0 += kAsgCen) {
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int l = 0; l < 4; ++l) acc[i][l] = 0.f;
+    for (int j0 = 0; j0 < d; j0 += kAsgD) {
+      for (int e = tid; e < kAsgKeys * kAsgD; e += 256) {
+        const int r = e / kAsgD, j = e % kAsgD;
+        const int64_t row = r0 + r;
+        As[j][r] = row < N ? key_elem(K, ks, row, d, j0 + j) : 0.f;
+      }
+      for (int e = tid; e < kAsgCen * kAsgD; e += 256) {
+        const int c = e / kAsgD, j = e % kAsgD;
+        Bs[j][c] = c0 + c < C ? cen[(int64_t)(c0 + c) * d + j0 + j] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int j = 0; j < kAsgD; ++j) {
+        const float4 a = *reinterpret_cast<const float4*>(&As[j][ty * 4]);
+        const float4 b = *reinterpret_cast<const float4*>(&Bs[j][tx * 4]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int l = 0; l < 4; ++l) acc[i][l] = fmaf(av[i], bv[l], acc[i][l]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+      const int c = c0 + tx * 4 + l;
+      if (c < C) {
+        const float nc = norm[c];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float dist = nc - 2.f * acc[i][l];
+          if (dist < best[i]) {  // centroids arrive in increasing order: the first minimum stays
+            best[i] = dist;
+            bi[i] = c;
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best[i], o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi[i], o);
+      if (ob < best[i] || (ob == best[i] && oi < bi[i])) {
+        best[i] = ob;
+        bi[i] = oi;
+      }
+    }
+    const int64_t row = r0 + ty * 4 + i;
+    if (tx == 0 && row < N) assign[row] = bi[i];
+  }
+}
+
 __global__ void ivf_accumulate_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ ks, int64_t N,
                                       int d, const int32_t* __restrict__ assign, float* __restrict__ sum,
                                       int32_t* __restrict__ count) {
@@ -176,7 +262,11 @@ int ivf_build(const void* K, const float* K_scale, int64_t N, int d, int C, int 
   ivf_init_kernel<<<C, 128, 0, st>>>(Kb, K_scale, N, d, C, x.cen);
   for (int it = 0; it < iters; ++it) {
     ivf_norm_kernel<<<(C + 7) / 8, 256, 0, st>>>(x.cen, C, d, norm);
-    ivf_assign_kernel<<<key_blocks, 256, 0, st>>>(Kb, K_scale, N, d, x.cen, norm, C, x.assign);
+    if (d % kAsgD == 0)
+      ivf_assign_tiled_kernel<<<(unsigned)((N + kAsgKeys - 1) / kAsgKeys), 256, 0, st>>>(Kb, K_scale, N, d, x.cen,
+                                                                                          norm, C, x.assign);
+    else
+      ivf_assign_kernel<<<key_blocks, 256, 0, st>>>(Kb, K_scale, N, d, x.cen, norm, C, x.assign);
     if (cudaMemsetAsync(sum, 0, (size_t)C * d * 4 + (size_t)C * 4, st) != cudaSuccess) return DSA_ERR_CUDA;
     ivf_accumulate_kernel<<<key_blocks, 256, 0, st>>>(Kb, K_scale, N, d, x.assign, sum, count);
     ivf_update_kernel<<<C, 128, 0, st>>>(sum, count, C, d, x.cen, it + 1 == iters ? (__nv_bfloat16*)x.cen_bf16 : nullptr);
