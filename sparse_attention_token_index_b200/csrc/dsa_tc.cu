@@ -282,17 +282,20 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ float relu_x2(float x) { return x + fabsf(x); }
 
 // acc += (w[h] / 2) * 2 ReLU(v[h]) over 32 heads (w2 points at those heads'
-// halved weights, four per 16-byte load), four packed accumulators.  Scaling
-// by 1/2 and 2 is exact, so each fma sees the product w[h] * ReLU(v[h]).
+// halved weights, four per 16-byte load) into one packed accumulator: even
+// heads in one lane, odd heads in the other.  Scaling by 1/2 and 2 is exact,
+// so each fma sees the product w[h] * ReLU(v[h]).  One serial chain is
+// enough: the ReLU adds and the other warps fill its latency, and the
+// registers it leaves free beat the parallel chains measurably.
 __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
-                                                  uint64_t (&acc)[4]) {
+                                                  uint64_t& acc) {
 #pragma unroll
   for (int h = 0; h < 32; h += 8) {
     const ulonglong2 wa = w2[h >> 2], wb = w2[(h >> 2) + 1];
-    acc[0] = ffma2(wa.x, pack2(relu_x2(v[h + 0]), relu_x2(v[h + 1])), acc[0]);
-    acc[1] = ffma2(wa.y, pack2(relu_x2(v[h + 2]), relu_x2(v[h + 3])), acc[1]);
-    acc[2] = ffma2(wb.x, pack2(relu_x2(v[h + 4]), relu_x2(v[h + 5])), acc[2]);
-    acc[3] = ffma2(wb.y, pack2(relu_x2(v[h + 6]), relu_x2(v[h + 7])), acc[3]);
+    acc = ffma2(wa.x, pack2(relu_x2(v[h + 0]), relu_x2(v[h + 1])), acc);
+    acc = ffma2(wa.y, pack2(relu_x2(v[h + 2]), relu_x2(v[h + 3])), acc);
+    acc = ffma2(wb.x, pack2(relu_x2(v[h + 4]), relu_x2(v[h + 5])), acc);
+    acc = ffma2(wb.y, pack2(relu_x2(v[h + 6]), relu_x2(v[h + 7])), acc);
   }
 }
 
@@ -534,7 +537,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         const bool mine = active && (jt & (team - 1)) == member;
         const float thr = row_threshold(st);  // read early: its latency hides behind the tile's loads
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // +0.0f pairs
+        uint64_t acc = 0ull;  // a +0.0f pair
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
         if (mine) {
           float v[32];
@@ -572,8 +575,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else if (kmap != nullptr) {
             kpos = in_range ? kmap[key] : -1;
           }
-          const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
-          float score = ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+          const float2 a0 = unpack2(acc);
+          float score = a0.x + a0.y;
           if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && (unsigned)kpos < n_vis;
