@@ -26,6 +26,7 @@
 // comparators (one query against its routed key blocks, or against its
 // probed clusters in the clustered keys).
 #include <atomic>
+#include <type_traits>
 
 #include "dsa_common.cuh"
 #include "dsa_topk.cuh"
@@ -285,8 +286,8 @@ __device__ __forceinline__ float relu_x2(float x) { return x + fabsf(x); }
 // halved weights, four per 16-byte load) into one packed accumulator: even
 // heads in one lane, odd heads in the other.  Scaling by 1/2 and 2 is exact,
 // so each fma sees the product w[h] * ReLU(v[h]).  One serial chain is
-// enough: the ReLU adds and the other warps fill its latency, and the
-// registers it leaves free beat the parallel chains measurably.
+// enough for unscaled keys: the ReLU adds and the other warps fill its
+// latency, and the registers it leaves free beat parallel chains.
 __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
                                                   uint64_t& acc) {
 #pragma unroll
@@ -299,7 +300,34 @@ __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ul
   }
 }
 
-template <bool kDebug, int kKind>
+// The same sum in four packed accumulators (four independent chains).  The
+// scaled-key kernels (fp8 keys, a per-key scale load after the sum) measured
+// faster this way.
+__device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
+                                                  uint64_t (&acc)[4]) {
+#pragma unroll
+  for (int h = 0; h < 32; h += 8) {
+    const ulonglong2 wa = w2[h >> 2], wb = w2[(h >> 2) + 1];
+    acc[0] = ffma2(wa.x, pack2(relu_x2(v[h + 0]), relu_x2(v[h + 1])), acc[0]);
+    acc[1] = ffma2(wa.y, pack2(relu_x2(v[h + 2]), relu_x2(v[h + 3])), acc[1]);
+    acc[2] = ffma2(wb.x, pack2(relu_x2(v[h + 4]), relu_x2(v[h + 5])), acc[2]);
+    acc[3] = ffma2(wb.y, pack2(relu_x2(v[h + 6]), relu_x2(v[h + 7])), acc[3]);
+  }
+}
+
+// Score pairs of the accumulators, summed.
+__device__ __forceinline__ float acc_sum(uint64_t acc) {
+  const float2 a0 = unpack2(acc);
+  return a0.x + a0.y;
+}
+__device__ __forceinline__ float acc_sum(const uint64_t (&acc)[4]) {
+  const float2 a0 = unpack2(acc[0]), a1 = unpack2(acc[1]), a2 = unpack2(acc[2]), a3 = unpack2(acc[3]);
+  return ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y));
+}
+
+// kScaled: the keys carry a per-key scale (fp8 keys); the scale pointer is
+// then non-null and applied after the head sum.
+template <bool kDebug, int kKind, bool kScaled>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_index_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ TcArgs a) {
@@ -511,7 +539,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // fp8 keys: score = scale[key] * sum_h w ReLU(q . k8), scale > 0; decode
       // groups index the scales of their own sequence
       const float* kscale =
-          (kKind == 2 && a.k_scale != nullptr && a.k_off != nullptr) ? a.k_scale + a.k_off[u.seq_split] : a.k_scale;
+          !kScaled ? nullptr : ((kKind == 2 && a.k_off != nullptr) ? a.k_scale + a.k_off[u.seq_split] : a.k_scale);
       const int u_key_row0 = u.key_row0;
       if (active) {
         if (ttid == 0) tb_retire(st);
@@ -537,7 +565,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         const bool mine = active && (jt & (team - 1)) == member;
         const float thr = row_threshold(st);  // read early: its latency hides behind the tile's loads
-        uint64_t acc = 0ull;  // a +0.0f pair
+        // +0.0f pairs
+        std::conditional_t<kScaled, uint64_t[4], uint64_t> acc{};
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
         if (mine) {
           float v[32];
@@ -575,9 +604,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else if (kmap != nullptr) {
             kpos = in_range ? kmap[key] : -1;
           }
-          const float2 a0 = unpack2(acc);
-          float score = a0.x + a0.y;
-          if (kscale != nullptr && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
+          float score = acc_sum(acc);
+          if (kScaled && in_range) score *= kscale[kKind == 1 ? (int64_t)u_key_row0 + key : kpos];
           score = score + 0.0f;  // -0 -> +0
           const bool valid = in_range && (unsigned)kpos < n_vis;
           if (kDebug && valid) a.dbg_scores[row * a.dbg_ld + kpos] = score;
@@ -655,7 +683,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem_base, 512);
 }
 
-template <bool kDebug, int kKind>
+template <bool kDebug, int kKind, bool kScaled>
 static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs& a, int grid, cudaStream_t stream) {
   // the shared-memory opt-in is a per-device function attribute: set it once
   // on each device the kernel runs on
@@ -664,12 +692,12 @@ static int launch_tc(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArg
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
   const uint64_t bit = uint64_t(1) << dev;
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    if (cudaFuncSetAttribute(tc_index_kernel<kDebug, kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc_index_kernel<kDebug, kKind, kScaled>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kTcSmemBytes) != cudaSuccess)
       return DSA_ERR_CUDA;
     configured.fetch_or(bit, std::memory_order_release);
   }
-  tc_index_kernel<kDebug, kKind><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
+  tc_index_kernel<kDebug, kKind, kScaled><<<grid, kTcThreads, kTcSmemBytes, stream>>>(tmQ, tmK, a);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -695,18 +723,19 @@ int launch_tc_index(const CUtensorMap& tmQ, const CUtensorMap& tmK, const TcArgs
   const TimerSlot ts = timer_acquire();
   if (ts.start) cudaEventRecord(ts.start, stream);
   int r;
+  const bool sc = a.k_scale != nullptr;
   if (a.dbg_scores != nullptr)
-    r = launch_tc<true, 0>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<true, 0, true>(tmQ, tmK, a, grid, stream) : launch_tc<true, 0, false>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 0)
-    r = launch_tc<false, 0>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<false, 0, true>(tmQ, tmK, a, grid, stream) : launch_tc<false, 0, false>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 1)
-    r = launch_tc<false, 1>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<false, 1, true>(tmQ, tmK, a, grid, stream) : launch_tc<false, 1, false>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 2)
-    r = launch_tc<false, 2>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<false, 2, true>(tmQ, tmK, a, grid, stream) : launch_tc<false, 2, false>(tmQ, tmK, a, grid, stream);
   else if (a.kind == 3)
-    r = launch_tc<false, 3>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<false, 3, true>(tmQ, tmK, a, grid, stream) : launch_tc<false, 3, false>(tmQ, tmK, a, grid, stream);
   else
-    r = launch_tc<false, 4>(tmQ, tmK, a, grid, stream);
+    r = sc ? launch_tc<false, 4, true>(tmQ, tmK, a, grid, stream) : launch_tc<false, 4, false>(tmQ, tmK, a, grid, stream);
   if (ts.end) cudaEventRecord(ts.end, stream);
   return r;
 }
