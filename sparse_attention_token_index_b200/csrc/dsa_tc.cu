@@ -24,7 +24,8 @@
 // group-refine blocks (up to 4 members of a group against the group's
 // gathered candidate bank), and the refine stages of the two routing
 // comparators (one query against its routed key blocks, or against its
-// probed clusters in the clustered keys).
+// probed clusters in the clustered keys).  A second template parameter marks
+// scaled keys (fp8 keys widened to bf16, a per-key scale after the head sum).
 #include <atomic>
 #include <type_traits>
 
