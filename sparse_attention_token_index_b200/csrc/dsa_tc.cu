@@ -283,16 +283,16 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 // use.  Exact: 2x for x > 0 (doubling is exact), +0 otherwise.
 __device__ __forceinline__ float relu_x2(float x) { return x + fabsf(x); }
 
-// acc += (w[h] / 2) * 2 ReLU(v[h]) over 32 heads (w2 points at those heads'
+// acc += (w[h] / 2) * 2 ReLU(v[h]) over 16 heads (w2 points at those heads'
 // halved weights, four per 16-byte load) into one packed accumulator: even
 // heads in one lane, odd heads in the other.  Scaling by 1/2 and 2 is exact,
 // so each fma sees the product w[h] * ReLU(v[h]).  One serial chain is
 // enough for unscaled keys: the ReLU adds and the other warps fill its
 // latency, and the registers it leaves free beat parallel chains.
-__device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
+__device__ __forceinline__ void head_accumulate16(const float (&v)[16], const ulonglong2* __restrict__ w2,
                                                   uint64_t& acc) {
 #pragma unroll
-  for (int h = 0; h < 32; h += 8) {
+  for (int h = 0; h < 16; h += 8) {
     const ulonglong2 wa = w2[h >> 2], wb = w2[(h >> 2) + 1];
     acc = ffma2(wa.x, pack2(relu_x2(v[h + 0]), relu_x2(v[h + 1])), acc);
     acc = ffma2(wa.y, pack2(relu_x2(v[h + 2]), relu_x2(v[h + 3])), acc);
@@ -301,9 +301,9 @@ __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ul
   }
 }
 
-// The same sum in four packed accumulators (four independent chains).  The
-// scaled-key kernels (fp8 keys, a per-key scale load after the sum) measured
-// faster this way.
+// The sum over 32 heads in four packed accumulators (four independent
+// chains).  The scaled-key kernels (fp8 keys, a per-key scale load after the
+// sum) measured faster this way.
 __device__ __forceinline__ void head_accumulate32(const float (&v)[32], const ulonglong2* __restrict__ w2,
                                                   uint64_t (&acc)[4]) {
 #pragma unroll
@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (ttid == 0) tb_retire(st);
         named_bar(tbar, tthr);
         row_reset(st, ttid, tthr);
-        if (ttid < kHeads) S.w[q][ttid] = 0.5f * a.w[row * kHeads + ttid];  // halved: see head_accumulate32
+        if (ttid < kHeads) S.w[q][ttid] = 0.5f * a.w[row * kHeads + ttid];  // halved: see head_accumulate16
         named_bar(tbar, tthr);
         if (ttid == 0) tb_open(st);
       }
@@ -570,16 +570,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         std::conditional_t<kScaled, uint64_t[4], uint64_t> acc{};
         const uint32_t col = tmem_base + lane_base + (uint32_t)(buf * 256 + q * kHeads);
         if (mine) {
-          float v[32];
-          tmem_ld_32x32b_x32(col, v);
-          tmem_ld_wait();
-          head_accumulate32(v, w2, acc);
-          tmem_ld_32x32b_x32(col + 32, v);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.t_empty[buf]);
-          head_accumulate32(v, w2 + 8, acc);
+          if constexpr (!kScaled) {
+            // the row's 64 columns in four loads of 16, each consumed before
+            // the next: 16 registers for the row instead of 32
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float v[16];
+              tmem_ld_32x32b_x16(col + 16 * c, v);
+              tmem_ld_wait();
+              if (c == 3) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.t_empty[buf]);
+              }
+              head_accumulate16(v, w2 + 4 * c, acc);
+            }
+          } else {
+            float v[32];
+            tmem_ld_32x32b_x32(col, v);
+            tmem_ld_wait();
+            head_accumulate32(v, w2, acc);
+            tmem_ld_32x32b_x32(col + 32, v);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.t_empty[buf]);
+            head_accumulate32(v, w2 + 8, acc);
+          }
         } else {
           tc_fence_before();
           __syncwarp();
